@@ -1,0 +1,449 @@
+"""Benchmark: prefix-sliding decode tokens/s and KV GB/s at W=4096 on B200.
+
+One step = one pass of the hot path over one batch: append the new token of
+each of B=8 sequences to its ring (ring write, eviction, position bookkeeping)
+and run the decode attention for those 8 sequences (visible-range derivation,
+split-K streaming of the prefix and window rows, split merge).  Workload:
+16 query / 8 kv heads, head_dim 128, P=128, W=4096, bf16 with fp32
+accumulation, every sequence past t=65536 so the window is full
+(4224 visible rows, 138.4 MB of K/V read per step).  Steps rotate over 4
+disjoint batches of 8 sequences (553 MB of resident K/V, more than 4x L2), so
+every step streams from HBM.  The timed steps are replayed from one CUDA graph.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+Under torchrun each rank runs its own sequences (weak scaling, no collective on
+the data path); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "prefix-sliding decode tokens/s and KV GB/s (% of B200 HBM peak) at W=4096"
+UNIT = "tokens/s"
+
+B, HQ, HKV, D, P, W = 8, 16, 8, 128, 128, 4096
+ROT = 4                     # disjoint batches rotated through
+T_START = 65536             # decode positions start here (window full)
+SEED = 0
+
+
+def workload_config():
+    n_vis = P + W
+    return {"workload": f"decode B={B} Hq={HQ} Hkv={HKV} d={D} P={P} W={W} bf16, t>={T_START} "
+                        f"(window full, {n_vis} visible rows)",
+            "global_batch": B, "Hq": HQ, "Hkv": HKV, "head_dim": D, "P": P, "W": W,
+            "t_start": T_START, "visible_rows": n_vis,
+            "l2": f"inputs larger than L2: {ROT} disjoint batches of {B} sequences rotated "
+                  f"({ROT * kv_bytes_per_step() / 1e6:.0f} MB resident K/V)"}
+
+
+def kv_bytes_per_seq():
+    return HKV * (P + W) * D * 2 * 2          # K and V rows, bf16
+
+
+def kv_bytes_per_step():
+    return B * kv_bytes_per_seq()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return j["hbm_gbs"], "measured"
+    return 6650.0, "fallback"
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------ clocks --------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        self.proc.wait()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for nm, val in zip(names, r[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        busy = sorted(sm)[len(sm) // 2:] if sm else []
+        return {"sm_mhz": statistics.median(busy) if busy else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ------------------------------------------------------------ our arm -------
+class Workload:
+    """Sequences, their synthetic histories and per-step inputs on one GPU."""
+
+    def __init__(self, rank: int, steps_needed: int):
+        import torch
+
+        import synth
+        from prefix_sliding_window_ring_b200 import PS_BF16, Cache
+
+        self.torch = torch
+        self.S = B * ROT
+        self.seed = SEED + 1000 * rank
+        self.kscale = synth.chan_scale(self.seed, HKV, D)
+        self.cache = Cache(W, P, HKV, D, PS_BF16, self.S)
+        self.scale = 1.0 / math.sqrt(D)
+
+        def dev(a):
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+
+        self.dev = dev
+        for s in range(self.S):
+            kp = synth.rows(self.seed, synth.TID_K, s, HKV, 0, P, D, "bf16", self.kscale)
+            vp = synth.rows(self.seed, synth.TID_V, s, HKV, 0, P, D, "bf16")
+            self.cache.seq_reset(s, (s * 613) % W)
+            self.cache.prefill_prefix(s, dev(kp), dev(vp), P)
+            t0 = T_START + s  # staggered positions
+            kw = synth.rows(self.seed, synth.TID_K, s, HKV, t0 - W, W, D, "bf16", self.kscale)
+            vw = synth.rows(self.seed, synth.TID_V, s, HKV, t0 - W, W, D, "bf16")
+            self.cache.import_window(s, t0, dev(kw), dev(vw), W, (s * 613) % W)
+        torch.cuda.synchronize()
+        self.next_pos = [T_START + s for s in range(self.S)]
+        # per-step inputs: each batch group appends one token per sequence per visit
+        visits = (steps_needed + ROT - 1) // ROT + 1
+        self.kin, self.vin, self.qin = {}, {}, {}
+        for s in range(self.S):
+            p0 = self.next_pos[s]
+            self.kin[s] = synth.rows(self.seed, synth.TID_K, s, HKV, p0, visits, D, "bf16", self.kscale)
+            self.vin[s] = synth.rows(self.seed, synth.TID_V, s, HKV, p0, visits, D, "bf16")
+            self.qin[s] = synth.rows(self.seed, synth.TID_Q, s, HQ, p0, visits, D, "bf16")
+        # device pools [ROT][visits][B][H][D]
+        self.visits = visits
+        self.k_pool = [dev(np.stack([self.kin[r * B + b] for b in range(B)], axis=1)) for r in range(ROT)]
+        self.v_pool = [dev(np.stack([self.vin[r * B + b] for b in range(B)], axis=1)) for r in range(ROT)]
+        self.q_pool = [dev(np.stack([self.qin[r * B + b] for b in range(B)], axis=1)) for r in range(ROT)]
+        self.out = [torch.empty((B, HQ, D), dtype=torch.bfloat16, device="cuda") for _ in range(ROT)]
+        self.ws = self.cache.decode_workspace(B, HQ)
+        self.visit = [0] * ROT
+
+    def ids(self, r):
+        return list(range(r * B, (r + 1) * B))
+
+    def step(self, i, stream=None, host=None):
+        """One hot-path step on batch group i % ROT (append + decode)."""
+        r = i % ROT
+        v = self.visit[r]
+        ids = self.ids(r)
+        ts = [self.next_pos[s] for s in ids]
+        if host is None:
+            k, vv, q = self.k_pool[r][v], self.v_pool[r][v], self.q_pool[r][v]
+        else:
+            k, vv, q = host(r, v)
+        self.cache.append_kv(ids, k, vv, 1, stream)
+        self.cache.attend_decode(q, ids, ts, HQ, self.scale, self.out[r], self.ws, stream)
+        for s in ids:
+            self.next_pos[s] += 1
+        self.visit[r] += 1
+        return self.out[r]
+
+    def decode_only(self, i, stream=None):
+        r = i % ROT
+        ids = self.ids(r)
+        ts = [self.next_pos[s] - 1 for s in ids]
+        self.cache.attend_decode(self.q_pool[r][0], ids, ts, HQ, self.scale, self.out[r], self.ws,
+                                 stream)
+
+
+def time_graph(torch, fn, n):
+    """Capture n calls of fn(i) into one CUDA graph, replay it once, return ms per call."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for i in range(n):
+            fn(i, s)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):
+        e0.record(s)
+        g.replay()
+        e1.record(s)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    del g
+    return ms / n
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import torch.distributed as td
+        import datetime
+        td.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                              device_id=torch.device("cuda", local_rank))
+        dist = td
+
+    K, Wm = args.steps, args.warmup
+    total_steps = Wm + K + Wm + K + 4
+    wl = Workload(rank, total_steps)
+    # warm-up (eager), also loads every kernel
+    for i in range(Wm):
+        wl.step(i)
+    torch.cuda.synchronize()
+    assert wl.cache.device_error() == 0
+
+    # ---- timed region: K steps replayed from one CUDA graph ----
+    clocks = ClockSampler(local_rank) if rank == 0 else None
+    if clocks:
+        clocks.start()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    base = Wm
+    with torch.cuda.graph(g, stream=s):
+        for i in range(K):
+            wl.step(base + i, s)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):
+        e0.record(s)
+        g.replay()
+        e1.record(s)
+    torch.cuda.synchronize()
+    ms_total = e0.elapsed_time(e1)
+    del g
+    if dist:
+        t = torch.tensor([ms_total], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    clk = clocks.stop() if clocks else None
+    assert wl.cache.device_error() == 0
+    ms_step = ms_total / K
+    value = world * B * K / (ms_total / 1e3)
+
+    # ---- dominant kernel (decode) timed on its own stream, rotating batches ----
+    ms_dec = time_graph(torch, lambda i, st: wl.decode_only(i, st), max(K, 4 * ROT))
+    bytes_launch = kv_bytes_per_step()
+    achieved = bytes_launch / (ms_dec / 1e3) / 1e9
+    peak, peak_kind = load_peaks()
+
+    # ---- end to end through the public API with host buffers ----
+    def host_inputs(r, v):
+        return hk[r][v], hv[r][v], hq[r][v]
+    hk = [wl.k_pool[r].cpu().pin_memory() for r in range(ROT)]
+    hv = [wl.v_pool[r].cpu().pin_memory() for r in range(ROT)]
+    hq = [wl.q_pool[r].cpu().pin_memory() for r in range(ROT)]
+    hout = torch.empty((B, HQ, D), dtype=torch.bfloat16).pin_memory()
+    dk = torch.empty((B, HKV, D), dtype=torch.bfloat16, device="cuda")
+    dv, dq = torch.empty_like(dk), torch.empty((B, HQ, D), dtype=torch.bfloat16, device="cuda")
+
+    def e2e_step(i):
+        r = i % ROT
+        v = wl.visit[r]
+        dk.copy_(hk[r][v], non_blocking=True)
+        dv.copy_(hv[r][v], non_blocking=True)
+        dq.copy_(hq[r][v], non_blocking=True)
+        out = wl.step(i, host=lambda r_, v_: (dk, dv, dq))
+        hout.copy_(out, non_blocking=True)
+
+    base = Wm + K
+    for i in range(2):
+        e2e_step(base + i)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record()
+    for i in range(K):
+        e2e_step(base + 2 + i)
+    e1.record()
+    torch.cuda.synchronize()
+    ms_e2e = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([ms_e2e], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+    assert wl.cache.device_error() == 0
+    e2e_value = world * B * K / (ms_e2e / 1e3)
+    h2d = (B * HKV * D * 2) * 2 + B * HQ * D * 2
+    d2h = B * HQ * D * 2
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl.seed, wl.kscale, budget_s=args.cpu_seconds)
+
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": Wm, "ms_per_step": round(ms_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {**workload_config(), "parallelism": f"replicas x{world} (sequences sharded, no collective)"},
+        "kv_gbs": round(kv_bytes_per_step() / (ms_step / 1e3) / 1e9, 1),
+        "kv_frac_of_peak": round(kv_bytes_per_step() / (ms_step / 1e3) / 1e9 / peak, 4),
+        "roofline": {"bound": "hbm", "kernel": "ps::k_decode<bf16,128,2>",
+                     "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "peak_source": peak_kind,
+                     "bytes_per_launch": bytes_launch, "ms_per_launch": round(ms_dec, 5),
+                     "traffic": None},
+        "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": 2 * K,
+        "clocks": clk,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------ CPU oracle ----
+def oracle_problems(seed, kscale, nseq):
+    """The oracle's inputs for nseq sequences of the workload at t=T_START."""
+    import oracle
+    import synth
+    G = HQ // HKV
+    batch = oracle.Batch()
+    scale = 1.0 / math.sqrt(D)
+    for s in range(nseq):
+        t = T_START + s
+        lo = t - W + 1
+        hp = np.concatenate([np.arange(0, P), np.arange(lo, t + 1)]).astype(np.int64)
+        K = np.concatenate([
+            synth.to_f64(synth.rows(seed, synth.TID_K, s, HKV, 0, P, D, "bf16", kscale)),
+            synth.to_f64(synth.rows(seed, synth.TID_K, s, HKV, lo, t + 1 - lo, D, "bf16", kscale))])
+        V = np.concatenate([
+            synth.to_f64(synth.rows(seed, synth.TID_V, s, HKV, 0, P, D, "bf16")),
+            synth.to_f64(synth.rows(seed, synth.TID_V, s, HKV, lo, t + 1 - lo, D, "bf16"))])
+        q = synth.to_f64(synth.rows(seed, synth.TID_Q, s, HQ, t, 1, D, "bf16"))[0]
+        for g in range(HKV):
+            batch.add(P, W, t, scale, q[g * G:(g + 1) * G], hp, np.ascontiguousarray(K[:, g]),
+                      np.ascontiguousarray(V[:, g]))
+    return batch
+
+
+def cpu_baseline(seed, kscale, budget_s=15.0, nthreads=None):
+    """Time the oracle, as it stands, on this host's cores over a bounded sample:
+    repeated decodes of one batch of B sequences of the workload."""
+    import oracle
+    nthreads = nthreads or oracle.host_threads()
+    batch = oracle_problems(seed, kscale, B)
+    reps = 0
+    t0 = time.perf_counter()
+    while True:
+        batch.run(nthreads)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or reps >= 1000:
+            break
+    tok = reps * B
+    return {"value": round(tok / el, 2), "unit": UNIT, "cores": nthreads, "kind": "oracle",
+            "sample": f"{reps} repetitions of one {B}-sequence decode step at t={T_START} "
+                      f"(float64 masked attention, {reps * B} sequence-decodes, {el:.1f} s)"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    import synth
+    kscale = synth.chan_scale(SEED, HKV, D)
+    cpu = cpu_baseline(SEED, kscale, budget_s=args.cpu_seconds)
+    # K timed steps of the same workload, each step = one B-sequence decode by the oracle
+    import oracle
+    batch = oracle_problems(SEED, kscale, B)
+    for _ in range(max(0, min(args.warmup, 1))):
+        batch.run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        batch.run()
+    el = time.perf_counter() - t0
+    value = B * args.steps / el
+    line = {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {**workload_config(), "parallelism": "host threads"},
+            "cpu_baseline": {**cpu, "value": round(value, 2)},
+            "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,203 @@
+/*
+ * ps.h -- prefix-sliding attention over a ring-buffer KV cache (C ABI).
+ *
+ * What it computes.  A query at absolute position t attends to the pinned
+ * prefix [0, P_s) of its sequence plus the recent window
+ * [max(P_s, t-W+1), t], and to nothing else ("Prefix Sliding" digest,
+ * longzhangge.com PaperDaily, section 03; stated there 1-indexed as
+ * [1,P] and [max(P+1, t-W+1), t]).  Each sequence's ring buffer holds exactly
+ * the last W window entries of its history, slot i of the logical view holding
+ * position base+i ("Formal verification of a sliding-window KV cache in
+ * Lean4", pnsm.cn blog, sections 2.3-2.4 and 3.2-3.4).  Positions are absolute
+ * and keep growing (the digest's section 05 "continue PE"); keys arrive
+ * already position-encoded and are never re-encoded.
+ *
+ * Conventions for every call.
+ *  - Tensor arguments are DEVICE pointers owned by the caller, contiguous,
+ *    of the cache's element type (PS_F32: float, PS_BF16: bfloat16 bit
+ *    patterns), 16-byte aligned.  Index and bookkeeping arguments marked
+ *    "host" are host pointers read before the call returns.
+ *  - Layouts are token-major: keys/values [tokens][Hkv][d], queries and
+ *    outputs [tokens][Hq][d].  Query head h uses key/value head h / (Hq/Hkv).
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and is asynchronous unless stated otherwise.  Calls that touch
+ *    the same cache must be ordered on one stream (or by the caller's events).
+ *  - Every argument, sequence state and position is validated on the host
+ *    BEFORE anything is enqueued.  A call that returns an error has changed
+ *    neither the device memory nor the host-side state; the message is
+ *    available from ps_last_error() in the calling thread.
+ *  - The library owns only the opaque host object.  All device storage lives
+ *    in the caller's buffer passed to ps_cache_create; decode scratch lives in
+ *    the caller's workspace passed to ps_attend_decode.
+ *  - Kernels never trap.  An internal inconsistency detected on the device sets
+ *    an error word that ps_device_error() reads back.
+ */
+#ifndef PS_H
+#define PS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PS_API __attribute__((visibility("default")))
+#else
+#define PS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PS_OK = 0,
+  PS_EINVAL = -1,      /* bad argument (size, pointer, alignment, duplicate id) */
+  PS_ENOMEM = -2,      /* caller's buffer or workspace too small */
+  PS_EPOS = -3,        /* position does not follow the sequence's history */
+  PS_ESTATE = -4,      /* sequence not in a state that allows the call */
+  PS_ECUDA = -5,       /* a CUDA runtime call failed (message has the details) */
+  PS_EUNSUPPORTED = -6 /* valid but unsupported configuration (e.g. head_dim) */
+} ps_status;
+
+typedef enum { PS_F32 = 0, PS_BF16 = 1 } ps_dtype;
+
+typedef struct ps_cache ps_cache; /* opaque, library-owned host object */
+
+/* Host-side view of one sequence (mirrors the device bookkeeping). */
+typedef struct {
+  int32_t state;     /* 0 = empty (after create/reset), 1 = active (prefix stored) */
+  int32_t P;         /* pinned prefix length P_s */
+  int64_t next_pos;  /* absolute position the next appended token gets */
+  int32_t head;      /* ring slot of the oldest window entry */
+  int32_t count;     /* window entries held, min(W, next_pos - P) */
+} ps_seq_info;
+
+/* ----------------------------------------------------------------- cache -- */
+
+/* Bytes of device memory a cache with these parameters needs (0 if invalid).
+ * W >= 1 window slots, P_max >= 0 prefix rows, Hkv >= 1 key/value heads,
+ * d in {64, 128}, dtype a ps_dtype, max_seqs >= 1 sequences. */
+PS_API size_t ps_cache_bytes(int W, int P_max, int Hkv, int d, int dtype, int max_seqs);
+
+/* Bind a cache to the caller's device buffer `dev_buf` (dev_bytes >=
+ * ps_cache_bytes(...), 256-byte aligned, owned by the caller and kept alive
+ * until ps_cache_destroy).  Every sequence starts empty with ring head 0.
+ * Enqueues the initialisation of the bookkeeping area on `stream`.
+ * Errors: PS_EINVAL, PS_EUNSUPPORTED, PS_ENOMEM, PS_ECUDA. */
+PS_API int ps_cache_create(int W, int P_max, int Hkv, int d, int dtype, int max_seqs,
+                    void* dev_buf, size_t dev_bytes, void* stream, ps_cache** out);
+
+/* Free the host object (the device buffer stays the caller's). NULL is a no-op. */
+PS_API void ps_cache_destroy(ps_cache* c);
+
+/* Return sequence `seq` to the empty state; its ring head starts at slot
+ * ring_head_offset (0 <= offset < W).  Results never depend on the offset.
+ * Errors: PS_EINVAL. */
+PS_API int ps_seq_reset(ps_cache* c, int seq, int ring_head_offset, void* stream);
+
+/* Host mirror of a sequence's state (no device access). Errors: PS_EINVAL. */
+PS_API int ps_seq_info_get(const ps_cache* c, int seq, ps_seq_info* out);
+
+/* ---------------------------------------------------------- a1 prefix ---- */
+
+/* Store the pinned prefix of an empty sequence: positions [0, P_s) with keys
+ * and values k, v [P_s][Hkv][d] (device).  The prefix is never evicted
+ * (digest section 03: KV_prefix = encode(prefix), kept for every step).
+ * 0 <= P_s <= P_max.  The sequence becomes active with next_pos = P_s and an
+ * empty window.  Errors: PS_EINVAL, PS_ESTATE (sequence not empty). */
+PS_API int ps_prefill_prefix(ps_cache* c, int seq, const void* k, const void* v, int P_s,
+                      void* stream);
+
+/* ---------------------------------------------------- a2 ring append ----- */
+
+/* Append n tokens to each of B active sequences seq_ids[0..B) (host array of
+ * distinct ids).  k, v: [B][n][Hkv][d] (device).  Token i of entry b gets
+ * position next_pos(b) + i.  Each token is one step of the cache update
+ * (blog section 3.3): while fewer than W entries are held it fills slot
+ * (head + count) mod W; afterwards it overwrites the oldest slot `head` and
+ * advances head.  n > W keeps only the last W tokens, exactly as n single
+ * steps would.  Positions are stored per slot.  B == 0 or n == 0 is a no-op.
+ * Errors: PS_EINVAL, PS_ESTATE. */
+PS_API int ps_append_kv(ps_cache* c, const int* seq_ids, int B, const void* k, const void* v,
+                 int n, void* stream);
+
+/* -------------------------------------------- a3-a5 decode attention ----- */
+
+/* Workspace bytes ps_attend_decode needs for a batch of B sequences with Hq
+ * query heads (an upper bound independent of the positions). */
+PS_API size_t ps_decode_workspace_bytes(const ps_cache* c, int B, int Hq);
+
+/* One decode step of attention for B active sequences seq_ids[0..B) (host,
+ * distinct) at positions t[0..B) (host), which must be the last appended
+ * position of each sequence (t[b] == next_pos - 1, t[b] >= P_s: append the
+ * token first, then attend, as the digest's section 03 loop does).
+ * q: [B][Hq][d] (device), out: [B][Hq][d] (device, same dtype).
+ * out[b][h] = sum over visible p of softmax_p(scale * <q[b][h], k_p>) v_p,
+ * computed in float32 (bf16 inputs are widened exactly; the bf16 output is
+ * rounded to nearest even).  Evicted positions are never read.
+ * workspace: device, >= ps_decode_workspace_bytes(c, B, Hq) bytes, zero-filled
+ * before its first use; every call leaves it ready for the next.  Calls that
+ * share a workspace must not overlap on the GPU.
+ * Hq must be a multiple of Hkv with Hq/Hkv in {1, 2, 4, 8}.
+ * Errors: PS_EINVAL, PS_ESTATE, PS_EPOS, PS_ENOMEM, PS_EUNSUPPORTED. */
+PS_API int ps_attend_decode(ps_cache* c, const void* q, const int* seq_ids, const int64_t* t,
+                     int B, int Hq, float scale, void* out, void* workspace,
+                     size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------- a6 chunked prefill/extend --- */
+
+/* Attention for a block of n consecutive queries of active sequence `seq` at
+ * positions [t0, t0+n), with t0 == next_pos (the block extends the history)
+ * and t0 >= P_s.  q: [n][Hq][d]; k_blk, v_blk: [n][Hkv][d], the block's own
+ * keys/values; out: [n][Hq][d] (all device).  Query t0+i sees the prefix, the
+ * ring entries in its window and block tokens t0..t0+i (causal inside the
+ * block).  The ring must still hold [max(P_s, t0-W+1), t0-1], which is always
+ * true before the block is appended.  If append_after != 0 the block is then
+ * appended as by ps_append_kv (only its last W tokens survive in the ring).
+ * bf16 with d = 128 and Hq/Hkv in {1, 2, 4, 8} runs on the tcgen05 tensor-core
+ * kernel; other configurations use a CUDA-core kernel.
+ * Errors: PS_EINVAL, PS_ESTATE, PS_EPOS, PS_EUNSUPPORTED. */
+PS_API int ps_attend_chunk(ps_cache* c, int seq, const void* q, const void* k_blk,
+                    const void* v_blk, int64_t t0, int n, int Hq, float scale, void* out,
+                    int append_after, void* stream);
+
+/* ------------------------------------------- checkpoint / debug export --- */
+
+/* Export the window of active sequence `seq` in logical order (oldest first,
+ * blog section 3.4 ringToList over the `count` held entries):
+ * k, v: [W][Hkv][d] (device; rows [0,count) written), pos: [W] int64 (device),
+ * count_out: one int32 (device).  Errors: PS_EINVAL, PS_ESTATE. */
+PS_API int ps_export_window(ps_cache* c, int seq, void* k, void* v, int64_t* pos,
+                     int32_t* count_out, void* stream);
+
+/* Set the window of active sequence `seq` as if positions [P_s, next_pos)
+ * had been appended: k, v: [n][Hkv][d] (device) hold positions
+ * [next_pos-n, next_pos) oldest first, n == min(W, next_pos - P_s), and the
+ * oldest lands in ring slot ring_head_offset (0 <= offset < W).
+ * Errors: PS_EINVAL, PS_ESTATE, PS_EPOS. */
+PS_API int ps_import_window(ps_cache* c, int seq, int64_t next_pos, const void* k, const void* v,
+                     int n, int ring_head_offset, void* stream);
+
+/* The positions the attention kernels read for a query of sequence `seq` at
+ * position t (t >= P_s), in the order they are visited: prefix rows, then the
+ * ring segments, then (for t >= next_pos, a chunk query) block positions
+ * next_pos..t.  Ring rows report the position stored in their slot.
+ * pos_out: device int64 with room for P_s + W entries; n_out: one int32
+ * (device).  Requires the ring to cover the window part below next_pos.
+ * Errors: PS_EINVAL, PS_ESTATE, PS_EPOS. */
+PS_API int ps_debug_visible(ps_cache* c, int seq, int64_t t, int64_t* pos_out, int32_t* n_out,
+                     void* stream);
+
+/* Synchronise `stream` and read (then clear) the device error word:
+ * *code = 0 when no kernel reported an inconsistency.  Errors: PS_ECUDA. */
+PS_API int ps_device_error(ps_cache* c, int32_t* code, void* stream);
+
+/* Message of the last failed call in this thread ("" if none). */
+PS_API const char* ps_last_error(void);
+
+/* Library version string. */
+PS_API const char* ps_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PS_H */

@@ -1,0 +1,429 @@
+// C ABI of the prefix-sliding ring-buffer attention library (see include/ps.h).
+//
+// Host side: argument validation, the host mirror of every sequence's
+// bookkeeping (used only to validate calls and size launches -- the kernels
+// read the device copy), and kernel launches.  Nothing is enqueued unless
+// every check passed, so a failed call leaves device memory and host state
+// untouched.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <string>
+#include <vector>
+
+#include "ps.h"
+#include "internal.h"
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+int ok() {
+  g_err.clear();
+  return PS_OK;
+}
+
+#define PS_CUDA(expr)                                                                   \
+  do {                                                                                  \
+    cudaError_t e_ = (expr);                                                            \
+    if (e_ != cudaSuccess) return fail(PS_ECUDA, "%s: %s", #expr, cudaGetErrorString(e_)); \
+  } while (0)
+
+struct SeqHost {
+  int32_t state;  // 0 empty, 1 active
+  int32_t P;
+  int64_t next_pos;
+  int32_t head;
+  int32_t count;
+};
+
+struct Layout {
+  size_t meta, tickets, err, pos, K, V, total;
+};
+
+size_t al(size_t x) { return (x + 255) & ~(size_t)255; }
+
+int esize_of(int dtype) { return dtype == PS_F32 ? 4 : (dtype == PS_BF16 ? 2 : 0); }
+
+bool make_layout(int W, int P_max, int Hkv, int d, int dtype, int S, Layout* L) {
+  int es = esize_of(dtype);
+  if (W < 1 || W > (1 << 28) || P_max < 0 || P_max > (1 << 28) || Hkv < 1 || Hkv > 1024 ||
+      S < 1 || S > (1 << 20) || es == 0)
+    return false;
+  if (d != 64 && d != 128) return false;
+  size_t off = 0;
+  L->meta = off; off += al((size_t)S * sizeof(ps::DevMeta));
+  L->tickets = off; off += al((size_t)S * sizeof(int32_t));
+  L->err = off; off += 256;
+  L->pos = off; off += al((size_t)S * W * sizeof(int64_t));
+  size_t slab = (size_t)S * Hkv * ((size_t)P_max + W) * d * es;
+  L->K = off; off += al(slab);
+  L->V = off; off += al(slab);
+  L->total = off;
+  return true;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
+
+}  // namespace
+
+struct ps_cache {
+  int W, P_max, Hkv, d, dtype, S, esize;
+  char* base;
+  size_t bytes;
+  int device;
+  int sm_count;
+  ps::CacheDev dev;
+  std::vector<SeqHost> seqs;
+};
+
+namespace {
+
+int check_device(const ps_cache* c) {
+  int cur = -1;
+  PS_CUDA(cudaGetDevice(&cur));
+  if (cur != c->device)
+    return fail(PS_EINVAL, "current device %d is not the cache's device %d", cur, c->device);
+  return PS_OK;
+}
+
+int check_seq(const ps_cache* c, int seq, bool need_active) {
+  if (seq < 0 || seq >= c->S) return fail(PS_EINVAL, "sequence %d out of range [0,%d)", seq, c->S);
+  if (need_active && c->seqs[seq].state != 1)
+    return fail(PS_ESTATE, "sequence %d has no stored prefix (call ps_prefill_prefix first)", seq);
+  return PS_OK;
+}
+
+int check_batch(const ps_cache* c, const int* ids, int B) {
+  if (B > 0 && !ids) return fail(PS_EINVAL, "seq_ids is NULL");
+  std::vector<char> seen(c->S, 0);
+  for (int b = 0; b < B; ++b) {
+    int r = check_seq(c, ids[b], true);
+    if (r) return r;
+    if (seen[ids[b]]) return fail(PS_EINVAL, "sequence %d appears twice in the batch", ids[b]);
+    seen[ids[b]] = 1;
+  }
+  return PS_OK;
+}
+
+int check_group(const ps_cache* c, int Hq, int* G) {
+  if (Hq < 1 || Hq % c->Hkv) return fail(PS_EINVAL, "Hq=%d is not a multiple of Hkv=%d", Hq, c->Hkv);
+  *G = Hq / c->Hkv;
+  if (*G != 1 && *G != 2 && *G != 4 && *G != 8)
+    return fail(PS_EUNSUPPORTED, "Hq/Hkv=%d not in {1,2,4,8}", *G);
+  return PS_OK;
+}
+
+void advance(SeqHost& s, int W, int64_t n) {
+  int64_t cn = (int64_t)s.count + n;
+  int64_t adv = cn - W > 0 ? cn - W : 0;
+  s.count = (int32_t)(cn < W ? cn : W);
+  s.head = (int32_t)(((int64_t)s.head + adv) % W);
+  s.next_pos += n;
+}
+
+ps::DevMeta to_dev(const SeqHost& s) {
+  ps::DevMeta m;
+  memset(&m, 0, sizeof(m));
+  m.next_pos = s.next_pos;
+  m.P = s.P;
+  m.head = s.head;
+  m.count = s.count;
+  return m;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ps_last_error(void) { return g_err.c_str(); }
+
+const char* ps_version(void) { return "prefix_sliding_window_ring_b200 0.1 (sm_100a)"; }
+
+size_t ps_cache_bytes(int W, int P_max, int Hkv, int d, int dtype, int max_seqs) {
+  Layout L;
+  if (!make_layout(W, P_max, Hkv, d, dtype, max_seqs, &L)) return 0;
+  return L.total;
+}
+
+int ps_cache_create(int W, int P_max, int Hkv, int d, int dtype, int max_seqs, void* dev_buf,
+                    size_t dev_bytes, void* stream, ps_cache** out) {
+  if (!out) return fail(PS_EINVAL, "out is NULL");
+  *out = nullptr;
+  if (d != 64 && d != 128) return fail(PS_EUNSUPPORTED, "head_dim %d not in {64,128}", d);
+  Layout L;
+  if (!make_layout(W, P_max, Hkv, d, dtype, max_seqs, &L))
+    return fail(PS_EINVAL, "invalid cache shape W=%d P_max=%d Hkv=%d d=%d dtype=%d seqs=%d", W,
+                P_max, Hkv, d, dtype, max_seqs);
+  if (!dev_buf || ((uintptr_t)dev_buf & 255))
+    return fail(PS_EINVAL, "dev_buf must be a non-NULL 256-byte aligned device pointer");
+  if (dev_bytes < L.total)
+    return fail(PS_ENOMEM, "dev_buf holds %zu bytes, the cache needs %zu", dev_bytes, L.total);
+  cudaPointerAttributes attr;
+  PS_CUDA(cudaPointerGetAttributes(&attr, dev_buf));
+  if (attr.type != cudaMemoryTypeDevice)
+    return fail(PS_EINVAL, "dev_buf is not device memory");
+  int sm = 0;
+  PS_CUDA(cudaDeviceGetAttribute(&sm, cudaDevAttrMultiProcessorCount, attr.device));
+  cudaStream_t st = (cudaStream_t)stream;
+  PS_CUDA(cudaMemsetAsync(dev_buf, 0, L.total, st));
+  ps_cache* c = new ps_cache();
+  c->W = W; c->P_max = P_max; c->Hkv = Hkv; c->d = d; c->dtype = dtype; c->S = max_seqs;
+  c->esize = esize_of(dtype);
+  c->base = (char*)dev_buf;
+  c->bytes = dev_bytes;
+  c->device = attr.device;
+  c->sm_count = sm;
+  c->dev.meta = (ps::DevMeta*)(c->base + L.meta);
+  c->dev.tickets = (int32_t*)(c->base + L.tickets);
+  c->dev.err = (int32_t*)(c->base + L.err);
+  c->dev.pos = (int64_t*)(c->base + L.pos);
+  c->dev.K = c->base + L.K;
+  c->dev.V = c->base + L.V;
+  c->dev.W = W; c->dev.P_max = P_max; c->dev.Hkv = Hkv; c->dev.d = d; c->dev.S = max_seqs;
+  c->dev.slab_rows = (int64_t)P_max + W;
+  c->seqs.assign(max_seqs, SeqHost{0, 0, 0, 0, 0});
+  *out = c;
+  return ok();
+}
+
+void ps_cache_destroy(ps_cache* c) { delete c; }
+
+int ps_seq_info_get(const ps_cache* c, int seq, ps_seq_info* out) {
+  if (!c || !out) return fail(PS_EINVAL, "NULL argument");
+  int r = check_seq(c, seq, false);
+  if (r) return r;
+  const SeqHost& s = c->seqs[seq];
+  out->state = s.state; out->P = s.P; out->next_pos = s.next_pos;
+  out->head = s.head; out->count = s.count;
+  return ok();
+}
+
+int ps_seq_reset(ps_cache* c, int seq, int ring_head_offset, void* stream) {
+  if (!c) return fail(PS_EINVAL, "cache is NULL");
+  int r = check_seq(c, seq, false);
+  if (r) return r;
+  if (ring_head_offset < 0 || ring_head_offset >= c->W)
+    return fail(PS_EINVAL, "ring_head_offset %d not in [0,%d)", ring_head_offset, c->W);
+  if ((r = check_device(c))) return r;
+  SeqHost s{0, 0, 0, ring_head_offset, 0};
+  PS_CUDA(ps::launch_meta_set(c->dev, seq, to_dev(s), (cudaStream_t)stream));
+  c->seqs[seq] = s;
+  return ok();
+}
+
+int ps_prefill_prefix(ps_cache* c, int seq, const void* k, const void* v, int P_s, void* stream) {
+  if (!c) return fail(PS_EINVAL, "cache is NULL");
+  int r = check_seq(c, seq, false);
+  if (r) return r;
+  if (c->seqs[seq].state != 0)
+    return fail(PS_ESTATE, "sequence %d already has a prefix (reset it first)", seq);
+  if (P_s < 0 || P_s > c->P_max) return fail(PS_EINVAL, "P_s=%d not in [0,%d]", P_s, c->P_max);
+  if (P_s > 0 && (!k || !v || !aligned16(k) || !aligned16(v)))
+    return fail(PS_EINVAL, "k/v must be non-NULL 16-byte aligned device pointers");
+  if ((r = check_device(c))) return r;
+  cudaStream_t st = (cudaStream_t)stream;
+  PS_CUDA(ps::launch_prefix_store(c->dev, c->esize, seq, k, v, P_s, st));
+  SeqHost s = c->seqs[seq];
+  s.state = 1; s.P = P_s; s.next_pos = P_s; s.count = 0;
+  PS_CUDA(ps::launch_meta_set(c->dev, seq, to_dev(s), st));
+  c->seqs[seq] = s;
+  return ok();
+}
+
+int ps_append_kv(ps_cache* c, const int* seq_ids, int B, const void* k, const void* v, int n,
+                 void* stream) {
+  if (!c) return fail(PS_EINVAL, "cache is NULL");
+  if (B < 0 || n < 0) return fail(PS_EINVAL, "negative B=%d or n=%d", B, n);
+  if (B == 0 || n == 0) return ok();
+  int r = check_batch(c, seq_ids, B);
+  if (r) return r;
+  if (!k || !v || !aligned16(k) || !aligned16(v))
+    return fail(PS_EINVAL, "k/v must be non-NULL 16-byte aligned device pointers");
+  if ((r = check_device(c))) return r;
+  cudaStream_t st = (cudaStream_t)stream;
+  size_t per_entry = (size_t)n * c->Hkv * c->d * c->esize;
+  for (int b0 = 0; b0 < B; b0 += ps::kMaxBatchPerLaunch) {
+    int nb = B - b0 < ps::kMaxBatchPerLaunch ? B - b0 : ps::kMaxBatchPerLaunch;
+    ps::BatchIds ids;
+    memset(&ids, 0, sizeof(ids));
+    for (int i = 0; i < nb; ++i) ids.seq[i] = seq_ids[b0 + i];
+    PS_CUDA(ps::launch_ring_append(c->dev, c->esize, ids, nb, (const char*)k + b0 * per_entry,
+                                   (const char*)v + b0 * per_entry, n, st));
+  }
+  for (int b = 0; b < B; ++b) advance(c->seqs[seq_ids[b]], c->W, n);
+  return ok();
+}
+
+size_t ps_decode_workspace_bytes(const ps_cache* c, int B, int Hq) {
+  if (!c || B < 0 || Hq < 1 || Hq % c->Hkv) return 0;
+  return ps::decode_workspace_bytes(B, Hq, c->Hkv, c->d, c->sm_count);
+}
+
+int ps_attend_decode(ps_cache* c, const void* q, const int* seq_ids, const int64_t* t, int B,
+                     int Hq, float scale, void* out, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+  if (!c) return fail(PS_EINVAL, "cache is NULL");
+  if (B < 0) return fail(PS_EINVAL, "negative B=%d", B);
+  int G = 0;
+  int r = check_group(c, Hq, &G);
+  if (r) return r;
+  if (B == 0) return ok();
+  if ((r = check_batch(c, seq_ids, B))) return r;
+  if (!t) return fail(PS_EINVAL, "t is NULL");
+  int n_max = 1;
+  for (int b = 0; b < B; ++b) {
+    const SeqHost& s = c->seqs[seq_ids[b]];
+    if (t[b] != s.next_pos - 1)
+      return fail(PS_EPOS, "sequence %d: t=%lld is not the last appended position %lld",
+                  seq_ids[b], (long long)t[b], (long long)(s.next_pos - 1));
+    if (t[b] < s.P)
+      return fail(PS_EPOS, "sequence %d: t=%lld lies inside the prefix (P=%d); append first",
+                  seq_ids[b], (long long)t[b], s.P);
+    int n = s.P + s.count;
+    if (n > n_max) n_max = n;
+  }
+  if (!q || !out || !aligned16(q) || !aligned16(out))
+    return fail(PS_EINVAL, "q/out must be non-NULL 16-byte aligned device pointers");
+  if (!workspace || ((uintptr_t)workspace & 255))
+    return fail(PS_EINVAL, "workspace must be a non-NULL 256-byte aligned device pointer");
+  ps::DecodePlan plan = ps::plan_decode(B, c->Hkv, n_max, c->sm_count);
+  size_t need = 0;
+  ps::DecodeWs ws = ps::decode_ws_layout(workspace, B, c->Hkv, G, c->d, plan.nsplit, &need);
+  if (need > workspace_bytes)
+    return fail(PS_ENOMEM, "workspace holds %zu bytes, this call needs %zu", workspace_bytes, need);
+  if ((r = check_device(c))) return r;
+  cudaStream_t st = (cudaStream_t)stream;
+  size_t per_entry = (size_t)Hq * c->d * c->esize;
+  for (int b0 = 0; b0 < B; b0 += ps::kMaxBatchPerLaunch) {
+    int nb = B - b0 < ps::kMaxBatchPerLaunch ? B - b0 : ps::kMaxBatchPerLaunch;
+    ps::BatchIds ids;
+    memset(&ids, 0, sizeof(ids));
+    for (int i = 0; i < nb; ++i) {
+      ids.seq[i] = seq_ids[b0 + i];
+      ids.t[i] = t[b0 + i];
+    }
+    PS_CUDA(ps::launch_decode(c->dev, c->dtype, G, ids, nb, b0, Hq,
+                              (const char*)q + b0 * per_entry, (char*)out + b0 * per_entry, scale,
+                              ws, plan, st));
+  }
+  return ok();
+}
+
+int ps_attend_chunk(ps_cache* c, int seq, const void* q, const void* k_blk, const void* v_blk,
+                    int64_t t0, int n, int Hq, float scale, void* out, int append_after,
+                    void* stream) {
+  if (!c) return fail(PS_EINVAL, "cache is NULL");
+  int r = check_seq(c, seq, true);
+  if (r) return r;
+  int G = 0;
+  if ((r = check_group(c, Hq, &G))) return r;
+  if (n < 0) return fail(PS_EINVAL, "negative n=%d", n);
+  const SeqHost& s = c->seqs[seq];
+  if (t0 != s.next_pos)
+    return fail(PS_EPOS, "t0=%lld does not follow the history (next position %lld)",
+                (long long)t0, (long long)s.next_pos);
+  if (t0 < s.P)
+    return fail(PS_EPOS, "t0=%lld lies inside the prefix (P=%d)", (long long)t0, s.P);
+  if (n == 0) return ok();
+  if (!q || !out || !k_blk || !v_blk || !aligned16(q) || !aligned16(out) || !aligned16(k_blk) ||
+      !aligned16(v_blk))
+    return fail(PS_EINVAL, "q/k_blk/v_blk/out must be non-NULL 16-byte aligned device pointers");
+  if ((r = check_device(c))) return r;
+  cudaStream_t st = (cudaStream_t)stream;
+  PS_CUDA(ps::launch_chunk_cc(c->dev, c->dtype, G, seq, t0, n, Hq, q, k_blk, v_blk, out, scale,
+                              st));
+  if (append_after) {
+    ps::BatchIds ids;
+    memset(&ids, 0, sizeof(ids));
+    ids.seq[0] = seq;
+    PS_CUDA(ps::launch_ring_append(c->dev, c->esize, ids, 1, k_blk, v_blk, n, st));
+    advance(c->seqs[seq], c->W, n);
+  }
+  return ok();
+}
+
+int ps_export_window(ps_cache* c, int seq, void* k, void* v, int64_t* pos, int32_t* count_out,
+                     void* stream) {
+  if (!c) return fail(PS_EINVAL, "cache is NULL");
+  int r = check_seq(c, seq, true);
+  if (r) return r;
+  if (!k || !v || !pos || !count_out || !aligned16(k) || !aligned16(v) || ((uintptr_t)pos & 7) ||
+      ((uintptr_t)count_out & 3))
+    return fail(PS_EINVAL, "k/v/pos/count_out must be non-NULL aligned device pointers");
+  if ((r = check_device(c))) return r;
+  PS_CUDA(ps::launch_ring_export(c->dev, c->esize, seq, k, v, pos, count_out,
+                                 (cudaStream_t)stream));
+  return ok();
+}
+
+int ps_import_window(ps_cache* c, int seq, int64_t next_pos, const void* k, const void* v, int n,
+                     int ring_head_offset, void* stream) {
+  if (!c) return fail(PS_EINVAL, "cache is NULL");
+  int r = check_seq(c, seq, true);
+  if (r) return r;
+  SeqHost s = c->seqs[seq];
+  if (next_pos < s.P)
+    return fail(PS_EPOS, "next_pos=%lld lies inside the prefix (P=%d)", (long long)next_pos, s.P);
+  int64_t want = next_pos - s.P < c->W ? next_pos - s.P : c->W;
+  if (n != want)
+    return fail(PS_EPOS, "n=%d rows given, the window of next_pos=%lld holds %lld", n,
+                (long long)next_pos, (long long)want);
+  if (ring_head_offset < 0 || ring_head_offset >= c->W)
+    return fail(PS_EINVAL, "ring_head_offset %d not in [0,%d)", ring_head_offset, c->W);
+  if (n > 0 && (!k || !v || !aligned16(k) || !aligned16(v)))
+    return fail(PS_EINVAL, "k/v must be non-NULL 16-byte aligned device pointers");
+  if ((r = check_device(c))) return r;
+  s.next_pos = next_pos;
+  s.head = ring_head_offset;
+  s.count = n;
+  PS_CUDA(ps::launch_ring_import(c->dev, c->esize, seq, to_dev(s), k, v, n,
+                                 (cudaStream_t)stream));
+  c->seqs[seq] = s;
+  return ok();
+}
+
+int ps_debug_visible(ps_cache* c, int seq, int64_t t, int64_t* pos_out, int32_t* n_out,
+                     void* stream) {
+  if (!c) return fail(PS_EINVAL, "cache is NULL");
+  int r = check_seq(c, seq, true);
+  if (r) return r;
+  const SeqHost& s = c->seqs[seq];
+  if (t < s.P) return fail(PS_EPOS, "t=%lld lies inside the prefix (P=%d)", (long long)t, s.P);
+  int64_t lo = t - c->W + 1 > s.P ? t - c->W + 1 : s.P;
+  int64_t base = s.next_pos - s.count;
+  if (lo < base && lo <= s.next_pos - 1)
+    return fail(PS_EPOS, "window of t=%lld starts at %lld, the ring holds from %lld",
+                (long long)t, (long long)lo, (long long)base);
+  if (!pos_out || !n_out || ((uintptr_t)pos_out & 7) || ((uintptr_t)n_out & 3))
+    return fail(PS_EINVAL, "pos_out/n_out must be non-NULL aligned device pointers");
+  if ((r = check_device(c))) return r;
+  PS_CUDA(ps::launch_debug_visible(c->dev, seq, t, pos_out, n_out, (cudaStream_t)stream));
+  return ok();
+}
+
+int ps_device_error(ps_cache* c, int32_t* code, void* stream) {
+  if (!c || !code) return fail(PS_EINVAL, "NULL argument");
+  int r = check_device(c);
+  if (r) return r;
+  cudaStream_t st = (cudaStream_t)stream;
+  PS_CUDA(cudaStreamSynchronize(st));
+  int32_t v = 0;
+  PS_CUDA(cudaMemcpy(&v, c->dev.err, sizeof(v), cudaMemcpyDeviceToHost));
+  PS_CUDA(cudaMemset(c->dev.err, 0, sizeof(int32_t)));
+  *code = v;
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,118 @@
+// Shared device-side definitions: cache layout, per-sequence bookkeeping and
+// the derivation of the visible row ranges (the part of the path that turns a
+// query position into the rows to stream, never addressing evicted rows).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ps {
+
+// Per-sequence bookkeeping kept in device memory (32 bytes).
+//   The ring holds positions [next_pos - count, next_pos); the oldest sits in
+//   slot `head`, position p in slot (head + (p - (next_pos - count))) mod W.
+//   P is the pinned prefix length; prefix row j holds position j.
+struct DevMeta {
+  int64_t next_pos;
+  int32_t P;
+  int32_t head;
+  int32_t count;
+  int32_t pad[3];
+};
+static_assert(sizeof(DevMeta) == 32, "DevMeta layout");
+
+// Device view of one cache, passed to kernels by value.
+//   K, V: [S][Hkv][P_max + W][d]; rows [0, P_max) of each (sequence, head)
+//   slab are the prefix store, rows [P_max, P_max + W) the ring slots.
+//   pos: [S][W] absolute position held by each ring slot.
+struct CacheDev {
+  DevMeta* meta;
+  int32_t* tickets;  // [S] completion counters of the ring writers (0 at rest)
+  int32_t* err;      // device error word (bit flags below)
+  int64_t* pos;
+  void* K;
+  void* V;
+  int32_t W, P_max, Hkv, d, S;
+  int64_t slab_rows;  // P_max + W
+};
+
+enum : int32_t {
+  ERR_COVERAGE = 1,  // a split-K launch did not cover every visible row
+  ERR_RING = 2,      // the ring does not hold the window a query needs
+  ERR_BATCH = 4,     // a batch entry's position disagrees with the bookkeeping
+};
+
+// Row ranges a query at position t reads, in visiting order (at most 4):
+//   src 0: prefix rows [0, P) of the slab;
+//   src 1: ring segment from slot s0 up to the physical end of the ring;
+//   src 1: ring segment wrapping around from slot 0;
+//   src 2: block rows (chunk queries): block row r holds position next_pos + r.
+// Visible set (digest section 03, 0-indexed): [0, P) and [max(P, t-W+1), t].
+struct SegSet {
+  int32_t n;
+  int32_t total;
+  int32_t len[4];
+  int64_t row0[4];  // first slab row (src 0/1) or first block row (src 2)
+  int32_t src[4];
+  int32_t ring_ok;  // 0 if the window part below next_pos is not held by the ring
+};
+
+__host__ __device__ inline SegSet build_segments(const DevMeta& m, int32_t W, int32_t P_max,
+                                                 int64_t t) {
+  SegSet s;
+  s.n = 0;
+  s.total = 0;
+  s.ring_ok = 1;
+  for (int i = 0; i < 4; ++i) { s.len[i] = 0; s.row0[i] = 0; s.src[i] = 0; }
+  if (m.P > 0) {
+    s.len[0] = m.P; s.row0[0] = 0; s.src[0] = 0; s.n = 1;
+  }
+  int64_t lo = t - (int64_t)W + 1;
+  if (lo < m.P) lo = m.P;
+  // ring part: positions [lo, min(t, next_pos - 1)]
+  int64_t hi = t < m.next_pos - 1 ? t : m.next_pos - 1;
+  int64_t base = m.next_pos - m.count;
+  if (hi >= lo) {
+    if (lo < base) {  // window reaches below what the ring holds
+      s.ring_ok = 0;
+      lo = base;
+    }
+    if (hi >= lo) {
+      int64_t nw = hi - lo + 1;
+      int64_t s0 = ((int64_t)m.head + (lo - base)) % W;
+      int64_t lenA = nw < (int64_t)W - s0 ? nw : (int64_t)W - s0;
+      s.len[s.n] = (int32_t)lenA; s.row0[s.n] = P_max + s0; s.src[s.n] = 1; s.n++;
+      if (nw > lenA) {
+        s.len[s.n] = (int32_t)(nw - lenA); s.row0[s.n] = P_max; s.src[s.n] = 1; s.n++;
+      }
+    }
+  }
+  // block part: positions [max(lo, next_pos), t]
+  int64_t blo = lo > m.next_pos ? lo : m.next_pos;
+  if (t >= blo) {
+    s.len[s.n] = (int32_t)(t - blo + 1); s.row0[s.n] = blo - m.next_pos; s.src[s.n] = 2; s.n++;
+  }
+  for (int i = 0; i < s.n; ++i) s.total += s.len[i];
+  return s;
+}
+
+// Segment index and offset of logical row j (0 <= j < total).
+__device__ __forceinline__ void seg_locate(const SegSet& s, int32_t j, int& si, int32_t& off) {
+  si = 0;
+  off = j;
+#pragma unroll
+  for (int i = 0; i < 3; ++i) {
+    if (si == i && i + 1 < s.n && off >= s.len[i]) { off -= s.len[i]; si = i + 1; }
+  }
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// float -> bfloat16 bits, round to nearest even (finite inputs).
+__device__ __forceinline__ uint16_t f2bf(float f) {
+  uint32_t u = __float_as_uint(f);
+  u += 0x7fffu + ((u >> 16) & 1u);
+  return (uint16_t)(u >> 16);
+}
+
+}  // namespace ps

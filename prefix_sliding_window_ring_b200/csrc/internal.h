@@ -1,0 +1,50 @@
+// Host-side declarations shared by the library's translation units.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace ps {
+
+constexpr int kMaxBatchPerLaunch = 256;  // batch entries passed by value per launch
+
+struct BatchIds {
+  int32_t seq[kMaxBatchPerLaunch];
+  int64_t t[kMaxBatchPerLaunch];
+};
+
+// ring.cu
+cudaError_t launch_meta_set(const CacheDev& c, int seq, const DevMeta& m, cudaStream_t st);
+cudaError_t launch_prefix_store(const CacheDev& c, int esize, int seq, const void* k,
+                                const void* v, int P_s, cudaStream_t st);
+cudaError_t launch_ring_append(const CacheDev& c, int esize, const BatchIds& ids, int B,
+                               const void* k, const void* v, int n, cudaStream_t st);
+cudaError_t launch_ring_import(const CacheDev& c, int esize, int seq, const DevMeta& m_new,
+                               const void* k, const void* v, int n, cudaStream_t st);
+cudaError_t launch_ring_export(const CacheDev& c, int esize, int seq, void* k, void* v,
+                               int64_t* pos, int32_t* count_out, cudaStream_t st);
+cudaError_t launch_debug_visible(const CacheDev& c, int seq, int64_t t, int64_t* pos_out,
+                                 int32_t* n_out, cudaStream_t st);
+
+// attend.cu (CUDA-core kernels)
+struct DecodePlan {
+  int nsplit;   // CTAs per (sequence, kv head)
+  int chunk;    // visible rows per CTA
+};
+DecodePlan plan_decode(int B, int Hkv, int n_max, int sm_count);
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int sm_count);
+struct DecodeWs {
+  int32_t* tick;    // [B][Hkv] arrival counters (0 at rest)
+  float* part_ml;   // [B][Hkv][nsplit][G][2] per-split (max, sum), base-2 domain
+  float* part_o;    // [B][Hkv][nsplit][G][d] per-split unnormalised accumulators
+};
+DecodeWs decode_ws_layout(void* ws, int B, int Hkv, int G, int d, int nsplit, size_t* bytes);
+cudaError_t launch_decode(const CacheDev& c, int dtype, int G, const BatchIds& ids, int B,
+                          int b_off, int Hq, const void* q, void* out, float scale,
+                          const DecodeWs& ws, const DecodePlan& plan, cudaStream_t st);
+cudaError_t launch_chunk_cc(const CacheDev& c, int dtype, int G, int seq, int64_t t0, int n,
+                            int Hq, const void* q, const void* k_blk, const void* v_blk,
+                            void* out, float scale, cudaStream_t st);
+
+}  // namespace ps

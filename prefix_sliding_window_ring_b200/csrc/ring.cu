@@ -1,0 +1,226 @@
+// Ring-buffer KV store: prefix store (a1), ring append with eviction and
+// position bookkeeping (a2), window import/export and the visible-row dump.
+//
+// Cache update rule ("Formal verification of a sliding-window KV cache in
+// Lean4", pnsm.cn blog, sections 3.3-3.4): a new entry fills slot
+// (head + count) mod W while fewer than W entries are held, otherwise it
+// overwrites the oldest slot `head` and head advances by one.  Over n tokens
+// that is count' = min(W, count + n), head' = head + max(0, count + n - W)
+// (mod W), and position p always lands in slot (head + p - base) mod W with
+// base = next_pos - count the oldest held position.
+#include "internal.h"
+
+namespace ps {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+__global__ void k_meta_set(DevMeta* meta, int seq, DevMeta m) { meta[seq] = m; }
+
+__device__ __forceinline__ size_t slab_row_off(const CacheDev& c, int s, int g, int64_t row,
+                                               int vpr) {
+  return (((size_t)s * c.Hkv + g) * (size_t)c.slab_rows + (size_t)row) * vpr;
+}
+
+// Prefix rows: input [P_s][Hkv][d] -> slab rows [0, P_s) of every head.
+__global__ void k_prefix_store(CacheDev c, int vpr, int seq, const uint4* __restrict__ k,
+                               const uint4* __restrict__ v, int P_s) {
+  uint4* K = (uint4*)c.K;
+  uint4* V = (uint4*)c.V;
+  int64_t total = (int64_t)P_s * c.Hkv * vpr;
+  for (int64_t x = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; x < total;
+       x += (int64_t)gridDim.x * blockDim.x) {
+    int vi = (int)(x % vpr);
+    int64_t r = x / vpr;
+    int g = (int)(r % c.Hkv);
+    int64_t j = r / c.Hkv;
+    size_t dst = slab_row_off(c, seq, g, j, vpr) + vi;
+    K[dst] = k[x];
+    V[dst] = v[x];
+  }
+}
+
+// Append n tokens to each batch entry (grid.y = batch entry).  Every CTA of an
+// entry reads the entry's bookkeeping before arriving on the entry's ticket;
+// the last CTA to arrive commits the new bookkeeping and re-arms the ticket.
+__global__ void k_ring_append(CacheDev c, int vpr, BatchIds ids, const uint4* __restrict__ k,
+                              const uint4* __restrict__ v, int n) {
+  const int b = blockIdx.y;
+  const int s = ids.seq[b];
+  const DevMeta m = c.meta[s];
+  const int64_t W = c.W;
+  const int64_t n_eff = n < W ? n : W;       // earlier tokens are overwritten in this call
+  const int64_t i0 = n - n_eff;
+  const int64_t base = m.next_pos - m.count;
+  uint4* K = (uint4*)c.K;
+  uint4* V = (uint4*)c.V;
+  const int64_t total = n_eff * c.Hkv * vpr;
+  for (int64_t x = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; x < total;
+       x += (int64_t)gridDim.x * blockDim.x) {
+    int vi = (int)(x % vpr);
+    int64_t r = x / vpr;
+    int g = (int)(r % c.Hkv);
+    int64_t i = i0 + r / c.Hkv;
+    int64_t p = m.next_pos + i;
+    int64_t slot = ((int64_t)m.head + (p - base)) % W;
+    size_t src = (((size_t)b * n + i) * c.Hkv + g) * vpr + vi;
+    size_t dst = slab_row_off(c, s, g, c.P_max + slot, vpr) + vi;
+    K[dst] = k[src];
+    V[dst] = v[src];
+    if (g == 0 && vi == 0) c.pos[(size_t)s * W + slot] = p;
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int old = atomicAdd(&c.tickets[s], 1);
+    if (old == (int)gridDim.x - 1) {
+      DevMeta nm = m;
+      int64_t cn = (int64_t)m.count + n;
+      nm.count = (int32_t)(cn < W ? cn : W);
+      int64_t adv = cn - W > 0 ? cn - W : 0;
+      nm.head = (int32_t)(((int64_t)m.head + adv) % W);
+      nm.next_pos = m.next_pos + n;
+      c.meta[s] = nm;
+      c.tickets[s] = 0;
+    }
+  }
+}
+
+// Import: rows i of [n][Hkv][d] hold positions next_pos - n + i, oldest at slot head.
+__global__ void k_ring_import(CacheDev c, int vpr, int seq, DevMeta mn,
+                              const uint4* __restrict__ k, const uint4* __restrict__ v, int n) {
+  uint4* K = (uint4*)c.K;
+  uint4* V = (uint4*)c.V;
+  const int64_t W = c.W;
+  const int64_t total = (int64_t)n * c.Hkv * vpr;
+  for (int64_t x = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; x < total;
+       x += (int64_t)gridDim.x * blockDim.x) {
+    int vi = (int)(x % vpr);
+    int64_t r = x / vpr;
+    int g = (int)(r % c.Hkv);
+    int64_t i = r / c.Hkv;
+    int64_t slot = ((int64_t)mn.head + i) % W;
+    size_t dst = slab_row_off(c, seq, g, c.P_max + slot, vpr) + vi;
+    K[dst] = k[x];
+    V[dst] = v[x];
+    if (g == 0 && vi == 0) c.pos[(size_t)seq * W + slot] = mn.next_pos - n + i;
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int old = atomicAdd(&c.tickets[seq], 1);
+    if (old == (int)gridDim.x - 1) {
+      c.meta[seq] = mn;
+      c.tickets[seq] = 0;
+    }
+  }
+}
+
+// Export the held window in logical order: entry i is slot (head + i) mod W.
+__global__ void k_ring_export(CacheDev c, int vpr, int seq, uint4* __restrict__ k,
+                              uint4* __restrict__ v, int64_t* __restrict__ pos,
+                              int32_t* __restrict__ count_out) {
+  const DevMeta m = c.meta[seq];
+  const uint4* K = (const uint4*)c.K;
+  const uint4* V = (const uint4*)c.V;
+  const int64_t total = (int64_t)m.count * c.Hkv * vpr;
+  for (int64_t x = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; x < total;
+       x += (int64_t)gridDim.x * blockDim.x) {
+    int vi = (int)(x % vpr);
+    int64_t r = x / vpr;
+    int g = (int)(r % c.Hkv);
+    int64_t i = r / c.Hkv;
+    int64_t slot = ((int64_t)m.head + i) % c.W;
+    size_t src = slab_row_off(c, seq, g, c.P_max + slot, vpr) + vi;
+    k[x] = K[src];
+    v[x] = V[src];
+    if (g == 0 && vi == 0) pos[i] = c.pos[(size_t)seq * c.W + slot];
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) *count_out = m.count;
+}
+
+// The rows the attention kernels visit for a query at t, as positions.
+__global__ void k_debug_visible(CacheDev c, int seq, int64_t t, int64_t* __restrict__ pos_out,
+                                int32_t* __restrict__ n_out) {
+  const DevMeta m = c.meta[seq];
+  const SegSet s = build_segments(m, c.W, c.P_max, t);
+  if (!s.ring_ok && threadIdx.x == 0) atomicOr(c.err, ERR_RING);
+  int32_t j0 = 0;
+  for (int i = 0; i < s.n; ++i) {
+    for (int32_t r = threadIdx.x; r < s.len[i]; r += blockDim.x) {
+      int64_t p;
+      if (s.src[i] == 0) {
+        p = s.row0[i] + r;  // prefix row j holds position j
+      } else if (s.src[i] == 1) {
+        int64_t slot = s.row0[i] - c.P_max + r;
+        p = c.pos[(size_t)seq * c.W + slot];
+      } else {
+        p = m.next_pos + s.row0[i] + r;
+      }
+      pos_out[j0 + r] = p;
+    }
+    j0 += s.len[i];
+  }
+  if (threadIdx.x == 0) *n_out = s.total;
+}
+
+int grid_for(int64_t work, int cap) {
+  int64_t g = (work + kThreads - 1) / kThreads;
+  if (g < 1) g = 1;
+  if (g > cap) g = cap;
+  return (int)g;
+}
+
+}  // namespace
+
+cudaError_t launch_meta_set(const CacheDev& c, int seq, const DevMeta& m, cudaStream_t st) {
+  k_meta_set<<<1, 1, 0, st>>>(c.meta, seq, m);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prefix_store(const CacheDev& c, int esize, int seq, const void* k,
+                                const void* v, int P_s, cudaStream_t st) {
+  int vpr = c.d * esize / 16;
+  int64_t work = (int64_t)P_s * c.Hkv * vpr;
+  if (work == 0) return cudaSuccess;
+  k_prefix_store<<<grid_for(work, 4096), kThreads, 0, st>>>(c, vpr, seq, (const uint4*)k,
+                                                            (const uint4*)v, P_s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ring_append(const CacheDev& c, int esize, const BatchIds& ids, int B,
+                               const void* k, const void* v, int n, cudaStream_t st) {
+  int vpr = c.d * esize / 16;
+  int64_t n_eff = n < c.W ? n : c.W;
+  int64_t work = n_eff * c.Hkv * vpr;
+  dim3 grid(grid_for(work, 256), B);
+  k_ring_append<<<grid, kThreads, 0, st>>>(c, vpr, ids, (const uint4*)k, (const uint4*)v, n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ring_import(const CacheDev& c, int esize, int seq, const DevMeta& m_new,
+                               const void* k, const void* v, int n, cudaStream_t st) {
+  int vpr = c.d * esize / 16;
+  int64_t work = (int64_t)n * c.Hkv * vpr;
+  k_ring_import<<<grid_for(work, 1024), kThreads, 0, st>>>(c, vpr, seq, m_new, (const uint4*)k,
+                                                           (const uint4*)v, n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ring_export(const CacheDev& c, int esize, int seq, void* k, void* v,
+                               int64_t* pos, int32_t* count_out, cudaStream_t st) {
+  int vpr = c.d * esize / 16;
+  int64_t work = (int64_t)c.W * c.Hkv * vpr;
+  k_ring_export<<<grid_for(work, 1024), kThreads, 0, st>>>(c, vpr, seq, (uint4*)k, (uint4*)v,
+                                                           pos, count_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_debug_visible(const CacheDev& c, int seq, int64_t t, int64_t* pos_out,
+                                 int32_t* n_out, cudaStream_t st) {
+  k_debug_visible<<<1, kThreads, 0, st>>>(c, seq, t, pos_out, n_out);
+  return cudaGetLastError();
+}
+
+}  // namespace ps

@@ -1,0 +1,64 @@
+"""The C-ABI library loads and exports every entry point include/ps.h declares;
+host-only calls and argument checks that run before any CUDA call (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"^PS_API\s+[\w\s\*]+?\b(ps_\w+)\s*\(", src, re.M)
+    return names
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_symbols())
+    for must in ["ps_cache_create", "ps_prefill_prefix", "ps_append_kv", "ps_attend_decode",
+                 "ps_attend_chunk", "ps_export_window", "ps_import_window", "ps_debug_visible"]:
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    from prefix_sliding_window_ring_b200 import abi
+    lib = ctypes.CDLL(abi.LIB_PATH)
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+        assert name in abi.SIGNATURES, f"binding lacks {name}"
+    assert set(abi.SIGNATURES) == set(declared_symbols())
+
+
+def test_cache_bytes_layout():
+    from prefix_sliding_window_ring_b200 import abi
+    n = abi.ps_cache_bytes(4096, 128, 8, 128, abi.PS_BF16, 8)
+    slab = 8 * 8 * (128 + 4096) * 128 * 2
+    assert n >= 2 * slab + 8 * 4096 * 8
+    assert n < 2 * slab + 8 * 4096 * 8 + 8192
+    assert abi.ps_cache_bytes(0, 1, 1, 64, abi.PS_F32, 1) == 0       # W = 0 rejected
+    assert abi.ps_cache_bytes(4, 1, 1, 96, abi.PS_F32, 1) == 0       # head_dim 96 unsupported
+    assert abi.ps_cache_bytes(4, -1, 1, 64, abi.PS_F32, 1) == 0
+    assert abi.ps_cache_bytes(4, 1, 1, 64, 7, 1) == 0                # unknown dtype
+
+
+def test_create_rejects_bad_arguments_before_touching_cuda():
+    from prefix_sliding_window_ring_b200 import abi
+    with pytest.raises(abi.PSError) as e:
+        abi.ps_cache_create(4, 1, 1, 64, abi.PS_F32, 1, None, 1 << 20, 0)
+    assert e.value.code == abi.PS_EINVAL
+    with pytest.raises(abi.PSError) as e:
+        abi.ps_cache_create(0, 1, 1, 64, abi.PS_F32, 1, 256, 1 << 20, 0)
+    assert e.value.code == abi.PS_EINVAL
+    with pytest.raises(abi.PSError) as e:
+        abi.ps_cache_create(4, 1, 1, 80, abi.PS_F32, 1, 256, 1 << 20, 0)
+    assert e.value.code == abi.PS_EUNSUPPORTED
+    with pytest.raises(abi.PSError) as e:
+        abi.ps_cache_create(4, 1, 1, 64, abi.PS_F32, 1, 256, 16, 0)
+    assert e.value.code == abi.PS_ENOMEM
+    assert "needs" in abi.ps_last_error()
+    assert abi.ps_decode_workspace_bytes(None, 1, 1) == 0
