@@ -143,6 +143,25 @@ PS_API int ps_attend_decode(ps_cache* c, const void* q, const int* seq_ids, cons
                      int B, int Hq, float scale, void* out, void* workspace,
                      size_t workspace_bytes, void* stream);
 
+/* ------------------------------ decode for callers that cannot allocate --- */
+
+/* ps_attend_decode without a workspace argument, for callers that cannot give
+ * the library device memory: a host runtime that owns all device memory through
+ * its own pool and offers plug-ins no allocation hook, or a latency-critical
+ * loop where a cudaMalloc (which synchronises the device) is not acceptable.
+ * The pages describe no such call; it exists for those callers only.
+ * Same arguments, results and errors as ps_attend_decode, except that the
+ * split-K scratch lives in a fixed 4 MiB array inside the library's device
+ * image (held by every GPU that loads the library until the process exits).
+ * It allocates nothing.  A batch whose scratch would exceed 4 MiB is rejected
+ * with PS_ENOMEM.  The first call on each device looks up the array's address
+ * and zero-fills it, which synchronises that device: make that first call
+ * before any stream capture.  All calls on a device share the array, so calls
+ * that overlap on the GPU (other streams, other threads) race; order them. */
+PS_API int ps_attend_decode_static(ps_cache* c, const void* q, const int* seq_ids,
+                                   const int64_t* t, int B, int Hq, float scale, void* out,
+                                   void* stream);
+
 /* ------------------------------------------- a6 chunked prefill/extend --- */
 
 /* Attention for a block of n consecutive queries of active sequence `seq` at

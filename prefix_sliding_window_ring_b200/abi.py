@@ -39,6 +39,7 @@ SIGNATURES = {
     "ps_append_kv": (_i, [_vp, _vp, _i, _vp, _vp, _i, _vp]),
     "ps_decode_workspace_bytes": (_sz, [_vp, _i, _i]),
     "ps_attend_decode": (_i, [_vp, _vp, _vp, _vp, _i, _i, _f, _vp, _vp, _sz, _vp]),
+    "ps_attend_decode_static": (_i, [_vp, _vp, _vp, _vp, _i, _i, _f, _vp, _vp]),
     "ps_attend_chunk": (_i, [_vp, _i, _vp, _vp, _vp, _i64, _i, _i, _f, _vp, _i, _vp]),
     "ps_export_window": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp]),
     "ps_import_window": (_i, [_vp, _i, _i64, _vp, _vp, _i, _i, _vp]),
@@ -51,7 +52,7 @@ SIGNATURES = {
 
 def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     if not os.path.exists(path):
-        raise ImportError(f"{path} is not built; run `python -m prefix_sliding_window_ring_b200.build`")
+        raise ImportError(f"{path} is not built; run `python prefix_sliding_window_ring_b200/build.py`")
     lib = ctypes.CDLL(path)
     for name, (res, args) in SIGNATURES.items():
         fn = getattr(lib, name)
@@ -153,6 +154,17 @@ def ps_attend_decode(cache, q, seq_ids, t, Hq, scale, out, workspace, workspace_
     _check("ps_attend_decode", _lib.ps_attend_decode(cache, _ptr(q), ids, ts, B, Hq, scale,
                                                      _ptr(out), _ptr(workspace), workspace_bytes,
                                                      _stream(stream)))
+
+
+def ps_attend_decode_static(cache, q, seq_ids, t, Hq, scale, out, stream=None) -> None:
+    """Decode with the library's fixed device scratch (no workspace, allocates nothing)."""
+    ids, B = _ints(seq_ids, ctypes.c_int)
+    ts, Bt = _ints(t, ctypes.c_int64)
+    if Bt != B:
+        raise ValueError("seq_ids and t differ in length")
+    _check("ps_attend_decode_static", _lib.ps_attend_decode_static(cache, _ptr(q), ids, ts, B, Hq,
+                                                                   scale, _ptr(out),
+                                                                   _stream(stream)))
 
 
 def ps_attend_chunk(cache, seq, q, k_blk, v_blk, t0, n, Hq, scale, out, append_after=0,

@@ -427,3 +427,21 @@ int ps_device_error(ps_cache* c, int32_t* code, void* stream) {
 }
 
 }  // extern "C"
+
+namespace ps {
+
+int set_error(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+int cache_hkv(const ps_cache* c) { return c->Hkv; }
+int cache_head_dim(const ps_cache* c) { return c->d; }
+int cache_sm_count(const ps_cache* c) { return c->sm_count; }
+
+}  // namespace ps

@@ -47,4 +47,14 @@ cudaError_t launch_chunk_cc(const CacheDev& c, int dtype, int G, int seq, int64_
                             int Hq, const void* q, const void* k_blk, const void* v_blk,
                             void* out, float scale, cudaStream_t st);
 
+// api.cu: error message of the calling thread, and cache accessors.
+int set_error(int code, const char* fmt, ...);
+
+}  // namespace ps
+
+struct ps_cache;
+namespace ps {
+int cache_hkv(const ps_cache* c);
+int cache_head_dim(const ps_cache* c);
+int cache_sm_count(const ps_cache* c);
 }  // namespace ps
