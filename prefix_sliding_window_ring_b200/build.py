@@ -1,6 +1,7 @@
 """Build step: compile the CUDA sources under csrc/ into libps.so (sm_100a).
 
-Run ``python -m prefix_sliding_window_ring_b200.build`` (or call ``build()``).
+Run ``python prefix_sliding_window_ring_b200/build.py`` (or call ``build()``).
+Importing the package needs the built library, so run this file by path.
 The library is built in-tree next to this file.
 """
 from __future__ import annotations
