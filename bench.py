@@ -201,6 +201,12 @@ class Workload:
                                  stream)
 
 
+def _check_device(wl):
+    code = wl.cache.device_error()
+    if code:
+        raise RuntimeError(f"device error word {code:#x} set by a kernel")
+
+
 def time_graph(torch, fn, n):
     """Capture n calls of fn(i) into one CUDA graph, replay it once, return ms per call."""
     s = torch.cuda.Stream()
@@ -239,7 +245,7 @@ def run_ours(args, rank, world, local_rank):
     for i in range(Wm):
         wl.step(i)
     torch.cuda.synchronize()
-    assert wl.cache.device_error() == 0
+    _check_device(wl)
 
     # ---- timed region: K steps replayed from one CUDA graph ----
     clocks = ClockSampler(local_rank) if rank == 0 else None
@@ -272,7 +278,7 @@ def run_ours(args, rank, world, local_rank):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_total = float(t.item())
     clk = clocks.stop() if clocks else None
-    assert wl.cache.device_error() == 0
+    _check_device(wl)
     ms_step = ms_total / K
     value = world * B * K / (ms_total / 1e3)
 
@@ -318,7 +324,7 @@ def run_ours(args, rank, world, local_rank):
         t = torch.tensor([ms_e2e], device="cuda", dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_e2e = float(t.item())
-    assert wl.cache.device_error() == 0
+    _check_device(wl)
     e2e_value = world * B * K / (ms_e2e / 1e3)
     h2d = (B * HKV * D * 2) * 2 + B * HQ * D * 2
     d2h = B * HQ * D * 2

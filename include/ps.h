@@ -90,7 +90,8 @@ PS_API int ps_cache_create(int W, int P_max, int Hkv, int d, int dtype, int max_
 PS_API void ps_cache_destroy(ps_cache* c);
 
 /* Return sequence `seq` to the empty state; its ring head starts at slot
- * ring_head_offset (0 <= offset < W).  Results never depend on the offset.
+ * ring_head_offset (0 <= offset < W).  Results do not depend on the offset
+ * beyond float32 rounding order.
  * Errors: PS_EINVAL. */
 PS_API int ps_seq_reset(ps_cache* c, int seq, int ring_head_offset, void* stream);
 

@@ -29,7 +29,10 @@ class Cache:
             self.handle = None
 
     def __del__(self):
-        self.close()
+        try:
+            self.close()
+        except Exception:  # interpreter shutdown: the binding may already be gone
+            pass
 
     # ---- calls, same names as the C ABI without the ps_ prefix ----
     def seq_reset(self, seq, ring_head_offset=0, stream=None):

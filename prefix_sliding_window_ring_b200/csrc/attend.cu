@@ -18,7 +18,10 @@
 #include <math.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "internal.h"
+#include "sm100_ptx.cuh"
 
 namespace ps {
 
@@ -71,65 +74,41 @@ template <int G, int D> struct MergeSmem {
   float o[kNW][G][D];
 };
 
-// Stream logical rows [j_begin, j_end) of `segs` for the G query heads of kv
-// head g; leave the CTA's merged state in (sm.m[0], sm.l[0], sm.o[0]).
+// Online-softmax state of one lane for the G query heads of a GQA group.
+// Rows are read LPR lanes per row, RPI rows per warp instruction, U row slots
+// per update; every lane of a row group ends an update with the same scores.
 template <typename T, int D, int G>
-__device__ __forceinline__ void stream_rows(const SegSet& segs, const T* __restrict__ kslab,
-                                            const T* __restrict__ vslab,
-                                            const T* __restrict__ kblk,
-                                            const T* __restrict__ vblk, int64_t blk_stride,
-                                            const T* __restrict__ qrow, float qscale,
-                                            int32_t j_begin, int32_t j_end,
-                                            MergeSmem<G, D>& sm) {
-  constexpr int VEC = Vec<T>::N;
-  constexpr int LPR = D / VEC;          // lanes per row
-  constexpr int RPI = 32 / LPR;         // rows per warp per load instruction
-  constexpr int U = G >= 8 ? 1 : (G >= 4 ? 2 : 4);
-  constexpr int STEP = RPI * U;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int c = lane % LPR, rs = lane / LPR;
-  const unsigned FULL = 0xffffffffu;
-
+struct AttnState {
+  static constexpr int VEC = Vec<T>::N;
+  static constexpr int LPR = D / VEC;   // lanes per row
+  static constexpr int RPI = 32 / LPR;  // rows per warp load instruction
+  static constexpr int U = G >= 8 ? 1 : (G >= 4 ? 2 : 4);
+  static constexpr int STEP = RPI * U;  // rows per update
   float q[G][VEC];
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    uint4 raw = *(const uint4*)(qrow + (size_t)h * D + c * VEC);
-    Vec<T>::unpack(raw, q[h]);
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) q[h][e] *= qscale;
-  }
   float mrun[G], lrun[G], o[G][VEC];
+  int c, rs;
+
+  __device__ __forceinline__ void init(const T* __restrict__ qrow, float qscale) {
+    const int lane = threadIdx.x & 31;
+    c = lane % LPR;
+    rs = lane / LPR;
 #pragma unroll
-  for (int h = 0; h < G; ++h) {
-    mrun[h] = -INFINITY; lrun[h] = 0.f;
+    for (int h = 0; h < G; ++h) {
+      uint4 raw = *(const uint4*)(qrow + (size_t)h * D + c * VEC);
+      Vec<T>::unpack(raw, q[h]);
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) o[h][e] = 0.f;
+      for (int e = 0; e < VEC; ++e) q[h][e] *= qscale;
+      mrun[h] = -INFINITY;
+      lrun[h] = 0.f;
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) o[h][e] = 0.f;
+    }
   }
 
-  for (int32_t g0 = j_begin + warp * STEP; g0 < j_end; g0 += kNW * STEP) {
-    uint4 kr[U], vr[U];
-    bool ok[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      int32_t j = g0 + u * RPI + rs;
-      ok[u] = j < j_end;
-      kr[u] = make_uint4(0, 0, 0, 0);
-      vr[u] = kr[u];
-      if (ok[u]) {
-        int si; int32_t off;
-        seg_locate(segs, j, si, off);
-        const T* kp; const T* vp;
-        if (segs.src[si] == 2) {
-          size_t r = (size_t)(segs.row0[si] + off) * blk_stride;
-          kp = kblk + r; vp = vblk + r;
-        } else {
-          size_t r = (size_t)(segs.row0[si] + off) * D;
-          kp = kslab + r; vp = vslab + r;
-        }
-        kr[u] = __ldcs((const uint4*)(kp + c * VEC));
-        vr[u] = __ldcs((const uint4*)(vp + c * VEC));
-      }
-    }
+  // Fold U rows (this lane's 16-byte slices kr/vr; ok = row exists) into the state.
+  __device__ __forceinline__ void update(const uint4 (&kr)[U], const uint4 (&vr)[U],
+                                         const bool (&ok)[U]) {
+    const unsigned FULL = 0xffffffffu;
     float sc[U][G];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -178,33 +157,61 @@ __device__ __forceinline__ void stream_rows(const SegSet& segs, const T* __restr
     }
   }
 
-  // merge the RPI row sub-groups of this warp
+  // Rows [0, nrows) of a contiguous tile (row stride D elements).
+  __device__ __forceinline__ void tile(const T* ks, const T* vs, int nrows) {
+    for (int r0 = 0; r0 < nrows; r0 += STEP) {
+      uint4 kr[U], vr[U];
+      bool ok[U];
 #pragma unroll
-  for (int off = LPR; off < 32; off <<= 1) {
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      float m2 = __shfl_xor_sync(FULL, mrun[h], off);
-      float l2 = __shfl_xor_sync(FULL, lrun[h], off);
-      float mm, ll, a1, a2;
-      merge_ml(mrun[h], lrun[h], m2, l2, mm, ll, a1, a2);
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) {
-        float o2 = __shfl_xor_sync(FULL, o[h][e], off);
-        o[h][e] = o[h][e] * a1 + o2 * a2;
+      for (int u = 0; u < U; ++u) {
+        int r = r0 + u * RPI + rs;
+        ok[u] = r < nrows;
+        kr[u] = make_uint4(0, 0, 0, 0);
+        vr[u] = kr[u];
+        if (ok[u]) {
+          kr[u] = *(const uint4*)(ks + (size_t)r * D + c * VEC);
+          vr[u] = *(const uint4*)(vs + (size_t)r * D + c * VEC);
+        }
       }
-      mrun[h] = mm; lrun[h] = ll;
+      update(kr, vr, ok);
     }
   }
-  if (rs == 0) {
+
+  // Merge this warp's row groups, then publish the warp's state in sm[warp].
+  __device__ __forceinline__ void to_smem(MergeSmem<G, D>& sm, int warp) {
+    const unsigned FULL = 0xffffffffu;
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      if (c == 0) { sm.m[warp][h] = mrun[h]; sm.l[warp][h] = lrun[h]; }
+    for (int off = LPR; off < 32; off <<= 1) {
 #pragma unroll
-      for (int e = 0; e < VEC; ++e) sm.o[warp][h][c * VEC + e] = o[h][e];
+      for (int h = 0; h < G; ++h) {
+        float m2 = __shfl_xor_sync(FULL, mrun[h], off);
+        float l2 = __shfl_xor_sync(FULL, lrun[h], off);
+        float mm, ll, a1, a2;
+        merge_ml(mrun[h], lrun[h], m2, l2, mm, ll, a1, a2);
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+          float o2 = __shfl_xor_sync(FULL, o[h][e], off);
+          o[h][e] = o[h][e] * a1 + o2 * a2;
+        }
+        mrun[h] = mm;
+        lrun[h] = ll;
+      }
+    }
+    if (rs == 0) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        if (c == 0) { sm.m[warp][h] = mrun[h]; sm.l[warp][h] = lrun[h]; }
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) sm.o[warp][h][c * VEC + e] = o[h][e];
+      }
     }
   }
+};
+
+// Merge the kNW warp states in sm into slot 0 (all threads of the CTA call this).
+template <int G, int D>
+__device__ __forceinline__ void merge_warps(MergeSmem<G, D>& sm) {
   __syncthreads();
-  // merge the warps into slot 0: first the per-head max/sum and warp weights
   if (threadIdx.x < G) {
     const int h = threadIdx.x;
     float mx = -INFINITY;
@@ -231,6 +238,50 @@ __device__ __forceinline__ void stream_rows(const SegSet& segs, const T* __restr
   __syncthreads();
 }
 
+// Stream logical rows [j_begin, j_end) of `segs` straight from global memory
+// (warp w takes row groups w, w+kNW, ...); leave the CTA state in sm slot 0.
+template <typename T, int D, int G>
+__device__ __forceinline__ void stream_rows(const SegSet& segs, const T* __restrict__ kslab,
+                                            const T* __restrict__ vslab,
+                                            const T* __restrict__ kblk,
+                                            const T* __restrict__ vblk, int64_t blk_stride,
+                                            const T* __restrict__ qrow, float qscale,
+                                            int32_t j_begin, int32_t j_end,
+                                            MergeSmem<G, D>& sm) {
+  using S = AttnState<T, D, G>;
+  S st;
+  st.init(qrow, qscale);
+  const int warp = threadIdx.x >> 5;
+  for (int32_t g0 = j_begin + warp * S::STEP; g0 < j_end; g0 += kNW * S::STEP) {
+    uint4 kr[S::U], vr[S::U];
+    bool ok[S::U];
+#pragma unroll
+    for (int u = 0; u < S::U; ++u) {
+      int32_t j = g0 + u * S::RPI + st.rs;
+      ok[u] = j < j_end;
+      kr[u] = make_uint4(0, 0, 0, 0);
+      vr[u] = kr[u];
+      if (ok[u]) {
+        int si; int32_t off;
+        seg_locate(segs, j, si, off);
+        const T* kp; const T* vp;
+        if (segs.src[si] == 2) {
+          size_t r = (size_t)(segs.row0[si] + off) * blk_stride;
+          kp = kblk + r; vp = vblk + r;
+        } else {
+          size_t r = (size_t)(segs.row0[si] + off) * D;
+          kp = kslab + r; vp = vslab + r;
+        }
+        kr[u] = __ldcs((const uint4*)(kp + st.c * S::VEC));
+        vr[u] = __ldcs((const uint4*)(vp + st.c * S::VEC));
+      }
+    }
+    st.update(kr, vr, ok);
+  }
+  st.to_smem(sm, warp);
+  merge_warps<G, D>(sm);
+}
+
 struct AttnArgs {
   CacheDev c;
   const void* q;
@@ -246,26 +297,156 @@ struct AttnArgs {
   BatchIds ids;
 };
 
+// ---------------------------------------------------------------- decode --
+// Pipelined split-K decode.  Warp kNW is the producer: one lane issues bulk
+// async copies (cp.async.bulk, no multicast) of contiguous K and V row tiles
+// into a kStages-deep shared-memory ring, each tile lying inside one visible
+// range (prefix rows, or one contiguous run of ring slots), so no evicted or
+// foreign row is ever fetched.  Warps 0..kNW-1 consume tiles round-robin with
+// the online softmax of AttnState.  Every wait is bounded: on a time-out the
+// CTA stops, reports ERR_TIMEOUT and drains its own copies before exiting.
+
+constexpr int kThreadsDec = (kNW + 1) * 32;
+// Tile i sits in stage i % kStages and is consumed by warp i % kNW.  With
+// kStages a multiple of kNW every stage belongs to one warp, which therefore
+// waits on its stages strictly in phase order: a warp can never reach a stage
+// two phases early, where the parity test would mistake the older completed
+// phase for the one it needs.
+constexpr int kStages = 8;
+static_assert(kStages % kNW == 0, "each pipeline stage must belong to one consumer warp");
+constexpr long long kWaitLimitCycles = 1ll << 30;  // about half a second
+
+template <typename T, int D> struct DecTile {
+  static constexpr int TR = 4096 / (D * (int)sizeof(T));  // rows per tile (4 KiB of K)
+};
+
+// Tiles of the logical range [jb, je): split at range boundaries and every TR rows.
+struct TilePlan {
+  int n;              // pieces
+  int ntiles;
+  int32_t len[4];
+  int32_t tbase[4];
+  int64_t row0[4];    // slab row of the first row of each piece
+};
+
+__device__ __forceinline__ TilePlan plan_tiles(const SegSet& s, int32_t jb, int32_t je, int TR,
+                                               bool* bad) {
+  TilePlan tp;
+  tp.n = 0;
+  tp.ntiles = 0;
+  int32_t L = 0;
+  for (int i = 0; i < s.n; ++i) {
+    int32_t a = max(L, jb), b = min(L + s.len[i], je);
+    if (b > a) {
+      if (s.src[i] == 2) {
+        *bad = true;
+      } else {
+        tp.len[tp.n] = b - a;
+        tp.tbase[tp.n] = tp.ntiles;
+        tp.row0[tp.n] = s.row0[i] + (a - L);
+        tp.ntiles += (b - a + TR - 1) / TR;
+        tp.n++;
+      }
+    }
+    L += s.len[i];
+  }
+  return tp;
+}
+
+__device__ __forceinline__ void tile_at(const TilePlan& tp, int i, int TR, int64_t& row,
+                                        int& nrows) {
+  int k = 0;
+#pragma unroll
+  for (int q = 1; q < 4; ++q)
+    if (q < tp.n && i >= tp.tbase[q]) k = q;
+  int32_t off = (i - tp.tbase[k]) * TR;
+  row = tp.row0[k] + off;
+  nrows = min(TR, tp.len[k] - off);
+}
+
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kThreadsAttn) k_decode(AttnArgs a) {
-  __shared__ MergeSmem<G, D> sm;
+__global__ void __launch_bounds__(kThreadsDec) k_decode(AttnArgs a) {
+  constexpr int TR = DecTile<T, D>::TR;
+  extern __shared__ __align__(1024) unsigned char dsm[];
+  T* ktile = (T*)dsm;                               // [kStages][TR][D]
+  T* vtile = ktile + (size_t)kStages * TR * D;      // [kStages][TR][D]
+  __shared__ __align__(8) uint64_t full[kStages], empty[kStages];
+  __shared__ int abort_flag;
   __shared__ int is_last;
+  __shared__ MergeSmem<G, D> sm;
+
   const int split = blockIdx.x, g = blockIdx.y, bl = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int s = a.ids.seq[bl];
   const DevMeta m = a.c.meta[s];
   const int64_t t = m.next_pos - 1;
   const SegSet segs = build_segments(m, a.c.W, a.c.P_max, t);
-  if (threadIdx.x == 0 && split == 0) {
-    if (t != a.ids.t[bl]) atomicOr(a.c.err, ERR_BATCH);
-    if (!segs.ring_ok) atomicOr(a.c.err, ERR_RING);
-    if ((int64_t)a.nsplit * a.chunk < segs.total) atomicOr(a.c.err, ERR_COVERAGE);
-  }
   const int32_t j_begin = split * a.chunk;
   const int32_t j_end = min(segs.total, j_begin + a.chunk);
+  bool bad = false;
+  const TilePlan tp = plan_tiles(segs, j_begin, j_end, TR, &bad);
+  if (threadIdx.x == 0) {
+    if (split == 0) {
+      if (t != a.ids.t[bl]) atomicOr(a.c.err, ERR_BATCH);
+      if (!segs.ring_ok) atomicOr(a.c.err, ERR_RING);
+      if ((int64_t)a.nsplit * a.chunk < segs.total) atomicOr(a.c.err, ERR_COVERAGE);
+    }
+    if (bad) atomicOr(a.c.err, ERR_BATCH);
+    for (int i = 0; i < kStages; ++i) {
+      ptx::mbar_init(&full[i], 1);
+      ptx::mbar_init(&empty[i], 1);
+    }
+    abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+
   const size_t slab = ((size_t)s * a.c.Hkv + g) * (size_t)a.c.slab_rows * D;
-  const T* qrow = (const T*)a.q + ((size_t)bl * a.Hq + (size_t)g * G) * D;
-  stream_rows<T, D, G>(segs, (const T*)a.c.K + slab, (const T*)a.c.V + slab, nullptr, nullptr,
-                       0, qrow, a.qscale, j_begin, j_end, sm);
+  const T* kslab = (const T*)a.c.K + slab;
+  const T* vslab = (const T*)a.c.V + slab;
+  if (warp == kNW) {
+    if (lane == 0) {  // producer
+      int issued = 0;
+      for (int i = 0; i < tp.ntiles; ++i) {
+        const int st = i % kStages;
+        if (i >= kStages &&
+            !ptx::mbar_wait_bounded(&empty[st], ((i / kStages) - 1) & 1, &abort_flag,
+                                    kWaitLimitCycles))
+          break;
+        int64_t row;
+        int nr;
+        tile_at(tp, i, TR, row, nr);
+        const uint32_t bytes = (uint32_t)nr * D * sizeof(T);
+        ptx::mbar_arrive_expect_tx(&full[st], 2 * bytes);
+        ptx::bulk_g2s(ktile + (size_t)st * TR * D, kslab + (size_t)row * D, bytes, &full[st]);
+        ptx::bulk_g2s(vtile + (size_t)st * TR * D, vslab + (size_t)row * D, bytes, &full[st]);
+        issued = i + 1;
+      }
+      if (abort_flag) {  // let the copies already issued land before the CTA exits
+        int quiet = 0;
+        for (int i = max(0, issued - kStages); i < issued; ++i)
+          ptx::mbar_wait_bounded(&full[i % kStages], (i / kStages) & 1, &quiet, kWaitLimitCycles);
+      }
+    }
+  } else {  // consumers
+    AttnState<T, D, G> st;
+    st.init((const T*)a.q + ((size_t)bl * a.Hq + (size_t)g * G) * D, a.qscale);
+    for (int i = warp; i < tp.ntiles; i += kNW) {
+      const int stg = i % kStages;
+      bool ok = ptx::mbar_wait_bounded(&full[stg], (i / kStages) & 1, &abort_flag,
+                                       kWaitLimitCycles);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      int64_t row;
+      int nr;
+      tile_at(tp, i, TR, row, nr);
+      st.tile(ktile + (size_t)stg * TR * D, vtile + (size_t)stg * TR * D, nr);
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&empty[stg]);
+    }
+    st.to_smem(sm, warp);
+  }
+  merge_warps<G, D>(sm);
+  if (threadIdx.x == 0 && abort_flag) atomicOr(a.c.err, ERR_TIMEOUT);
 
   const int bg = (a.b_off + bl) * a.c.Hkv + g;  // workspace slot of (batch entry, kv head)
   float* pml = a.part_ml + ((size_t)bg * a.nsplit + split) * G * 2;
@@ -328,16 +509,33 @@ __global__ void __launch_bounds__(kThreadsAttn) k_chunk_cc(AttnArgs a) {
   }
 }
 
+template <typename T, int D, int G>
+cudaError_t launch_decode_kernel(dim3 grid, const AttnArgs& a, cudaStream_t st) {
+  constexpr size_t dyn = (size_t)2 * kStages * DecTile<T, D>::TR * D * sizeof(T);
+  static std::atomic<uint64_t> configured{0};  // one bit per device
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (!(configured.load() & bit)) {
+    e = cudaFuncSetAttribute(k_decode<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)dyn);
+    if (e != cudaSuccess) return e;
+    configured.fetch_or(bit);
+  }
+  k_decode<T, D, G><<<grid, kThreadsDec, dyn, st>>>(a);
+  return cudaGetLastError();
+}
+
 template <typename T, int D>
 cudaError_t dispatch_decode_G(int G, dim3 grid, const AttnArgs& a, cudaStream_t st) {
   switch (G) {
-    case 1: k_decode<T, D, 1><<<grid, kThreadsAttn, 0, st>>>(a); break;
-    case 2: k_decode<T, D, 2><<<grid, kThreadsAttn, 0, st>>>(a); break;
-    case 4: k_decode<T, D, 4><<<grid, kThreadsAttn, 0, st>>>(a); break;
-    case 8: k_decode<T, D, 8><<<grid, kThreadsAttn, 0, st>>>(a); break;
+    case 1: return launch_decode_kernel<T, D, 1>(grid, a, st);
+    case 2: return launch_decode_kernel<T, D, 2>(grid, a, st);
+    case 4: return launch_decode_kernel<T, D, 4>(grid, a, st);
+    case 8: return launch_decode_kernel<T, D, 8>(grid, a, st);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 template <typename T, int D>
@@ -352,32 +550,46 @@ cudaError_t dispatch_chunk_G(int G, dim3 grid, const AttnArgs& a, cudaStream_t s
   return cudaGetLastError();
 }
 
-int target_ctas(int sm_count) { return sm_count * 8; }
+// Upper bound on decode CTAs per launch (sizes the workspace): 4 waves.
+int max_ctas_per_launch(int sm_count) { return sm_count * 12; }
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 }  // namespace
 
 DecodePlan plan_decode(int B, int Hkv, int n_max, int sm_count) {
-  DecodePlan p;
-  int pairs = B * Hkv;
-  int ns = (target_ctas(sm_count) + pairs - 1) / pairs;
-  if (ns < 1) ns = 1;
-  if (ns > kMaxSplit) ns = kMaxSplit;
-  int per = (n_max + ns - 1) / ns;
-  if (per < 64) per = 64;
-  per = (per + 31) / 32 * 32;
-  p.chunk = per;
-  p.nsplit = (n_max + per - 1) / per;
-  if (p.nsplit < 1) p.nsplit = 1;
-  return p;
+  // Pick the split count that minimises (waves x rows per CTA): every CTA of
+  // a wave streams at about the same rate, so a launch lasts about that long.
+  const int slots = sm_count * 3;  // resident decode CTAs per SM
+  const int pairs = B * Hkv;
+  DecodePlan best{1, n_max};
+  long long best_cost = -1;
+  const long long max_ctas = pairs > max_ctas_per_launch(sm_count) ? pairs
+                                                                     : max_ctas_per_launch(sm_count);
+  for (int ns = 1; ns <= kMaxSplit; ++ns) {
+    int per = (n_max + ns - 1) / ns;
+    if (per < 128 && ns > 1) break;
+    per = (per + 31) / 32 * 32;
+    int ns_eff = (n_max + per - 1) / per;
+    long long ctas = (long long)pairs * ns_eff;
+    if (ctas > max_ctas) break;
+    long long waves = (ctas + slots - 1) / slots;
+    long long cost = waves * (per + 96);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best.nsplit = ns_eff;
+      best.chunk = per;
+    }
+  }
+  return best;
 }
 
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int sm_count) {
   int G = Hq / Hkv;
   size_t tick = align256((size_t)B * Hkv * sizeof(int32_t));
-  size_t slots = (size_t)B * Hkv + (size_t)target_ctas(sm_count);  // >= B*Hkv*nsplit
-  if (slots > (size_t)B * Hkv * kMaxSplit) slots = (size_t)B * Hkv * kMaxSplit;
+  size_t pairs = (size_t)B * Hkv;  // B*Hkv*nsplit never exceeds max(pairs, max CTAs)
+  size_t slots = pairs > (size_t)max_ctas_per_launch(sm_count) ? pairs
+                                                               : (size_t)max_ctas_per_launch(sm_count);
   size_t ml = align256(slots * G * 2 * sizeof(float));
   size_t o = align256(slots * G * d * sizeof(float));
   return tick + ml + o;

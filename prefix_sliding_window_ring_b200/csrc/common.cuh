@@ -39,6 +39,7 @@ enum : int32_t {
   ERR_COVERAGE = 1,  // a split-K launch did not cover every visible row
   ERR_RING = 2,      // the ring does not hold the window a query needs
   ERR_BATCH = 4,     // a batch entry's position disagrees with the bookkeeping
+  ERR_TIMEOUT = 8,   // a pipeline wait gave up (the kernel stopped early)
 };
 
 // Row ranges a query at position t reads, in visiting order (at most 4):

@@ -110,11 +110,12 @@ def test_boundary_sweep(W, P, dtype):
 
 @pytest.mark.parametrize("W,P,h0", [(129, 100, 77), (4096, 1, 4000), (2, 0, 1)])
 def test_ring_head_offset_invariance(W, P, h0):
-    """The same history gives bit-identical outputs for any initial ring head."""
+    """The same history gives the same outputs for any initial ring head (up to
+    the order of float32 rounding: tiles split at the physical wrap of the ring)."""
     s = workloads.sweep_shape(W, P, "bf16")
     t_last = min(3 * W + P, P + W + 300)
     a, _ = run_sweep(s.Hq, s.Hkv, s.d, P, W, "bf16", t_last, h0=0, every_visible=97,
                      every_ring=997, every_out=53)
     b, _ = run_sweep(s.Hq, s.Hkv, s.d, P, W, "bf16", t_last, h0=h0, every_visible=97,
                      every_ring=997, every_out=53)
-    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    check_close(to_f64(b), to_f64(a), "bf16", f"head offset {h0} vs 0")

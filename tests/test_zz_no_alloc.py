@@ -51,7 +51,7 @@ def test_static_scratch_matches_workspace_decode_twice():
 
 
 def test_static_scratch_rejects_batches_over_its_size():
-    B, Hq, Hkv, d, P, W = 128, 64, 8, 128, 1, 128
+    B, Hq, Hkv, d, P, W = 128, 64, 8, 128, 1, 256
     c = Cache(W, P, Hkv, d, ps_dtype("bf16"), B)
     sd = SeqData(1, 0, Hq, Hkv, d, "bf16")
     kp, vp = to_torch(sd.k(0, P)), to_torch(sd.v(0, P))
