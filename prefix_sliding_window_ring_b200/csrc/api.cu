@@ -282,7 +282,7 @@ int ps_attend_decode(ps_cache* c, const void* q, const int* seq_ids, const int64
   if (B == 0) return ok();
   if ((r = check_batch(c, seq_ids, B))) return r;
   if (!t) return fail(PS_EINVAL, "t is NULL");
-  int n_max = 1;
+  std::vector<int32_t> rows(B);
   for (int b = 0; b < B; ++b) {
     const SeqHost& s = c->seqs[seq_ids[b]];
     if (t[b] != s.next_pos - 1)
@@ -291,16 +291,14 @@ int ps_attend_decode(ps_cache* c, const void* q, const int* seq_ids, const int64
     if (t[b] < s.P)
       return fail(PS_EPOS, "sequence %d: t=%lld lies inside the prefix (P=%d); append first",
                   seq_ids[b], (long long)t[b], s.P);
-    int n = s.P + s.count;
-    if (n > n_max) n_max = n;
+    rows[b] = s.P + s.count;
   }
   if (!q || !out || !aligned16(q) || !aligned16(out))
     return fail(PS_EINVAL, "q/out must be non-NULL 16-byte aligned device pointers");
   if (!workspace || ((uintptr_t)workspace & 255))
     return fail(PS_EINVAL, "workspace must be a non-NULL 256-byte aligned device pointer");
-  ps::DecodePlan plan = ps::plan_decode(B, c->Hkv, n_max, c->sm_count);
   size_t need = 0;
-  ps::DecodeWs ws = ps::decode_ws_layout(workspace, B, c->Hkv, G, c->d, plan.nsplit, &need);
+  ps::DecodeWs ws = ps::decode_ws_layout(workspace, B, c->Hkv, G, c->d, c->sm_count, &need);
   if (need > workspace_bytes)
     return fail(PS_ENOMEM, "workspace holds %zu bytes, this call needs %zu", workspace_bytes, need);
   if ((r = check_device(c))) return r;
@@ -314,9 +312,9 @@ int ps_attend_decode(ps_cache* c, const void* q, const int* seq_ids, const int64
       ids.seq[i] = seq_ids[b0 + i];
       ids.t[i] = t[b0 + i];
     }
-    PS_CUDA(ps::launch_decode(c->dev, c->dtype, G, ids, nb, b0, Hq,
+    PS_CUDA(ps::launch_decode(c->dev, c->dtype, G, ids, rows.data() + b0, nb, Hq,
                               (const char*)q + b0 * per_entry, (char*)out + b0 * per_entry, scale,
-                              ws, plan, st));
+                              ws, c->sm_count, st));
   }
   return ok();
 }

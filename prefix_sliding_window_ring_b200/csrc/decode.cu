@@ -1,0 +1,631 @@
+// Decode attention (visible-range derivation, split streaming, split merge).
+//
+// Work division.  The visible rows of all (batch entry, kv head) pairs of a
+// launch are laid end to end and cut into `nctas` equal ranges, one per CTA
+// (a multiple of the SM count), so every SM streams the same number of rows
+// whatever the batch shape.  A CTA walks the pairs its range touches; for each
+// it emits one partial (max, sum, accumulator) triple, and the last CTA to
+// finish a pair -- an atomic ticket, no spinning -- merges the pair's partials
+// into the output.
+//
+// Streaming.  Warp kCW is the producer: one lane issues bulk async copies
+// (cp.async.bulk, no multicast) of contiguous K and V row tiles of 16 KiB each
+// into a kStages-deep shared-memory ring (bulk copies much smaller than that
+// leave HBM bandwidth unused).  A tile never crosses a visible range (prefix
+// rows, or one contiguous run of ring slots split at the physical wrap), so no
+// evicted row is ever fetched ("Prefix Sliding" digest, section 06: iterate
+// the prefix blocks and the window blocks separately).  Each of the kCW
+// consumer warps takes its own share of every tile and keeps its own
+// online-softmax state; a stage is refilled once all of them have released it.
+//
+// Consumer arithmetic (per warp, LPR lanes per row, 8 scores per update):
+// each lane forms partial dot products for 8 (row, query head) scores, a
+// transpose-reduction leaves every lane with one complete score, the lane
+// exponentiates only that score, and the 8 weights are gathered back for the
+// weighted sum of the value rows.  Pairs of float32 lanes use the packed
+// fma.rn.f32x2 instruction (each half is an ordinary IEEE fma).
+//
+// Every wait is bounded; a time-out stops the CTA, sets ERR_TIMEOUT and lets
+// the copies already issued land before the CTA exits.
+#include <math.h>
+#include <string.h>
+
+#include <atomic>
+
+#include "attn_common.cuh"
+#include "internal.h"
+#include "sm100_ptx.cuh"
+
+#ifndef PS_DEC_STAGES
+#define PS_DEC_STAGES 3
+#endif
+#ifndef PS_DEC_TILE_BYTES
+#define PS_DEC_TILE_BYTES 16384
+#endif
+#ifndef PS_DEC_CTAS_PER_SM
+#define PS_DEC_CTAS_PER_SM 2
+#endif
+
+namespace ps {
+
+namespace {
+
+using namespace attn;
+
+#ifndef PS_DEC_CONSUMER_WARPS
+#define PS_DEC_CONSUMER_WARPS 8
+#endif
+constexpr int kCW = PS_DEC_CONSUMER_WARPS;   // consumer warps
+constexpr int kThreadsDec = (kCW + 1) * 32;  // plus one producer warp
+// Tile i sits in stage i % kStages.  Every consumer warp waits on every tile
+// in order and releases it, so no warp can reach a stage two phases ahead of
+// the one it needs (where the parity test would accept the older phase).
+constexpr int kStages = PS_DEC_STAGES;
+constexpr long long kWaitLimitCycles = 1ll << 30;  // about half a second
+constexpr int kMinRowsPerCta = 128;
+constexpr int kPieceBatch = 8;  // partials read together by the pair merge
+
+template <typename T, int D> struct DecTile {
+  static constexpr int TR = PS_DEC_TILE_BYTES / (D * (int)sizeof(T));  // rows per tile
+  static constexpr int RW = TR / kCW;                                    // rows per warp
+  static_assert(TR % kCW == 0, "tile rows must split evenly over the consumer warps");
+};
+
+struct DecodeArgs {
+  CacheDev c;
+  const void* q;
+  void* out;
+  float qscale;
+  int Hq, B, nctas;
+  int64_t total;    // visible rows of all pairs of the launch
+  float* part_ml;   // [nctas + B*Hkv][G][2]: per (pair, CTA) piece (max, sum), base 2
+  float* part_o;    // [nctas + B*Hkv][G][D]: per piece unnormalised accumulators
+  int32_t* tick;    // [B*Hkv] arrival counters, 0 at rest
+  int32_t seq[kMaxBatchPerLaunch];
+  int64_t t[kMaxBatchPerLaunch];
+  int64_t cum[kMaxBatchPerLaunch + 1];  // cum[b] = Hkv * (rows of entries before b)
+};
+
+__device__ __forceinline__ int64_t range_start(int64_t c, int64_t R, int64_t NC) {
+  return R * c / NC;
+}
+// CTA whose range holds row x: the largest c with range_start(c) <= x.
+__device__ __forceinline__ int64_t cta_of_row(int64_t x, int64_t R, int64_t NC) {
+  return ((x + 1) * NC - 1) / R;
+}
+
+__device__ __forceinline__ void cbar() {  // the consumer warps only
+  asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory");
+}
+
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0,
+                                      float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rd, {%0, %1};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rd;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+__device__ __forceinline__ void fmul2(float& d0, float& d1, float a) {
+  asm("{\n\t.reg .b64 ra, rd;\n\t"
+      "mov.b64 ra, {%2, %2};\n\t"
+      "mov.b64 rd, {%0, %1};\n\t"
+      "mul.rn.f32x2 rd, rd, ra;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a));
+}
+
+// Online-softmax state of one lane (see the file comment).
+template <typename T, int D, int G>
+struct DecState {
+  static constexpr int VEC = Vec<T>::N;
+  static constexpr int LPR = D / VEC;   // lanes per row
+  static constexpr int RPI = 32 / LPR;  // rows per warp load instruction
+  static constexpr int U = 8 / G;       // rows per row group per update
+  static constexpr int STEP = RPI * U;  // rows per warp per update
+  static constexpr int S1 = LPR / 2, S2 = LPR / 4, S3 = LPR / 8;
+  static_assert(LPR >= 8, "the transpose-reduction needs at least 8 lanes per row");
+
+  float q[G][VEC];
+  float m[G], o[G][VEC];
+  float mo, lpart;  // running max and partial sum of this lane's own head
+  int c, rs, base, kown;
+
+  __device__ __forceinline__ static int lane_of(int k) {
+    return ((k & 4) ? S1 : 0) | ((k & 2) ? S2 : 0) | ((k & 1) ? S3 : 0);
+  }
+
+  __device__ __forceinline__ void init(const T* __restrict__ qrow, float qscale) {
+    const int lane = threadIdx.x & 31;
+    c = lane % LPR;
+    rs = lane / LPR;
+    base = rs * LPR;
+    kown = ((c & S1) ? 4 : 0) | ((c & S2) ? 2 : 0) | ((c & S3) ? 1 : 0);
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      uint4 raw = *(const uint4*)(qrow + (size_t)h * D + c * VEC);
+      Vec<T>::unpack(raw, q[h]);
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) q[h][e] *= qscale;
+      m[h] = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) o[h][e] = 0.f;
+    }
+    mo = -INFINITY;
+    lpart = 0.f;
+  }
+
+  __device__ __forceinline__ void update(const uint4 (&kr)[U], const uint4 (&vr)[U],
+                                         const bool (&ok)[U]) {
+    const unsigned FULL = 0xffffffffu;
+    const int lane = threadIdx.x & 31;
+    // partial dot products of the 8 (row u, head h) scores, index u*G + h
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      float kf[VEC];
+      Vec<T>::unpack(kr[u], kf);
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int e = 0; e < VEC; e += 2) ffma2(a0, a1, q[h][e], q[h][e + 1], kf[e], kf[e + 1]);
+        v[u * G + h] = a0 + a1;
+      }
+    }
+    // transpose-reduction: 8 values -> 1 complete score per lane
+    {
+      const bool b1 = (lane & S1) != 0;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float send = b1 ? v[k] : v[k + 4];
+        float keep = b1 ? v[k + 4] : v[k];
+        v[k] = keep + __shfl_xor_sync(FULL, send, S1);
+      }
+      const bool b2 = (lane & S2) != 0;
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        float send = b2 ? v[k] : v[k + 2];
+        float keep = b2 ? v[k + 2] : v[k];
+        v[k] = keep + __shfl_xor_sync(FULL, send, S2);
+      }
+      const bool b3 = (lane & S3) != 0;
+      {
+        float send = b3 ? v[0] : v[1];
+        float keep = b3 ? v[1] : v[0];
+        v[0] = keep + __shfl_xor_sync(FULL, send, S3);
+      }
+#pragma unroll
+      for (int s = S3 / 2; s >= 1; s >>= 1) v[0] += __shfl_xor_sync(FULL, v[0], s);
+    }
+    bool okown = false;
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (kown / G == u) okown = ok[u];
+    const float sc = okown ? v[0] : -INFINITY;
+    // tile max of this lane's head (reduce over the lanes holding other rows)
+    float tm = sc;
+    if (G <= 4) tm = fmaxf(tm, __shfl_xor_sync(FULL, tm, S1));
+    if (G <= 2) tm = fmaxf(tm, __shfl_xor_sync(FULL, tm, S2));
+    if (G == 1) tm = fmaxf(tm, __shfl_xor_sync(FULL, tm, S3));
+    const float mo_new = fmaxf(mo, tm);
+    const float p = okown ? exp2f(sc - mo_new) : 0.f;
+    const float ao = (mo_new == -INFINITY) ? 1.f : exp2f(mo - mo_new);
+    lpart = lpart * ao + p;
+    mo = mo_new;
+    // every head's new max and rescale factor, in every lane
+    float alpha[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float th = __shfl_sync(FULL, tm, base | lane_of(h));
+      const float mn = fmaxf(m[h], th);
+      alpha[h] = (mn == -INFINITY) ? 1.f : exp2f(m[h] - mn);
+      m[h] = mn;
+    }
+    float pk[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) pk[k] = __shfl_sync(FULL, p, base | lane_of(k));
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+      for (int e = 0; e < VEC; e += 2) fmul2(o[h][e], o[h][e + 1], alpha[h]);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      float vf[VEC];
+      Vec<T>::unpack(vr[u], vf);
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float w = pk[u * G + h];
+#pragma unroll
+        for (int e = 0; e < VEC; e += 2) ffma2(o[h][e], o[h][e + 1], w, w, vf[e], vf[e + 1]);
+      }
+    }
+  }
+
+  // Rows [0, nrows) of a contiguous tile in shared memory (row stride D).
+  __device__ __forceinline__ void tile(const T* ks, const T* vs, int nrows) {
+    for (int r0 = 0; r0 < nrows; r0 += STEP) {
+      uint4 kr[U], vr[U];
+      bool ok[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int r = r0 + u * RPI + rs;
+        ok[u] = r < nrows;
+        kr[u] = make_uint4(0, 0, 0, 0);
+        vr[u] = kr[u];
+        if (ok[u]) {
+          kr[u] = *(const uint4*)(ks + (size_t)r * D + c * VEC);
+          vr[u] = *(const uint4*)(vs + (size_t)r * D + c * VEC);
+        }
+      }
+      update(kr, vr, ok);
+    }
+  }
+
+  // Finish the row group's sums, merge the warp's row groups, publish in sm[warp].
+  __device__ __forceinline__ void to_smem(MergeSmem<G, D, kCW>& sm, int warp) {
+    const unsigned FULL = 0xffffffffu;
+    float ls = lpart;
+    if (G <= 4) ls += __shfl_xor_sync(FULL, ls, S1);
+    if (G <= 2) ls += __shfl_xor_sync(FULL, ls, S2);
+    if (G == 1) ls += __shfl_xor_sync(FULL, ls, S3);
+    float l[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) l[h] = __shfl_sync(FULL, ls, base | lane_of(h));
+#pragma unroll
+    for (int off = LPR; off < 32; off <<= 1) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float m2 = __shfl_xor_sync(FULL, m[h], off);
+        const float l2 = __shfl_xor_sync(FULL, l[h], off);
+        float mm, ll, a1, a2;
+        merge_ml(m[h], l[h], m2, l2, mm, ll, a1, a2);
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+          const float o2 = __shfl_xor_sync(FULL, o[h][e], off);
+          o[h][e] = o[h][e] * a1 + o2 * a2;
+        }
+        m[h] = mm;
+        l[h] = ll;
+      }
+    }
+    if (rs == 0) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        if (c == 0) { sm.m[warp][h] = m[h]; sm.l[warp][h] = l[h]; }
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) sm.o[warp][h][c * VEC + e] = o[h][e];
+      }
+    }
+  }
+};
+
+// Merge the kCW consumer warps' states into slot 0 (consumer threads only).
+template <int G, int D>
+__device__ __forceinline__ void merge_consumers(MergeSmem<G, D, kCW>& sm) {
+  cbar();
+  if (threadIdx.x < G) {
+    const int h = threadIdx.x;
+    float mx = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kCW; ++w) mx = fmaxf(mx, sm.m[w][h]);
+    float l = 0.f;
+#pragma unroll
+    for (int w = 0; w < kCW; ++w) {
+      const float a = (mx == -INFINITY) ? 0.f : exp2f(sm.m[w][h] - mx);
+      sm.wt[w][h] = a;
+      l += sm.l[w][h] * a;
+    }
+    sm.m[0][h] = mx;
+    sm.l[0][h] = l;
+  }
+  cbar();
+  for (int idx = threadIdx.x; idx < G * D; idx += kCW * 32) {
+    const int h = idx / D, e = idx % D;
+    float acc = 0.f;
+#pragma unroll
+    for (int w = 0; w < kCW; ++w) acc += sm.o[w][h][e] * sm.wt[w][h];
+    sm.o[0][h][e] = acc;
+  }
+  cbar();
+}
+
+// Calls f(slab_row, nrows) for the tiles of the logical rows [jb, je) of one
+// pair: split at visible-range boundaries and every TR rows.  Registers only.
+// Sets *bad if the range reaches block rows (a decode query never does).
+template <typename F>
+__device__ __forceinline__ void for_each_tile(const SegSet& s, int32_t jb, int32_t je, int TR,
+                                              bool* bad, F&& f) {
+  int32_t L = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if (i < s.n) {
+      const int32_t a = max(L, jb), b = min(L + s.len[i], je);
+      if (b > a) {
+        if (s.src[i] == 2) {
+          *bad = true;
+        } else {
+          for (int32_t x = a; x < b; x += TR) f(s.row0[i] + (x - L), min(TR, b - x));
+        }
+      }
+      L += s.len[i];
+    }
+  }
+}
+
+// One pair (batch entry b, kv head g) restricted to local rows [lo, hi).
+struct PairPiece {
+  int b, g;
+  int64_t start;  // first flattened row of the pair
+  int32_t n;      // rows of the pair
+  int32_t lo, hi;
+};
+
+__device__ __forceinline__ PairPiece piece_at(const DecodeArgs& a, int64_t r, int64_t r1) {
+  int lo = 0, hi = a.B - 1;
+  while (lo < hi) {  // last entry with cum[b] <= r
+    const int mid = (lo + hi + 1) >> 1;
+    if (a.cum[mid] <= r) lo = mid; else hi = mid - 1;
+  }
+  PairPiece pp;
+  pp.b = lo;
+  pp.n = (int32_t)((a.cum[lo + 1] - a.cum[lo]) / a.c.Hkv);
+  pp.g = (int)((r - a.cum[lo]) / pp.n);
+  pp.start = a.cum[lo] + (int64_t)pp.g * pp.n;
+  pp.lo = (int32_t)(r - pp.start);
+  pp.hi = (int32_t)min((int64_t)pp.n, r1 - pp.start);
+  return pp;
+}
+
+template <typename T, int D, int G>
+__global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8) k_decode(const __grid_constant__ DecodeArgs a) {
+  constexpr int TR = DecTile<T, D>::TR;
+  extern __shared__ __align__(128) unsigned char dsm[];
+  T* ktile = (T*)dsm;                           // [kStages][TR][D]
+  T* vtile = ktile + (size_t)kStages * TR * D;  // [kStages][TR][D]
+  __shared__ __align__(8) uint64_t full[kStages], empty[kStages];
+  __shared__ int abort_flag;
+  __shared__ int is_last;
+  __shared__ MergeSmem<G, D, kCW> sm;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t NC = a.nctas, R = a.total;
+  const int64_t r0 = range_start(blockIdx.x, R, NC), r1 = range_start(blockIdx.x + 1, R, NC);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      ptx::mbar_init(&full[i], 1);
+      ptx::mbar_init(&empty[i], kCW);
+    }
+    abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kCW) {
+    if (lane != 0) return;
+    // ------------------------------------------------------------ producer --
+    int i = 0;
+    for (int64_t r = r0; r < r1 && !abort_flag;) {
+      const PairPiece pp = piece_at(a, r, r1);
+      r = pp.start + pp.hi;
+      const int s = a.seq[pp.b];
+      const DevMeta m = a.c.meta[s];
+      const SegSet segs = build_segments(m, a.c.W, a.c.P_max, m.next_pos - 1);
+      bool bad = false;
+      const size_t slab = ((size_t)s * a.c.Hkv + pp.g) * (size_t)a.c.slab_rows * D;
+      for_each_tile(segs, pp.lo, min(pp.hi, segs.total), TR, &bad, [&](int64_t row, int nr) {
+        if (abort_flag) return;
+        const int st = i % kStages;
+        if (i >= kStages && !ptx::mbar_wait_bounded(&empty[st], ((i / kStages) - 1) & 1,
+                                                    &abort_flag, kWaitLimitCycles))
+          return;
+        const uint32_t bytes = (uint32_t)nr * D * sizeof(T);
+        ptx::mbar_arrive_expect_tx(&full[st], 2 * bytes);
+        ptx::bulk_g2s(ktile + (size_t)st * TR * D, (const T*)a.c.K + slab + (size_t)row * D,
+                      bytes, &full[st]);
+        ptx::bulk_g2s(vtile + (size_t)st * TR * D, (const T*)a.c.V + slab + (size_t)row * D,
+                      bytes, &full[st]);
+        ++i;
+      });
+    }
+    if (abort_flag) {  // let the copies already issued land before the CTA exits
+      int quiet = 0;
+      for (int k = max(0, i - kStages); k < i; ++k)
+        ptx::mbar_wait_bounded(&full[k % kStages], (k / kStages) & 1, &quiet, kWaitLimitCycles);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers --
+  int i = 0;  // tiles consumed so far (all consumer warps see every tile)
+  for (int64_t r = r0; r < r1;) {
+    const PairPiece pp = piece_at(a, r, r1);
+    r = pp.start + pp.hi;
+    const int s = a.seq[pp.b];
+    const DevMeta m = a.c.meta[s];
+    const int64_t t = m.next_pos - 1;
+    const SegSet segs = build_segments(m, a.c.W, a.c.P_max, t);
+    DecState<T, D, G> st;
+    st.init((const T*)a.q + ((size_t)pp.b * a.Hq + (size_t)pp.g * G) * D, a.qscale);
+    constexpr int RW = DecTile<T, D>::RW;
+    bool bad = false, stop = false;
+    for_each_tile(segs, pp.lo, min(pp.hi, segs.total), TR, &bad, [&](int64_t, int nr) {
+      if (stop) return;
+      const int stg = i % kStages;
+      const bool ok = ptx::mbar_wait_bounded(&full[stg], (i / kStages) & 1, &abort_flag,
+                                             kWaitLimitCycles);
+      if (!__all_sync(0xffffffffu, ok)) {
+        stop = true;
+        return;
+      }
+      const int mine = min(RW, nr - warp * RW);  // this warp's rows of the tile
+      if (mine > 0)
+        st.tile(ktile + ((size_t)stg * TR + warp * RW) * D,
+                vtile + ((size_t)stg * TR + warp * RW) * D, mine);
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&empty[stg]);
+      ++i;
+    });
+    if (threadIdx.x == 0) {
+      if (t != a.t[pp.b] || segs.total != pp.n || bad) atomicOr(a.c.err, ERR_BATCH);
+      if (!segs.ring_ok) atomicOr(a.c.err, ERR_RING);
+    }
+    st.to_smem(sm, warp);
+    merge_consumers<G, D>(sm);
+
+    // publish this piece, then merge the pair if this CTA is the last to finish it
+    const int pair = pp.b * a.c.Hkv + pp.g;
+    const int64_t slot = (int64_t)blockIdx.x + pair;
+    float* pml = a.part_ml + (size_t)slot * G * 2;
+    float* po = a.part_o + (size_t)slot * G * D;
+    for (int idx = threadIdx.x; idx < G * D; idx += kCW * 32) po[idx] = sm.o[0][idx / D][idx % D];
+    if (threadIdx.x < G) {
+      pml[threadIdx.x * 2] = sm.m[0][threadIdx.x];
+      pml[threadIdx.x * 2 + 1] = sm.l[0][threadIdx.x];
+    }
+    __threadfence();
+    cbar();
+    const int64_t first = cta_of_row(pp.start, R, NC);
+    const int64_t last = cta_of_row(pp.start + pp.n - 1, R, NC);
+    if (threadIdx.x == 0) {
+      const int old = atomicAdd(&a.tick[pair], 1);
+      is_last = (old == (int)(last - first));
+    }
+    cbar();
+    if (is_last) {
+      __threadfence();
+      T* orow = (T*)a.out + ((size_t)pp.b * a.Hq + (size_t)pp.g * G) * D;
+      for (int idx = threadIdx.x; idx < G * D; idx += kCW * 32) {
+        const int h = idx / D, e = idx % D;
+        // online merge of the pieces, kPieceBatch independent loads at a time
+        float M = -INFINITY, L = 0.f, A = 0.f;
+        for (int64_t c0 = first; c0 <= last; c0 += kPieceBatch) {
+          float mj[kPieceBatch], lj[kPieceBatch], oj[kPieceBatch];
+#pragma unroll
+          for (int j = 0; j < kPieceBatch; ++j) {
+            const int64_t sl = c0 + j + pair;
+            const bool in = c0 + j <= last;
+            mj[j] = in ? __ldcg(a.part_ml + ((size_t)sl * G + h) * 2) : -INFINITY;
+            lj[j] = in ? __ldcg(a.part_ml + ((size_t)sl * G + h) * 2 + 1) : 0.f;
+            oj[j] = in ? __ldcg(a.part_o + ((size_t)sl * G + h) * D + e) : 0.f;
+          }
+          float bm = M;
+#pragma unroll
+          for (int j = 0; j < kPieceBatch; ++j) bm = fmaxf(bm, mj[j]);
+          if (bm == -INFINITY) continue;
+          const float sc = exp2f(M - bm);  // M = -inf gives 0
+          L *= sc;
+          A *= sc;
+#pragma unroll
+          for (int j = 0; j < kPieceBatch; ++j) {
+            const float w = (mj[j] == -INFINITY) ? 0.f : exp2f(mj[j] - bm);
+            L += lj[j] * w;
+            A += oj[j] * w;
+          }
+          M = bm;
+        }
+        store_out<T>(orow + (size_t)h * D + e, A / L);
+      }
+      if (threadIdx.x == 0) a.tick[pair] = 0;
+    }
+    cbar();
+  }
+  if (threadIdx.x == 0 && abort_flag) atomicOr(a.c.err, ERR_TIMEOUT);
+}
+
+template <typename T, int D, int G>
+cudaError_t launch_kernel(int nctas, const DecodeArgs& a, cudaStream_t st) {
+  constexpr size_t dyn = (size_t)2 * kStages * DecTile<T, D>::TR * D * sizeof(T);
+  static std::atomic<uint64_t> configured{0};  // one bit per device
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (!(configured.load() & bit)) {
+    e = cudaFuncSetAttribute(k_decode<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)dyn);
+    if (e != cudaSuccess) return e;
+    configured.fetch_or(bit);
+  }
+  k_decode<T, D, G><<<nctas, kThreadsDec, dyn, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t dispatch_G(int G, int nctas, const DecodeArgs& a, cudaStream_t st) {
+  switch (G) {
+    case 1: return launch_kernel<T, D, 1>(nctas, a, st);
+    case 2: return launch_kernel<T, D, 2>(nctas, a, st);
+    case 4: return launch_kernel<T, D, 4>(nctas, a, st);
+    case 8: return launch_kernel<T, D, 8>(nctas, a, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+int max_ctas(int sm_count) { return sm_count * PS_DEC_CTAS_PER_SM; }
+
+}  // namespace
+
+DecodeWs decode_ws_layout(void* ws, int B, int Hkv, int G, int d, int sm_count, size_t* bytes) {
+  const int Bl = B < kMaxBatchPerLaunch ? B : kMaxBatchPerLaunch;  // launches run in turn
+  const size_t pairs = (size_t)Bl * Hkv;
+  const size_t slots = (size_t)max_ctas(sm_count) + pairs;
+  const size_t tick = align256(pairs * sizeof(int32_t));
+  const size_t ml = align256(slots * G * 2 * sizeof(float));
+  const size_t o = align256(slots * G * d * sizeof(float));
+  DecodeWs w;
+  char* p = (char*)ws;
+  w.tick = (int32_t*)p;
+  w.part_ml = (float*)(p + tick);
+  w.part_o = (float*)(p + tick + ml);
+  if (bytes) *bytes = tick + ml + o;
+  return w;
+}
+
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int sm_count) {
+  size_t bytes = 0;
+  decode_ws_layout(nullptr, B, Hkv, Hq / Hkv, d, sm_count, &bytes);
+  return bytes;
+}
+
+cudaError_t launch_decode(const CacheDev& c, int dtype, int G, const BatchIds& ids,
+                          const int32_t* rows, int B, int Hq, const void* q, void* out,
+                          float scale, const DecodeWs& ws, int sm_count, cudaStream_t st) {
+  DecodeArgs a;
+  memset(&a, 0, sizeof(a));
+  a.c = c;
+  a.q = q;
+  a.out = out;
+  a.qscale = scale * kLog2e;
+  a.Hq = Hq;
+  a.B = B;
+  a.part_ml = ws.part_ml;
+  a.part_o = ws.part_o;
+  a.tick = ws.tick;
+  a.cum[0] = 0;
+  for (int b = 0; b < B; ++b) {
+    a.seq[b] = ids.seq[b];
+    a.t[b] = ids.t[b];
+    a.cum[b + 1] = a.cum[b] + (int64_t)c.Hkv * rows[b];
+  }
+  a.total = a.cum[B];
+  int64_t nc = (a.total + kMinRowsPerCta - 1) / kMinRowsPerCta;
+  if (nc > max_ctas(sm_count)) nc = max_ctas(sm_count);
+  if (nc < 1) nc = 1;
+  a.nctas = (int)nc;
+  if (dtype == 0) {
+    if (c.d == 64) return dispatch_G<float, 64>(G, a.nctas, a, st);
+    return dispatch_G<float, 128>(G, a.nctas, a, st);
+  }
+  if (c.d == 64) return dispatch_G<uint16_t, 64>(G, a.nctas, a, st);
+  return dispatch_G<uint16_t, 128>(G, a.nctas, a, st);
+}
+
+}  // namespace ps

@@ -64,20 +64,12 @@ int ps_attend_decode_static(ps_cache* c, const void* q, const int* seq_ids, cons
   if (B < 0 || Hq < 1) return ps::set_error(PS_EINVAL, "ps_attend_decode_static: bad B or Hq");
   if (B > 0 && (!seq_ids || !t))
     return ps::set_error(PS_EINVAL, "ps_attend_decode_static: seq_ids/t is NULL");
-  // Scratch this call needs, from the same plan ps_attend_decode uses.
-  int Hkv = ps::cache_hkv(c), d = ps::cache_head_dim(c);
+  // Scratch this call needs: the same layout ps_attend_decode uses.
+  const int Hkv = ps::cache_hkv(c);
   if (Hq % Hkv) return ps_attend_decode(c, q, seq_ids, t, B, Hq, scale, out, nullptr, 0, stream);
-  int n_max = 1;
-  for (int b = 0; b < B; ++b) {
-    ps_seq_info info;
-    int r = ps_seq_info_get(c, seq_ids[b], &info);
-    if (r) return r;
-    int n = info.P + info.count;
-    if (n > n_max) n_max = n;
-  }
-  ps::DecodePlan plan = ps::plan_decode(B, Hkv, n_max, ps::cache_sm_count(c));
   size_t need = 0;
-  ps::decode_ws_layout(nullptr, B, Hkv, Hq / Hkv, d, plan.nsplit, &need);
+  ps::decode_ws_layout(nullptr, B, Hkv, Hq / Hkv, ps::cache_head_dim(c), ps::cache_sm_count(c),
+                       &need);
   if (need > kStaticScratchBytes)
     return ps::set_error(PS_ENOMEM,
                          "ps_attend_decode_static: this batch needs %zu bytes of scratch, above "

@@ -7,7 +7,7 @@
 
 namespace ps {
 
-constexpr int kMaxBatchPerLaunch = 256;  // batch entries passed by value per launch
+constexpr int kMaxBatchPerLaunch = 128;  // batch entries passed by value per launch
 
 struct BatchIds {
   int32_t seq[kMaxBatchPerLaunch];
@@ -27,22 +27,22 @@ cudaError_t launch_ring_export(const CacheDev& c, int esize, int seq, void* k, v
 cudaError_t launch_debug_visible(const CacheDev& c, int seq, int64_t t, int64_t* pos_out,
                                  int32_t* n_out, cudaStream_t st);
 
-// attend.cu (CUDA-core kernels)
-struct DecodePlan {
-  int nsplit;   // CTAs per (sequence, kv head)
-  int chunk;    // visible rows per CTA
-};
-DecodePlan plan_decode(int B, int Hkv, int n_max, int sm_count);
-size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int sm_count);
+// decode.cu
 struct DecodeWs {
   int32_t* tick;    // [B][Hkv] arrival counters (0 at rest)
-  float* part_ml;   // [B][Hkv][nsplit][G][2] per-split (max, sum), base-2 domain
-  float* part_o;    // [B][Hkv][nsplit][G][d] per-split unnormalised accumulators
+  float* part_ml;   // per (pair, CTA) piece: (max, sum) per query head, base-2 domain
+  float* part_o;    // per piece: unnormalised accumulators [G][d]
 };
-DecodeWs decode_ws_layout(void* ws, int B, int Hkv, int G, int d, int nsplit, size_t* bytes);
-cudaError_t launch_decode(const CacheDev& c, int dtype, int G, const BatchIds& ids, int B,
-                          int b_off, int Hq, const void* q, void* out, float scale,
-                          const DecodeWs& ws, const DecodePlan& plan, cudaStream_t st);
+// Workspace of one decode call (launches of more than kMaxBatchPerLaunch
+// entries run in turn and reuse it).
+DecodeWs decode_ws_layout(void* ws, int B, int Hkv, int G, int d, int sm_count, size_t* bytes);
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int sm_count);
+// rows[b]: visible rows of entry b (P + count), as the host bookkeeping has them.
+cudaError_t launch_decode(const CacheDev& c, int dtype, int G, const BatchIds& ids,
+                          const int32_t* rows, int B, int Hq, const void* q, void* out,
+                          float scale, const DecodeWs& ws, int sm_count, cudaStream_t st);
+
+// attend.cu (CUDA-core chunk kernel)
 cudaError_t launch_chunk_cc(const CacheDev& c, int dtype, int G, int seq, int64_t t0, int n,
                             int Hq, const void* q, const void* k_blk, const void* v_blk,
                             void* out, float scale, cudaStream_t st);
