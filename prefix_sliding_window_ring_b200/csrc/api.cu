@@ -340,8 +340,11 @@ int ps_attend_chunk(ps_cache* c, int seq, const void* q, const void* k_blk, cons
     return fail(PS_EINVAL, "q/k_blk/v_blk/out must be non-NULL 16-byte aligned device pointers");
   if ((r = check_device(c))) return r;
   cudaStream_t st = (cudaStream_t)stream;
-  PS_CUDA(ps::launch_chunk_cc(c->dev, c->dtype, G, seq, t0, n, Hq, q, k_blk, v_blk, out, scale,
-                              st));
+  if (ps::chunk_tc_supported(c->dtype, c->d, G))
+    PS_CUDA(ps::launch_chunk_tc(c->dev, G, seq, t0, n, Hq, q, k_blk, v_blk, out, scale, st));
+  else
+    PS_CUDA(ps::launch_chunk_cc(c->dev, c->dtype, G, seq, t0, n, Hq, q, k_blk, v_blk, out, scale,
+                                st));
   if (append_after) {
     ps::BatchIds ids;
     memset(&ids, 0, sizeof(ids));

@@ -1,0 +1,495 @@
+// Chunked prefill/extend on the tcgen05 tensor cores (bf16, head_dim 128).
+//
+// A block of n queries at positions t0..t0+n-1 attends to the pinned prefix,
+// the ring entries of each query's window and the block itself, causally
+// ("Prefix Sliding" digest, sections 03 and 06).  One CTA takes a 128-row
+// query tile: 128/G consecutive positions of each of the G query heads that
+// share one key/value head, so every key tile feeds all G heads at once.
+//
+// Key tiles (128 rows) are walked range by range -- prefix rows, the ring
+// window as at most two contiguous slot runs split at the physical wrap, then
+// the block rows -- so no evicted row is ever loaded; only tiles on a window
+// or causal edge are masked element by element.
+//
+// Roles (8 warps):
+//   warp 0   TMA producer: Q once, then K and V tiles into 2-stage rings
+//            (tensor-map tiled loads with 128-byte swizzle, no multicast);
+//   warp 1   MMA issuer: S_j = Q K_j^T into one of two TMEM buffers, then
+//            O += P_j V_j with P_j read from TMEM (kind::f16, f32 accumulate);
+//   warp 2   owns the TMEM allocation;
+//   warps 4-7 softmax: each thread owns one query row -- loads S_j from TMEM,
+//            masks, keeps a running max (raised lazily, rescaling O in TMEM
+//            only when it grows by more than 2^8), writes P_j (bf16) back over
+//            S_j and finally normalises O into the output.
+// Every wait is bounded: a time-out sets ERR_TIMEOUT, every role stops, the
+// MMA issuer waits for its issued work and the TMEM is freed.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "internal.h"
+#include "sm100_ptx.cuh"
+
+namespace ps {
+
+namespace {
+
+constexpr int kBM = 128;          // query rows per CTA
+constexpr int kBN = 128;          // key rows per tile
+constexpr int kHD = 128;          // head dim
+constexpr int kThreadsTC = 256;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColO = 256;
+constexpr float kRaiseThreshold = 8.0f;  // log2 units: rescale O only past 2^8
+constexpr long long kWaitLimit = 1ll << 31;  // about a second
+constexpr uint32_t kTileBytes = kBN * kHD * 2;  // one K or V tile: 32 KiB
+
+__host__ __device__ __forceinline__ uint32_t col_s(int st) { return st ? 128u : 0u; }
+
+struct ChunkArgs {
+  CUtensorMap qmap;   // q [n][Hq][128]: box (64, 1, PT)
+  CUtensorMap kslab;  // cache K [S*Hkv][slab_rows][128]: box (64, 128, 1)
+  CUtensorMap vslab;
+  CUtensorMap kblk;   // k_blk [n][Hkv][128]: box (64, 1, 128)
+  CUtensorMap vblk;
+  CacheDev c;
+  void* out;
+  int seq, n, Hq, G, PT;
+  int64_t t0;
+  float sc;  // softmax scale * log2(e)
+};
+
+struct __align__(1024) TcSmem {
+  uint8_t q[2][kBM * 128];       // two 64-column blocks of 128-byte rows
+  uint8_t k[2][2][kBN * 128];    // [stage][column block]
+  uint8_t v[2][2][kBN * 128];
+};
+
+// The key tiles of one query tile: up to 4 ranges, each tiled from its start.
+struct KSched {
+  int n;
+  int ntiles;
+  int src[4];       // 0: cache slab row, 1: block row
+  int64_t row0[4];  // first slab row / block row of the range
+  int64_t pos0[4];  // position of that row
+  int32_t len[4];
+  int32_t tbase[4];
+};
+
+struct KTile {
+  int src;
+  int64_t row, pos0;
+  int valid;
+};
+
+__device__ __forceinline__ void add_range(KSched& s, int src, int64_t row0, int64_t pos0,
+                                          int64_t len) {
+  if (len <= 0) return;
+  s.src[s.n] = src;
+  s.row0[s.n] = row0;
+  s.pos0[s.n] = pos0;
+  s.len[s.n] = (int32_t)len;
+  s.tbase[s.n] = s.ntiles;
+  s.ntiles += (int32_t)((len + kBN - 1) / kBN);
+  s.n++;
+}
+
+// Query positions [plo, phi]; the ring holds [next_pos - count, next_pos - 1] = [.., t0 - 1].
+__device__ __forceinline__ KSched make_sched(const DevMeta& m, int W, int P_max, int64_t t0,
+                                             int64_t plo, int64_t phi) {
+  KSched s;
+  s.n = 0;
+  s.ntiles = 0;
+  for (int i = 0; i < 4; ++i) { s.src[i] = 0; s.row0[i] = 0; s.pos0[i] = 0; s.len[i] = 0; s.tbase[i] = 0; }
+  add_range(s, 0, 0, 0, m.P);  // pinned prefix
+  int64_t lo = plo - W + 1;
+  if (lo < m.P) lo = m.P;
+  const int64_t base = m.next_pos - m.count;
+  int64_t rlo = lo < base ? base : lo;  // never below what the ring holds
+  if (t0 - 1 >= rlo) {
+    const int64_t nw = t0 - rlo;
+    const int64_t s0 = ((int64_t)m.head + (rlo - base)) % W;
+    const int64_t lenA = nw < W - s0 ? nw : W - s0;
+    add_range(s, 0, P_max + s0, rlo, lenA);
+    add_range(s, 0, P_max, rlo + lenA, nw - lenA);
+  }
+  const int64_t blo = lo > t0 ? lo : t0;
+  add_range(s, 1, blo - t0, blo, phi - blo + 1);
+  return s;
+}
+
+__device__ __forceinline__ KTile tile_of(const KSched& s, int j) {
+  KTile t;
+  t.src = s.src[0]; t.row = s.row0[0]; t.pos0 = s.pos0[0]; t.valid = 0;
+  int k = 0;
+#pragma unroll
+  for (int q = 1; q < 4; ++q)
+    if (q < s.n && j >= s.tbase[q]) k = q;
+  int64_t off = 0, len = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    if (q == k) {
+      t.src = s.src[q];
+      off = (int64_t)(j - s.tbase[q]) * kBN;
+      t.row = s.row0[q] + off;
+      t.pos0 = s.pos0[q] + off;
+      len = s.len[q];
+    }
+  t.valid = (int)(len - off < kBN ? len - off : kBN);
+  return t;
+}
+
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, int* abort_flag) {
+  return ptx::mbar_wait_bounded(bar, parity, abort_flag, kWaitLimit);
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constant__ ChunkArgs a) {
+  extern __shared__ uint8_t dsm_raw[];
+  TcSmem& sm = *reinterpret_cast<TcSmem*>(
+      (uint8_t*)(((uintptr_t)dsm_raw + 1023) & ~(uintptr_t)1023));
+  __shared__ __align__(8) uint64_t q_full, k_full[2], k_empty[2], v_full[2], v_empty[2];
+  __shared__ __align__(8) uint64_t s_full[2], p_full[2], o_full, mma_done;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = blockIdx.y;
+  const int PT = a.PT;
+  const int i0 = blockIdx.x * PT;
+  const DevMeta m = a.c.meta[a.seq];
+  const int64_t plo = a.t0 + i0;
+  const int64_t phi = a.t0 + min(i0 + PT, a.n) - 1;
+  const KSched ks = make_sched(m, a.c.W, a.c.P_max, a.t0, plo, phi);
+  const int T = ks.ntiles;
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&k_full[i], 1);
+      ptx::mbar_init(&k_empty[i], 1);
+      ptx::mbar_init(&v_full[i], 1);
+      ptx::mbar_init(&v_empty[i], 1);
+      ptx::mbar_init(&s_full[i], 1);
+      ptx::mbar_init(&p_full[i], 4);
+    }
+    ptx::mbar_init(&o_full, 1);
+    ptx::mbar_init(&mma_done, 1);
+    abort_flag = 0;
+    ptx::fence_mbar_init();
+    if (m.next_pos != a.t0 && blockIdx.x == 0 && g == 0) atomicOr(a.c.err, ERR_BATCH);
+  }
+  if (warp == 2) {
+    ptx::tmem_alloc(&tmem_slot, kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0) {
+      const int slab_z = a.seq * a.c.Hkv + g;
+      int issued_k = 0, issued_v = 0;
+      ptx::mbar_arrive_expect_tx(&q_full, 2 * kBM * 128);
+      for (int hh = 0; hh < a.G; ++hh)
+        for (int b = 0; b < 2; ++b)
+          ptx::tma_load_3d(&sm.q[b][hh * PT * 128], &a.qmap, b * 64, g * a.G + hh, i0, &q_full);
+      for (int j = 0; j < T && !abort_flag; ++j) {
+        const int st = j & 1;
+        const KTile kt = tile_of(ks, j);
+        if (j >= 2 && !wait_bar(&k_empty[st], ((j >> 1) - 1) & 1, &abort_flag)) break;
+        ptx::mbar_arrive_expect_tx(&k_full[st], kTileBytes);
+        for (int b = 0; b < 2; ++b) {
+          if (kt.src == 0)
+            ptx::tma_load_3d(sm.k[st][b], &a.kslab, b * 64, (int32_t)kt.row, slab_z, &k_full[st]);
+          else
+            ptx::tma_load_3d(sm.k[st][b], &a.kblk, b * 64, g, (int32_t)kt.row, &k_full[st]);
+        }
+        issued_k = j + 1;
+        if (j >= 2 && !wait_bar(&v_empty[st], ((j >> 1) - 1) & 1, &abort_flag)) break;
+        ptx::mbar_arrive_expect_tx(&v_full[st], kTileBytes);
+        for (int b = 0; b < 2; ++b) {
+          if (kt.src == 0)
+            ptx::tma_load_3d(sm.v[st][b], &a.vslab, b * 64, (int32_t)kt.row, slab_z, &v_full[st]);
+          else
+            ptx::tma_load_3d(sm.v[st][b], &a.vblk, b * 64, g, (int32_t)kt.row, &v_full[st]);
+        }
+        issued_v = j + 1;
+      }
+      if (abort_flag) {  // let the copies already issued land before the CTA exits
+        int quiet = 0;
+        ptx::mbar_wait_bounded(&q_full, 0, &quiet, kWaitLimit);
+        for (int j = issued_k > 2 ? issued_k - 2 : 0; j < issued_k; ++j)
+          ptx::mbar_wait_bounded(&k_full[j & 1], (j >> 1) & 1, &quiet, kWaitLimit);
+        for (int j = issued_v > 2 ? issued_v - 2 : 0; j < issued_v; ++j)
+          ptx::mbar_wait_bounded(&v_full[j & 1], (j >> 1) & 1, &quiet, kWaitLimit);
+      }
+    }
+  } else if (warp == 1) {
+    // --------------------------------------------------------- MMA issuer --
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = ptx::idesc_bf16_f32(kBM, kBN, 0, 0);
+      constexpr uint32_t idesc_o = ptx::idesc_bf16_f32(kBM, kHD, 0, 1);
+      bool ok = wait_bar(&q_full, 0, &abort_flag);
+      int pv_next = 0;  // next P V product to issue
+      auto issue_pv = [&](int jj) -> bool {
+        const int st = jj & 1;
+        if (!wait_bar(&p_full[st], (jj >> 1) & 1, &abort_flag)) return false;
+        if (!wait_bar(&v_full[st], (jj >> 1) & 1, &abort_flag)) return false;
+        ptx::tc_fence_after();
+        for (int k = 0; k < kBN / 16; ++k) {
+          // B = V tile, MN-major: 64-column blocks 16 KiB apart, 8-row groups 1 KiB apart
+          const uint64_t bdesc = ptx::sdesc_sw128(sm.v[st][0] + k * 16 * 128, 16384, 1024);
+          ptx::mma_ts(tmem + kColO, tmem + col_s(st) + k * 8, bdesc, idesc_o,
+                      (jj > 0 || k > 0) ? 1u : 0u);
+        }
+        ptx::mma_commit(&v_empty[st]);
+        ptx::mma_commit(&o_full);
+        return true;
+      };
+      for (int j = 0; j < T && ok; ++j) {
+        const int st = j & 1;
+        if (!wait_bar(&k_full[st], (j >> 1) & 1, &abort_flag)) { ok = false; break; }
+        ptx::tc_fence_after();
+        for (int k = 0; k < kHD / 16; ++k) {
+          const int b = k >> 2, kk = k & 3;
+          const uint64_t adesc = ptx::sdesc_sw128(sm.q[b] + kk * 32, 16, 1024);
+          const uint64_t bdesc = ptx::sdesc_sw128(sm.k[st][b] + kk * 32, 16, 1024);
+          ptx::mma_ss(tmem + col_s(st), adesc, bdesc, idesc_s, k > 0 ? 1u : 0u);
+        }
+        ptx::mma_commit(&s_full[st]);
+        ptx::mma_commit(&k_empty[st]);
+        if (j >= 1) {
+          if (!issue_pv(j - 1)) { ok = false; break; }
+          pv_next = j;
+        }
+      }
+      if (ok && T > 0) issue_pv(pv_next);
+      ptx::mma_commit(&mma_done);
+      int quiet = 0;
+      ptx::mbar_wait_bounded(&mma_done, 0, &quiet, kWaitLimit);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------- softmax --
+    const int wq = warp - 4;
+    const int r = wq * 32 + lane;  // query row of this thread
+    const int hh = r / PT, i = i0 + r % PT;
+    const int64_t tq = a.t0 + i;
+    const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
+    const int W = a.c.W, P = m.P;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < T; ++j) {
+      const int st = j & 1;
+      ok = wait_bar(&s_full[st], (j >> 1) & 1, &abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      ptx::tc_fence_after();
+      float x[kBN];
+      {
+        uint32_t raw[32];
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          ptx::tmem_ld32(tmem + lane_base + col_s(st) + c4 * 32, raw);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) x[c4 * 32 + c] = __uint_as_float(raw[c]) * a.sc;
+        }
+      }
+      const KTile kt = tile_of(ks, j);
+      // element masks only for tiles on a window or causal edge
+      const bool full = kt.valid == kBN &&
+                        (kt.src == 0 && kt.pos0 + kBN <= P
+                             ? true
+                             : (kt.pos0 >= phi - W + 1 && kt.pos0 + kBN - 1 <= plo));
+      if (!full) {
+        auto clampc = [](int64_t v) -> int { return v < -1 ? -1 : (v > kBN ? kBN : (int)v); };
+        const int pre_c = clampc(P - kt.pos0);           // c < pre_c: pinned prefix
+        const int lo_c = clampc(tq - W + 1 - kt.pos0);   // window start
+        const int hi_c = clampc(tq - kt.pos0);           // causal end
+#pragma unroll
+        for (int c = 0; c < kBN; ++c) {
+          const bool vis = c < kt.valid && (c < pre_c || (c >= lo_c && c <= hi_c));
+          if (!vis) x[c] = -INFINITY;
+        }
+      }
+      float mx = x[0];
+#pragma unroll
+      for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, x[c]);
+      // Raise the reference max lazily.  tcgen05.ld/st are warp-collective, so
+      // the O rescale runs for the whole warp when any lane needs it.
+      const bool raise = mx > m_run + kRaiseThreshold || (m_run == -INFINITY && mx > -INFINITY);
+      const float m_new = raise ? mx : m_run;
+      const bool need_o = raise && j > 0 && m_run > -INFINITY;
+      if (__any_sync(0xffffffffu, need_o)) {
+        const float alpha = need_o ? ex2(m_run - m_new) : 1.f;
+        // O holds P_0..P_{j-1} times V: wait for the last product, then rescale it
+        ok = wait_bar(&o_full, (j - 1) & 1, &abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          uint32_t o[32];
+          ptx::tmem_ld32(tmem + lane_base + kColO + c4 * 32, o);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+          ptx::tmem_st32(tmem + lane_base + kColO + c4 * 32, o);
+        }
+        ptx::tmem_wait_st();
+        l_run *= alpha;
+      }
+      m_run = m_new;
+      const float mu = m_run == -INFINITY ? 0.f : m_run;
+      float lsum = 0.f;
+      uint32_t pk[kBN / 2];
+#pragma unroll
+      for (int c = 0; c < kBN; c += 2) {
+        const float p0 = ex2(x[c] - mu), p1 = ex2(x[c + 1] - mu);
+        lsum += p0 + p1;
+        pk[c / 2] = pack_bf16(p0, p1);
+      }
+      l_run += lsum;
+      {
+        uint32_t half[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) half[c] = pk[c];
+        ptx::tmem_st32(tmem + lane_base + col_s(st), half);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) half[c] = pk[32 + c];
+        ptx::tmem_st32(tmem + lane_base + col_s(st) + 32, half);
+      }
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&p_full[st]);
+    }
+    if (ok && T > 0) {
+      // mma_done is committed once, after the last product: a parity wait on
+      // o_full here could take an older phase while two products are in flight.
+      ok = wait_bar(&mma_done, 0, &abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (ok && T > 0) {
+      ptx::tc_fence_after();
+      const float inv = 1.f / l_run;
+      uint16_t* orow = (uint16_t*)a.out + ((size_t)i * a.Hq + (size_t)g * a.G + hh) * kHD;
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+        uint32_t o[32];
+        ptx::tmem_ld32(tmem + lane_base + kColO + c4 * 32, o);
+        ptx::tmem_wait_ld();
+        if (i < a.n) {
+          uint32_t w[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            w[c] = pack_bf16(__uint_as_float(o[2 * c]) * inv, __uint_as_float(o[2 * c + 1]) * inv);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            *(uint4*)(orow + c4 * 32 + v4 * 8) =
+                make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+        }
+      }
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && abort_flag) atomicOr(a.c.err, ERR_TIMEOUT);
+  if (warp == 2) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------ tensor maps --
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
+  });
+  return fn;
+}
+
+// 3-D bf16 map, dims innermost first, byte strides of dims 1 and 2, 128B swizzle.
+bool map3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
+           uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {s1, s2};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool chunk_tc_supported(int dtype, int d, int G) {
+  return dtype == 1 && d == kHD && (G == 1 || G == 2 || G == 4 || G == 8);
+}
+
+cudaError_t launch_chunk_tc(const CacheDev& c, int G, int seq, int64_t t0, int n, int Hq,
+                            const void* q, const void* k_blk, const void* v_blk, void* out,
+                            float scale, cudaStream_t st) {
+  ChunkArgs a;
+  memset(&a, 0, sizeof(a));
+  const uint64_t row = kHD * 2;  // bytes per head row
+  const int PT = kBM / G;
+  bool ok = map3d(&a.qmap, q, kHD, Hq, n, row, (uint64_t)Hq * row, 64, 1, PT);
+  ok = ok && map3d(&a.kslab, c.K, kHD, c.slab_rows, (uint64_t)c.S * c.Hkv, row,
+                   (uint64_t)c.slab_rows * row, 64, kBN, 1);
+  ok = ok && map3d(&a.vslab, c.V, kHD, c.slab_rows, (uint64_t)c.S * c.Hkv, row,
+                   (uint64_t)c.slab_rows * row, 64, kBN, 1);
+  ok = ok && map3d(&a.kblk, k_blk, kHD, c.Hkv, n, row, (uint64_t)c.Hkv * row, 64, 1, kBN);
+  ok = ok && map3d(&a.vblk, v_blk, kHD, c.Hkv, n, row, (uint64_t)c.Hkv * row, 64, 1, kBN);
+  if (!ok) return cudaErrorInvalidValue;
+  a.c = c;
+  a.out = out;
+  a.seq = seq;
+  a.n = n;
+  a.Hq = Hq;
+  a.G = G;
+  a.PT = PT;
+  a.t0 = t0;
+  a.sc = scale * 1.4426950408889634f;
+  const size_t dyn = sizeof(TcSmem) + 1024;
+  static std::atomic<uint64_t> configured{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (!(configured.load() & (1ull << (dev & 63)))) {
+    e = cudaFuncSetAttribute(k_chunk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
+    if (e != cudaSuccess) return e;
+    configured.fetch_or(1ull << (dev & 63));
+  }
+  dim3 grid((n + PT - 1) / PT, c.Hkv);
+  k_chunk_tc<<<grid, kThreadsTC, dyn, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace ps

@@ -42,6 +42,12 @@ cudaError_t launch_decode(const CacheDev& c, int dtype, int G, const BatchIds& i
                           const int32_t* rows, int B, int Hq, const void* q, void* out,
                           float scale, const DecodeWs& ws, int sm_count, cudaStream_t st);
 
+// chunk_tc.cu (tcgen05 chunk kernel: bf16, head_dim 128)
+bool chunk_tc_supported(int dtype, int d, int G);
+cudaError_t launch_chunk_tc(const CacheDev& c, int G, int seq, int64_t t0, int n, int Hq,
+                            const void* q, const void* k_blk, const void* v_blk, void* out,
+                            float scale, cudaStream_t st);
+
 // attend.cu (CUDA-core chunk kernel)
 cudaError_t launch_chunk_cc(const CacheDev& c, int dtype, int G, int seq, int64_t t0, int n,
                             int Hq, const void* q, const void* k_blk, const void* v_blk,
