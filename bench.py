@@ -329,6 +329,10 @@ def run_ours(args, rank, world, local_rank):
     h2d = (B * HKV * D * 2) * 2 + B * HQ * D * 2
     d2h = B * HQ * D * 2
 
+    prefill = None
+    if rank == 0 and not args.no_prefill:
+        prefill = prefill_measure(max(3, min(args.steps, 10)))
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl.seed, wl.kscale, budget_s=args.cpu_seconds)
@@ -355,8 +359,76 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": 2 * K,
         "clocks": clk,
         "cpu_baseline": cpu,
+        "prefill": prefill,
     }
     print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------ prefill -------
+PF_P, PF_N, PF_T0, PF_SEQS = 256, 2048, 100000, 4
+
+
+def load_bf16_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f)["bf16_tflops"], "measured (burst)"
+    return 1590.0, "fallback"
+
+
+def prefill_measure(steps: int):
+    """Chunked prefill/extend on the tensor-core kernel: 4 sequences, each a
+    2048-query block at t0=100000 (window full), P=256, W in {4096, 16384}.
+    One step = the 4 calls.  Throughput counts only visible (query, key) pairs:
+    4 * d * Hq * sum over queries of (P + W) flops."""
+    import torch
+
+    import synth
+    from prefix_sliding_window_ring_b200 import PS_BF16, Cache
+    peak, peak_src = load_bf16_peak()
+
+    def dev(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+
+    res = {"workload": f"{PF_SEQS} sequences x {PF_N}-query blocks at t0={PF_T0}, "
+                       f"Hq={HQ} Hkv={HKV} d={D} P={PF_P}, bf16",
+           "kernel": "ps::k_chunk_tc (tcgen05)", "peak": peak, "peak_source": peak_src,
+           "unit": "TFLOP/s"}
+    for Wp in (4096, 16384):
+        c = Cache(Wp, PF_P, HKV, D, PS_BF16, PF_SEQS)
+        blocks = []
+        for s in range(PF_SEQS):
+            c.seq_reset(s, 0)
+            c.prefill_prefix(s, dev(synth.rows(SEED, synth.TID_K, s, HKV, 0, PF_P, D, "bf16")),
+                             dev(synth.rows(SEED, synth.TID_V, s, HKV, 0, PF_P, D, "bf16")), PF_P)
+            c.import_window(s, PF_T0,
+                            dev(synth.rows(SEED, synth.TID_K, s, HKV, PF_T0 - Wp, Wp, D, "bf16")),
+                            dev(synth.rows(SEED, synth.TID_V, s, HKV, PF_T0 - Wp, Wp, D, "bf16")),
+                            Wp, (977 * s) % Wp)
+            q = dev(synth.rows(SEED, synth.TID_Q, s, HQ, PF_T0, PF_N, D, "bf16"))
+            kb = dev(synth.rows(SEED, synth.TID_K, s, HKV, PF_T0, PF_N, D, "bf16"))
+            vb = dev(synth.rows(SEED, synth.TID_V, s, HKV, PF_T0, PF_N, D, "bf16"))
+            blocks.append((q, kb, vb, torch.empty_like(q)))
+        scale = 1.0 / math.sqrt(D)
+
+        def step(i, st=None):
+            for s, (q, kb, vb, o) in enumerate(blocks):
+                c.attend_chunk(s, q, kb, vb, PF_T0, PF_N, HQ, scale, o, 0, st)
+
+        for i in range(3):
+            step(i)
+        torch.cuda.synchronize()
+        if c.device_error():
+            raise RuntimeError("device error word set by the chunk kernel")
+        ms = min(time_graph(torch, step, steps) for _ in range(2))
+        flops = 4.0 * D * HQ * PF_N * (PF_P + Wp) * PF_SEQS
+        tf = flops / (ms / 1e3) / 1e12
+        res[f"W{Wp}"] = {"ms_per_step": round(ms, 4), "gflop_per_step": round(flops / 1e9, 1),
+                         "achieved": round(tf, 1), "frac": round(tf / peak, 4)}
+        c.close()
+        del blocks
+        torch.cuda.empty_cache()
+    return res
 
 
 # ------------------------------------------------------------ CPU oracle ----
@@ -439,6 +511,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-prefill", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

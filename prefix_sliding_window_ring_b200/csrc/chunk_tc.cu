@@ -17,10 +17,12 @@
 //   warp 1   MMA issuer: S_j = Q K_j^T into one of two TMEM buffers, then
 //            O += P_j V_j with P_j read from TMEM (kind::f16, f32 accumulate);
 //   warp 2   owns the TMEM allocation;
-//   warps 4-7 softmax: each thread owns one query row -- loads S_j from TMEM,
-//            masks, keeps a running max (raised lazily, rescaling O in TMEM
-//            only when it grows by more than 2^8), writes P_j (bf16) back over
-//            S_j and finally normalises O into the output.
+//   warps 4-11 softmax: each query row is shared by two threads (same TMEM
+//            lane, one half of the columns each), which exchange row maxima
+//            and sums through shared memory.  They load S_j from TMEM, mask,
+//            keep a running max (raised lazily, rescaling O in TMEM only when
+//            it grows by more than 2^8), write P_j (bf16) back over S_j and
+//            finally normalise O into the output.
 // Every wait is bounded: a time-out sets ERR_TIMEOUT, every role stops, the
 // MMA issuer waits for its issued work and the TMEM is freed.
 #include <cuda.h>
@@ -41,7 +43,8 @@ namespace {
 constexpr int kBM = 128;          // query rows per CTA
 constexpr int kBN = 128;          // key rows per tile
 constexpr int kHD = 128;          // head dim
-constexpr int kThreadsTC = 256;
+constexpr int kThreadsTC = 384;  // 4 service warps + 8 softmax warps
+constexpr int kSoftWarps = 8;    // two per TMEM lane quadrant, one per half of the columns
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 256;
 constexpr float kRaiseThreshold = 8.0f;  // log2 units: rescale O only past 2^8
@@ -167,6 +170,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
   __shared__ __align__(8) uint64_t s_full[2], p_full[2], o_full, mma_done;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
+  __shared__ float xchg[2][2][kBM];  // [parity][column half][row]: partial maxima / sums
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = blockIdx.y;
@@ -186,7 +190,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
       ptx::mbar_init(&v_full[i], 1);
       ptx::mbar_init(&v_empty[i], 1);
       ptx::mbar_init(&s_full[i], 1);
-      ptx::mbar_init(&p_full[i], 4);
+      ptx::mbar_init(&p_full[i], kSoftWarps);
     }
     ptx::mbar_init(&o_full, 1);
     ptx::mbar_init(&mma_done, 1);
@@ -289,50 +293,68 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------- softmax --
-    const int wq = warp - 4;
-    const int r = wq * 32 + lane;  // query row of this thread
+    const int quad = warp & 3;            // TMEM lane quadrant this warp may access
+    const int half = (warp - 4) >> 2;     // which 64 columns of S / O it owns
+    const int r = quad * 32 + lane;       // query row of this thread
     const int hh = r / PT, i = i0 + r % PT;
     const int64_t tq = a.t0 + i;
-    const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
+    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+    const int cbase = half * 64;          // first S/O column of this thread
     const int W = a.c.W, P = m.P;
-    float m_run = -INFINITY, l_run = 0.f;
+    const float sc = a.sc;
+    const int pair_bar = 2 + quad;        // named barrier of the two warps of this quadrant
+    auto pair_sync = [&]() { asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory"); };
+    float m_run = -INFINITY, l_run = 0.f;  // m_run: reference max (log2 units); l_run: my half
+    // After a failed wait (ok == false) a warp skips all work but still meets its
+    // partner at every pair barrier, so neither can be left waiting there.
     bool ok = true;
     for (int j = 0; j < T; ++j) {
       const int st = j & 1;
-      ok = wait_bar(&s_full[st], (j >> 1) & 1, &abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      ptx::tc_fence_after();
-      float x[kBN];
-      {
-        uint32_t raw[32];
+      if (ok) ok = __all_sync(0xffffffffu, wait_bar(&s_full[st], (j >> 1) & 1, &abort_flag));
+      float x[64];
+      float mloc = -INFINITY;
+      if (ok) {
+        ptx::tc_fence_after();
+        uint32_t raw0[32], raw1[32];
+        ptx::tmem_ld32(tmem + lane_base + col_s(st) + cbase, raw0);
+        ptx::tmem_ld32(tmem + lane_base + col_s(st) + cbase + 32, raw1);
+        ptx::tmem_wait_ld();
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          ptx::tmem_ld32(tmem + lane_base + col_s(st) + c4 * 32, raw);
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 32; ++c) x[c4 * 32 + c] = __uint_as_float(raw[c]) * a.sc;
+        for (int c = 0; c < 32; ++c) {
+          x[c] = __uint_as_float(raw0[c]);
+          x[32 + c] = __uint_as_float(raw1[c]);
         }
-      }
-      const KTile kt = tile_of(ks, j);
-      // element masks only for tiles on a window or causal edge
-      const bool full = kt.valid == kBN &&
-                        (kt.src == 0 && kt.pos0 + kBN <= P
-                             ? true
-                             : (kt.pos0 >= phi - W + 1 && kt.pos0 + kBN - 1 <= plo));
-      if (!full) {
-        auto clampc = [](int64_t v) -> int { return v < -1 ? -1 : (v > kBN ? kBN : (int)v); };
-        const int pre_c = clampc(P - kt.pos0);           // c < pre_c: pinned prefix
-        const int lo_c = clampc(tq - W + 1 - kt.pos0);   // window start
-        const int hi_c = clampc(tq - kt.pos0);           // causal end
+        const KTile kt = tile_of(ks, j);
+        // element masks only for tiles on a window or causal edge
+        const bool full = kt.valid == kBN &&
+                          (kt.src == 0 && kt.pos0 + kBN <= P
+                               ? true
+                               : (kt.pos0 >= phi - W + 1 && kt.pos0 + kBN - 1 <= plo));
+        if (!full) {
+          auto clampc = [](int64_t v) -> int { return v < -1 ? -1 : (v > kBN ? kBN : (int)v); };
+          const int pre_c = clampc(P - kt.pos0) - cbase;          // c < pre_c: pinned prefix
+          const int lo_c = clampc(tq - W + 1 - kt.pos0) - cbase;  // window start
+          const int hi_c = clampc(tq - kt.pos0) - cbase;          // causal end
+          const int vc = kt.valid - cbase;
 #pragma unroll
-        for (int c = 0; c < kBN; ++c) {
-          const bool vis = c < kt.valid && (c < pre_c || (c >= lo_c && c <= hi_c));
-          if (!vis) x[c] = -INFINITY;
+          for (int c = 0; c < 64; ++c) {
+            const bool vis = c < vc && (c < pre_c || (c >= lo_c && c <= hi_c));
+            if (!vis) x[c] = -INFINITY;
+          }
         }
-      }
-      float mx = x[0];
+        // row max of the raw scores (the scale is positive), as a tree
+        float t8[8];
 #pragma unroll
-      for (int c = 1; c < kBN; ++c) mx = fmaxf(mx, x[c]);
+        for (int u = 0; u < 8; ++u) t8[u] = x[u];
+#pragma unroll
+        for (int c = 8; c < 64; ++c) t8[c & 7] = fmaxf(t8[c & 7], x[c]);
+        mloc = fmaxf(fmaxf(fmaxf(t8[0], t8[1]), fmaxf(t8[2], t8[3])),
+                     fmaxf(fmaxf(t8[4], t8[5]), fmaxf(t8[6], t8[7])));
+      }
+      xchg[st][half][r] = mloc;
+      pair_sync();
+      if (!ok) continue;
+      const float mx = fmaxf(mloc, xchg[st][half ^ 1][r]) * sc;  // row max, log2 units
       // Raise the reference max lazily.  tcgen05.ld/st are warp-collective, so
       // the O rescale runs for the whole warp when any lane needs it.
       const bool raise = mx > m_run + kRaiseThreshold || (m_run == -INFINITY && mx > -INFINITY);
@@ -340,42 +362,38 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
       const bool need_o = raise && j > 0 && m_run > -INFINITY;
       if (__any_sync(0xffffffffu, need_o)) {
         const float alpha = need_o ? ex2(m_run - m_new) : 1.f;
-        // O holds P_0..P_{j-1} times V: wait for the last product, then rescale it
-        ok = wait_bar(&o_full, (j - 1) & 1, &abort_flag);
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        // O holds P_0..P_{j-1} times V: wait for the last product, then rescale my half
+        ok = __all_sync(0xffffffffu, wait_bar(&o_full, (j - 1) & 1, &abort_flag));
+        if (!ok) continue;
         ptx::tc_fence_after();
+        uint32_t o0[32], o1[32];
+        ptx::tmem_ld32(tmem + lane_base + kColO + cbase, o0);
+        ptx::tmem_ld32(tmem + lane_base + kColO + cbase + 32, o1);
+        ptx::tmem_wait_ld();
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          uint32_t o[32];
-          ptx::tmem_ld32(tmem + lane_base + kColO + c4 * 32, o);
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-          ptx::tmem_st32(tmem + lane_base + kColO + c4 * 32, o);
+        for (int c = 0; c < 32; ++c) {
+          o0[c] = __float_as_uint(__uint_as_float(o0[c]) * alpha);
+          o1[c] = __float_as_uint(__uint_as_float(o1[c]) * alpha);
         }
+        ptx::tmem_st32(tmem + lane_base + kColO + cbase, o0);
+        ptx::tmem_st32(tmem + lane_base + kColO + cbase + 32, o1);
         ptx::tmem_wait_st();
         l_run *= alpha;
       }
       m_run = m_new;
       const float mu = m_run == -INFINITY ? 0.f : m_run;
-      float lsum = 0.f;
-      uint32_t pk[kBN / 2];
+      float s8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[32];
 #pragma unroll
-      for (int c = 0; c < kBN; c += 2) {
-        const float p0 = ex2(x[c] - mu), p1 = ex2(x[c + 1] - mu);
-        lsum += p0 + p1;
-        pk[c / 2] = pack_bf16(p0, p1);
+      for (int c = 0; c < 64; c += 2) {
+        const float p0 = ex2(fmaf(x[c], sc, -mu)), p1 = ex2(fmaf(x[c + 1], sc, -mu));
+        s8[(c >> 1) & 7] += p0 + p1;
+        pk[c >> 1] = pack_bf16(p0, p1);
       }
-      l_run += lsum;
-      {
-        uint32_t half[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) half[c] = pk[c];
-        ptx::tmem_st32(tmem + lane_base + col_s(st), half);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) half[c] = pk[32 + c];
-        ptx::tmem_st32(tmem + lane_base + col_s(st) + 32, half);
-      }
+      l_run += ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
+      // P occupies the first 64 columns of the S buffer; my 64 keys are 32 of them.
+      // The partner read its scores from those columns before the pair barrier.
+      ptx::tmem_st32(tmem + lane_base + col_s(st) + half * 32, pk);
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       __syncwarp();
@@ -387,14 +405,18 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
       ok = wait_bar(&mma_done, 0, &abort_flag);
       ok = __all_sync(0xffffffffu, ok);
     }
+    // row sum = both halves (the parity slot 0/1 of the last tile is not reused here)
+    xchg[T & 1][half][r] = l_run;
+    pair_sync();
+    const float l_row = l_run + xchg[T & 1][half ^ 1][r];
     if (ok && T > 0) {
       ptx::tc_fence_after();
-      const float inv = 1.f / l_run;
+      const float inv = 1.f / l_row;
       uint16_t* orow = (uint16_t*)a.out + ((size_t)i * a.Hq + (size_t)g * a.G + hh) * kHD;
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
+      for (int c2 = 0; c2 < 2; ++c2) {
         uint32_t o[32];
-        ptx::tmem_ld32(tmem + lane_base + kColO + c4 * 32, o);
+        ptx::tmem_ld32(tmem + lane_base + kColO + cbase + c2 * 32, o);
         ptx::tmem_wait_ld();
         if (i < a.n) {
           uint32_t w[16];
@@ -403,7 +425,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
             w[c] = pack_bf16(__uint_as_float(o[2 * c]) * inv, __uint_as_float(o[2 * c + 1]) * inv);
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4)
-            *(uint4*)(orow + c4 * 32 + v4 * 8) =
+            *(uint4*)(orow + cbase + c2 * 32 + v4 * 8) =
                 make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
         }
       }
