@@ -50,6 +50,26 @@ def workload_config():
                   f"({ROT * kv_bytes_per_step() / 1e6:.0f} MB resident K/V)"}
 
 
+def rank_seed(rank: int) -> int:
+    """Each rank decodes its own sequences: the inputs of rank r use seed SEED + 1000 r."""
+    return SEED + 1000 * rank
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """Largest value over all ranks (the job lasts as long as its slowest rank)."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world: int, steps: int, ms_total: float) -> float:
+    """Whole-job decode throughput: B tokens per step on every rank."""
+    return world * B * steps / (ms_total / 1e3)
+
+
 def kv_bytes_per_seq():
     return HKV * (P + W) * D * 2 * 2          # K and V rows, bf16
 
@@ -136,7 +156,7 @@ class Workload:
 
         self.torch = torch
         self.S = B * ROT
-        self.seed = SEED + 1000 * rank
+        self.seed = rank_seed(rank)
         self.kscale = synth.chan_scale(self.seed, HKV, D)
         self.cache = Cache(W, P, HKV, D, PS_BF16, self.S)
         self.scale = 1.0 / math.sqrt(D)
@@ -273,14 +293,11 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     ms_total = e0.elapsed_time(e1)
     del g
-    if dist:
-        t = torch.tensor([ms_total], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, dist, "cuda")
     clk = clocks.stop() if clocks else None
     _check_device(wl)
     ms_step = ms_total / K
-    value = world * B * K / (ms_total / 1e3)
+    value = job_tokens_per_s(world, K, ms_total)
 
     # ---- dominant kernel (decode) timed on its own stream, rotating batches ----
     ms_dec = time_graph(torch, lambda i, st: wl.decode_only(i, st), max(K, 4 * ROT))
@@ -320,12 +337,9 @@ def run_ours(args, rank, world, local_rank):
     e1.record()
     torch.cuda.synchronize()
     ms_e2e = e0.elapsed_time(e1)
-    if dist:
-        t = torch.tensor([ms_e2e], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
+    ms_e2e = max_over_ranks(ms_e2e, dist, "cuda")
     _check_device(wl)
-    e2e_value = world * B * K / (ms_e2e / 1e3)
+    e2e_value = job_tokens_per_s(world, K, ms_e2e)
     h2d = (B * HKV * D * 2) * 2 + B * HQ * D * 2
     d2h = B * HQ * D * 2
 
