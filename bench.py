@@ -78,6 +78,24 @@ def kv_bytes_per_step():
     return B * kv_bytes_per_seq()
 
 
+def decode_traffic():
+    """DRAM bytes per decode launch from the committed ncu record, or None when
+    the decode kernel's sources have changed since that capture."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    h = hashlib.sha256()
+    for src in rec["sources"]:
+        with open(os.path.join(ROOT, src), "rb") as f:
+            h.update(f.read())
+    if h.hexdigest() != rec["sources_sha256"]:
+        return None
+    return rec["dram_bytes_read_per_launch"] + rec["dram_bytes_write_per_launch"]
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -367,7 +385,7 @@ def run_ours(args, rank, world, local_rank):
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_source": peak_kind,
                      "bytes_per_launch": bytes_launch, "ms_per_launch": round(ms_dec, 5),
-                     "traffic": None},
+                     "traffic": decode_traffic()},
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": 2 * K,
@@ -425,9 +443,18 @@ def prefill_measure(steps: int):
             blocks.append((q, kb, vb, torch.empty_like(q)))
         scale = 1.0 / math.sqrt(D)
 
+        side = [torch.cuda.Stream() for _ in blocks]
+
         def step(i, st=None):
+            # The sequences are independent: one stream each, joined at the end,
+            # so their CTAs fill the GPU together (one sequence is 1.7 waves).
+            st = st or torch.cuda.current_stream()
+            for ss in side:
+                ss.wait_stream(st)
             for s, (q, kb, vb, o) in enumerate(blocks):
-                c.attend_chunk(s, q, kb, vb, PF_T0, PF_N, HQ, scale, o, 0, st)
+                c.attend_chunk(s, q, kb, vb, PF_T0, PF_N, HQ, scale, o, 0, side[s])
+            for ss in side:
+                st.wait_stream(ss)
 
         for i in range(3):
             step(i)
