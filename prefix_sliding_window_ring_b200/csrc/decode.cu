@@ -9,7 +9,7 @@
 // into the output.
 //
 // Streaming.  Warp kCW is the producer: one lane issues bulk async copies
-// (cp.async.bulk, no multicast) of contiguous K and V row tiles of 16 KiB each
+// (cp.async.bulk, no multicast) of contiguous K and V row tiles of 14 KiB each
 // into a kStages-deep shared-memory ring (bulk copies much smaller than that
 // leave HBM bandwidth unused).  A tile never crosses a visible range (prefix
 // rows, or one contiguous run of ring slots split at the physical wrap), so no
@@ -39,8 +39,8 @@
 #ifndef PS_DEC_STAGES
 #define PS_DEC_STAGES 3
 #endif
-#ifndef PS_DEC_TILE_BYTES
-#define PS_DEC_TILE_BYTES 16384
+#ifndef PS_DEC_WARP_BYTES
+#define PS_DEC_WARP_BYTES 2048
 #endif
 #ifndef PS_DEC_CTAS_PER_SM
 #define PS_DEC_CTAS_PER_SM 2
@@ -53,8 +53,12 @@ namespace {
 using namespace attn;
 
 #ifndef PS_DEC_CONSUMER_WARPS
-#define PS_DEC_CONSUMER_WARPS 8
+#define PS_DEC_CONSUMER_WARPS 7
 #endif
+// 7 consumer warps + 1 producer: 8 warps per CTA.  Warps are spread over the
+// four SM sub-partitions, each with its own quarter of the register file, so
+// two CTAs of 9 warps would put 5 warps on one sub-partition and only one CTA
+// would fit; with 8 warps two CTAs of up to 128 registers fit.
 constexpr int kCW = PS_DEC_CONSUMER_WARPS;   // consumer warps
 constexpr int kThreadsDec = (kCW + 1) * 32;  // plus one producer warp
 // Tile i sits in stage i % kStages.  Every consumer warp waits on every tile
@@ -66,9 +70,8 @@ constexpr int kMinRowsPerCta = 128;
 constexpr int kPieceBatch = 8;  // partials read together by the pair merge
 
 template <typename T, int D> struct DecTile {
-  static constexpr int TR = PS_DEC_TILE_BYTES / (D * (int)sizeof(T));  // rows per tile
-  static constexpr int RW = TR / kCW;                                    // rows per warp
-  static_assert(TR % kCW == 0, "tile rows must split evenly over the consumer warps");
+  static constexpr int RW = PS_DEC_WARP_BYTES / (D * (int)sizeof(T));  // rows per warp per tile
+  static constexpr int TR = RW * kCW;                                  // rows per tile (14 KiB)
 };
 
 struct DecodeArgs {
@@ -549,6 +552,9 @@ cudaError_t launch_kernel(int nctas, const DecodeArgs& a, cudaStream_t st) {
   if (!(configured.load() & bit)) {
     e = cudaFuncSetAttribute(k_decode<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)dyn);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(k_decode<T, D, G>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
