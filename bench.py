@@ -166,7 +166,7 @@ class ClockSampler:
 class Workload:
     """Sequences, their synthetic histories and per-step inputs on one GPU."""
 
-    def __init__(self, rank: int, steps_needed: int):
+    def __init__(self, rank: int, steps_needed: int, prefix: int = P):
         import torch
 
         import synth
@@ -176,7 +176,8 @@ class Workload:
         self.S = B * ROT
         self.seed = rank_seed(rank)
         self.kscale = synth.chan_scale(self.seed, HKV, D)
-        self.cache = Cache(W, P, HKV, D, PS_BF16, self.S)
+        self.P = prefix
+        self.cache = Cache(W, max(prefix, 1), HKV, D, PS_BF16, self.S)
         self.scale = 1.0 / math.sqrt(D)
 
         def dev(a):
@@ -184,10 +185,10 @@ class Workload:
 
         self.dev = dev
         for s in range(self.S):
-            kp = synth.rows(self.seed, synth.TID_K, s, HKV, 0, P, D, "bf16", self.kscale)
-            vp = synth.rows(self.seed, synth.TID_V, s, HKV, 0, P, D, "bf16")
+            kp = synth.rows(self.seed, synth.TID_K, s, HKV, 0, prefix, D, "bf16", self.kscale)
+            vp = synth.rows(self.seed, synth.TID_V, s, HKV, 0, prefix, D, "bf16")
             self.cache.seq_reset(s, (s * 613) % W)
-            self.cache.prefill_prefix(s, dev(kp), dev(vp), P)
+            self.cache.prefill_prefix(s, dev(kp), dev(vp), prefix)
             t0 = T_START + s  # staggered positions
             kw = synth.rows(self.seed, synth.TID_K, s, HKV, t0 - W, W, D, "bf16", self.kscale)
             vw = synth.rows(self.seed, synth.TID_V, s, HKV, t0 - W, W, D, "bf16")
@@ -323,6 +324,26 @@ def run_ours(args, rank, world, local_rank):
     achieved = bytes_launch / (ms_dec / 1e3) / 1e9
     peak, peak_kind = load_peaks()
 
+    # ---- prefix overhead: the same decode with no pinned prefix (plain sliding window) ----
+    overhead = None
+    if rank == 0 and not args.no_prefill:
+        wl0 = Workload(rank, 4, prefix=0)
+        for i in range(4):
+            wl0.decode_only(i)
+        torch.cuda.synchronize()
+        ms0 = time_graph(torch, lambda i, st: wl0.decode_only(i, st), max(K, 4 * ROT))
+        _check_device(wl0)
+        bytes0 = B * HKV * W * D * 2 * 2
+        overhead = {"note": "decode kernel, same W and batch; P=0 is plain sliding-window attention",
+                    "P128": {"us_per_launch": round(ms_dec * 1e3, 2), "visible_rows": P + W,
+                             "GBps": round(achieved, 1)},
+                    "P0": {"us_per_launch": round(ms0 * 1e3, 2), "visible_rows": W,
+                           "GBps": round(bytes0 / (ms0 / 1e3) / 1e9, 1)},
+                    "time_ratio": round(ms_dec / ms0, 4)}
+        wl0.cache.close()
+        del wl0
+        torch.cuda.empty_cache()
+
     # ---- end to end through the public API with host buffers ----
     def host_inputs(r, v):
         return hk[r][v], hv[r][v], hq[r][v]
@@ -392,6 +413,7 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk,
         "cpu_baseline": cpu,
         "prefill": prefill,
+        "prefix_overhead": overhead,
     }
     print(json.dumps(line), flush=True)
 

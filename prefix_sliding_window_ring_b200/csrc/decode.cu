@@ -2,11 +2,12 @@
 //
 // Work division.  The visible rows of all (batch entry, kv head) pairs of a
 // launch are laid end to end and cut into `nctas` equal ranges, one per CTA
-// (a multiple of the SM count), so every SM streams the same number of rows
-// whatever the batch shape.  A CTA walks the pairs its range touches; for each
-// it emits one partial (max, sum, accumulator) triple, and the last CTA to
-// finish a pair -- an atomic ticket, no spinning -- merges the pair's partials
-// into the output.
+// (two CTAs per SM), so every SM streams the same number of rows whatever the
+// batch shape.  For every (range, pair) piece a CTA emits one partial (max,
+// sum, accumulator) triple, and the last CTA to finish a pair -- an atomic
+// ticket, no spinning -- merges the pair's partials into the output.  The
+// producer hands each tile to the consumers with a small descriptor (pair,
+// rows, first/last of piece) next to the tile's data.
 //
 // Streaming.  Warp kCW is the producer: one lane issues bulk async copies
 // (cp.async.bulk, no multicast) of contiguous K and V row tiles of 14 KiB each
@@ -66,7 +67,6 @@ constexpr int kThreadsDec = (kCW + 1) * 32;  // plus one producer warp
 // the one it needs (where the parity test would accept the older phase).
 constexpr int kStages = PS_DEC_STAGES;
 constexpr long long kWaitLimitCycles = 1ll << 30;  // about half a second
-constexpr int kMinRowsPerCta = 128;
 constexpr int kPieceBatch = 8;  // partials read together by the pair merge
 
 template <typename T, int D> struct DecTile {
@@ -80,26 +80,14 @@ struct DecodeArgs {
   void* out;
   float qscale;
   int Hq, B, nctas;
-  int64_t total;    // visible rows of all pairs of the launch
-  float* part_ml;   // [nctas + B*Hkv][G][2]: per (pair, CTA) piece (max, sum), base 2
-  float* part_o;    // [nctas + B*Hkv][G][D]: per piece unnormalised accumulators
-  int32_t* tick;    // [B*Hkv] arrival counters, 0 at rest
+  int64_t total;       // visible rows of all pairs of the launch
+  float* part_ml;      // [nctas + B*Hkv][G][2]: per (CTA range, pair) piece (max, sum), base 2
+  float* part_o;       // [nctas + B*Hkv][G][D]: per piece unnormalised accumulators
+  int32_t* tick;       // [B*Hkv] pieces finished per pair, 0 at rest
   int32_t seq[kMaxBatchPerLaunch];
   int64_t t[kMaxBatchPerLaunch];
   int64_t cum[kMaxBatchPerLaunch + 1];  // cum[b] = Hkv * (rows of entries before b)
 };
-
-__device__ __forceinline__ int64_t range_start(int64_t c, int64_t R, int64_t NC) {
-  return R * c / NC;
-}
-// CTA whose range holds row x: the largest c with range_start(c) <= x.
-__device__ __forceinline__ int64_t cta_of_row(int64_t x, int64_t R, int64_t NC) {
-  return ((x + 1) * NC - 1) / R;
-}
-
-__device__ __forceinline__ void cbar() {  // the consumer warps only
-  asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory");
-}
 
 __device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0,
                                       float b1) {
@@ -308,36 +296,6 @@ struct DecState {
   }
 };
 
-// Merge the kCW consumer warps' states into slot 0 (consumer threads only).
-template <int G, int D>
-__device__ __forceinline__ void merge_consumers(MergeSmem<G, D, kCW>& sm) {
-  cbar();
-  if (threadIdx.x < G) {
-    const int h = threadIdx.x;
-    float mx = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kCW; ++w) mx = fmaxf(mx, sm.m[w][h]);
-    float l = 0.f;
-#pragma unroll
-    for (int w = 0; w < kCW; ++w) {
-      const float a = (mx == -INFINITY) ? 0.f : exp2f(sm.m[w][h] - mx);
-      sm.wt[w][h] = a;
-      l += sm.l[w][h] * a;
-    }
-    sm.m[0][h] = mx;
-    sm.l[0][h] = l;
-  }
-  cbar();
-  for (int idx = threadIdx.x; idx < G * D; idx += kCW * 32) {
-    const int h = idx / D, e = idx % D;
-    float acc = 0.f;
-#pragma unroll
-    for (int w = 0; w < kCW; ++w) acc += sm.o[w][h][e] * sm.wt[w][h];
-    sm.o[0][h][e] = acc;
-  }
-  cbar();
-}
-
 // Calls f(slab_row, nrows) for the tiles of the logical rows [jb, je) of one
 // pair: split at visible-range boundaries and every TR rows.  Registers only.
 // Sets *bad if the range reaches block rows (a decode query never does).
@@ -385,25 +343,47 @@ __device__ __forceinline__ PairPiece piece_at(const DecodeArgs& a, int64_t r, in
   return pp;
 }
 
+// One tile as the producer hands it to the consumers (through shared memory,
+// published by the mbarrier arrive that also carries the tile's bytes).
+struct TileDesc {
+  int32_t pair, nrows, flags;
+};
+
+// First flattened row of CTA c's range, and the CTA whose range holds row x.
+__device__ __forceinline__ int64_t range_start(int64_t c, int64_t R, int64_t NC) {
+  return R * c / NC;
+}
+__device__ __forceinline__ int64_t cta_of_row(int64_t x, int64_t R, int64_t NC) {
+  return ((x + 1) * NC - 1) / R;
+}
+enum : int32_t { TD_FIRST = 1, TD_LAST = 2, TD_END = 4 };
+
 template <typename T, int D, int G>
-__global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8) k_decode(const __grid_constant__ DecodeArgs a) {
+__global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8)
+    k_decode(const __grid_constant__ DecodeArgs a) {
   constexpr int TR = DecTile<T, D>::TR;
+  constexpr int RW = DecTile<T, D>::RW;
   extern __shared__ __align__(128) unsigned char dsm[];
   T* ktile = (T*)dsm;                           // [kStages][TR][D]
   T* vtile = ktile + (size_t)kStages * TR * D;  // [kStages][TR][D]
   __shared__ __align__(8) uint64_t full[kStages], empty[kStages];
+  __shared__ __align__(8) uint64_t sync_a, sync_b, sync_c;
+  __shared__ TileDesc desc[kStages];
   __shared__ int abort_flag;
   __shared__ int is_last;
   __shared__ MergeSmem<G, D, kCW> sm;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t NC = a.nctas, R = a.total;
-  const int64_t r0 = range_start(blockIdx.x, R, NC), r1 = range_start(blockIdx.x + 1, R, NC);
+  const int Hkv = a.c.Hkv;
+  const int64_t R = a.total, NC = a.nctas;
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
       ptx::mbar_init(&full[i], 1);
       ptx::mbar_init(&empty[i], kCW);
     }
+    ptx::mbar_init(&sync_a, kCW);
+    ptx::mbar_init(&sync_b, kCW);
+    ptx::mbar_init(&sync_c, 1);
     abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -412,29 +392,58 @@ __global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8) 
   if (warp == kCW) {
     if (lane != 0) return;
     // ------------------------------------------------------------ producer --
-    int i = 0;
-    for (int64_t r = r0; r < r1 && !abort_flag;) {
+    int i = 0;  // tiles handed out so far
+    auto put = [&](const TileDesc& d, const T* ksrc, const T* vsrc) -> bool {
+      const int st = i % kStages;
+      if (i >= kStages && !ptx::mbar_wait_bounded(&empty[st], ((i / kStages) - 1) & 1,
+                                                  &abort_flag, kWaitLimitCycles))
+        return false;
+      desc[st] = d;
+      if (d.flags & TD_END) {
+        ptx::mbar_arrive(&full[st]);
+      } else {
+        const uint32_t bytes = (uint32_t)d.nrows * D * sizeof(T);
+        ptx::mbar_arrive_expect_tx(&full[st], 2 * bytes);
+        ptx::bulk_g2s(ktile + (size_t)st * TR * D, ksrc, bytes, &full[st]);
+        ptx::bulk_g2s(vtile + (size_t)st * TR * D, vsrc, bytes, &full[st]);
+      }
+      ++i;
+      return true;
+    };
+    bool alive = true;
+    int64_t r = range_start(blockIdx.x, R, NC);
+    const int64_t r1 = range_start(blockIdx.x + 1, R, NC);
+    while (r < r1 && alive) {
       const PairPiece pp = piece_at(a, r, r1);
       r = pp.start + pp.hi;
       const int s = a.seq[pp.b];
       const DevMeta m = a.c.meta[s];
-      const SegSet segs = build_segments(m, a.c.W, a.c.P_max, m.next_pos - 1);
+      const int64_t t = m.next_pos - 1;
+      const SegSet segs = build_segments(m, a.c.W, a.c.P_max, t);
       bool bad = false;
-      const size_t slab = ((size_t)s * a.c.Hkv + pp.g) * (size_t)a.c.slab_rows * D;
-      for_each_tile(segs, pp.lo, min(pp.hi, segs.total), TR, &bad, [&](int64_t row, int nr) {
-        if (abort_flag) return;
-        const int st = i % kStages;
-        if (i >= kStages && !ptx::mbar_wait_bounded(&empty[st], ((i / kStages) - 1) & 1,
-                                                    &abort_flag, kWaitLimitCycles))
-          return;
-        const uint32_t bytes = (uint32_t)nr * D * sizeof(T);
-        ptx::mbar_arrive_expect_tx(&full[st], 2 * bytes);
-        ptx::bulk_g2s(ktile + (size_t)st * TR * D, (const T*)a.c.K + slab + (size_t)row * D,
-                      bytes, &full[st]);
-        ptx::bulk_g2s(vtile + (size_t)st * TR * D, (const T*)a.c.V + slab + (size_t)row * D,
-                      bytes, &full[st]);
-        ++i;
+      if (t != a.t[pp.b] || segs.total != pp.n || !segs.ring_ok) atomicOr(a.c.err, ERR_BATCH);
+      const size_t slab = ((size_t)s * Hkv + pp.g) * (size_t)a.c.slab_rows * D;
+      const int32_t hi = min(pp.hi, segs.total);
+      int ntiles = 0;
+      for_each_tile(segs, pp.lo, hi, TR, &bad, [&](int64_t, int) { ++ntiles; });
+      int k = 0;
+      const int pair = pp.b * Hkv + pp.g;
+      for_each_tile(segs, pp.lo, hi, TR, &bad, [&](int64_t row, int nr) {
+        if (!alive) return;
+        TileDesc d;
+        d.pair = pair;
+        d.nrows = nr;
+        d.flags = (k == 0 ? TD_FIRST : 0) | (k == ntiles - 1 ? TD_LAST : 0);
+        alive = put(d, (const T*)a.c.K + slab + (size_t)row * D,
+                    (const T*)a.c.V + slab + (size_t)row * D);
+        ++k;
       });
+      if (bad) atomicOr(a.c.err, ERR_BATCH);
+    }
+    if (alive) {
+      TileDesc end;
+      end.pair = 0; end.nrows = 0; end.flags = TD_END;
+      put(end, nullptr, nullptr);
     }
     if (abort_flag) {  // let the copies already issued land before the CTA exits
       int quiet = 0;
@@ -445,64 +454,80 @@ __global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8) 
   }
 
   // -------------------------------------------------------------- consumers --
-  int i = 0;  // tiles consumed so far (all consumer warps see every tile)
-  for (int64_t r = r0; r < r1;) {
-    const PairPiece pp = piece_at(a, r, r1);
-    r = pp.start + pp.hi;
-    const int s = a.seq[pp.b];
-    const DevMeta m = a.c.meta[s];
-    const int64_t t = m.next_pos - 1;
-    const SegSet segs = build_segments(m, a.c.W, a.c.P_max, t);
-    DecState<T, D, G> st;
-    st.init((const T*)a.q + ((size_t)pp.b * a.Hq + (size_t)pp.g * G) * D, a.qscale);
-    constexpr int RW = DecTile<T, D>::RW;
-    bool bad = false, stop = false;
-    for_each_tile(segs, pp.lo, min(pp.hi, segs.total), TR, &bad, [&](int64_t, int nr) {
-      if (stop) return;
-      const int stg = i % kStages;
-      const bool ok = ptx::mbar_wait_bounded(&full[stg], (i / kStages) & 1, &abort_flag,
-                                             kWaitLimitCycles);
-      if (!__all_sync(0xffffffffu, ok)) {
-        stop = true;
-        return;
-      }
-      const int mine = min(RW, nr - warp * RW);  // this warp's rows of the tile
-      if (mine > 0)
-        st.tile(ktile + ((size_t)stg * TR + warp * RW) * D,
-                vtile + ((size_t)stg * TR + warp * RW) * D, mine);
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&empty[stg]);
-      ++i;
-    });
-    if (threadIdx.x == 0) {
-      if (t != a.t[pp.b] || segs.total != pp.n || bad) atomicOr(a.c.err, ERR_BATCH);
-      if (!segs.ring_ok) atomicOr(a.c.err, ERR_RING);
-    }
-    st.to_smem(sm, warp);
-    merge_consumers<G, D>(sm);
+  // The piece epilogue synchronises the consumer warps with three mbarriers
+  // (bounded waits, one phase per piece) rather than a named barrier, so a
+  // warp that gives up can never leave the others waiting for good.
+  DecState<T, D, G> st;
+  int np = 0;  // pieces finished by this CTA
+  for (int i = 0;; ++i) {
+    const int stg = i % kStages;
+    const bool ok = ptx::mbar_wait_bounded(&full[stg], (i / kStages) & 1, &abort_flag,
+                                           kWaitLimitCycles);
+    if (!__all_sync(0xffffffffu, ok)) break;
+    const TileDesc d = desc[stg];
+    if (d.flags & TD_END) break;
+    const int b = d.pair / Hkv, g = d.pair % Hkv;
+    if (d.flags & TD_FIRST)
+      st.init((const T*)a.q + ((size_t)b * a.Hq + (size_t)g * G) * D, a.qscale);
+    const int mine = min(RW, d.nrows - warp * RW);  // this warp's rows of the tile
+    if (mine > 0)
+      st.tile(ktile + ((size_t)stg * TR + warp * RW) * D,
+              vtile + ((size_t)stg * TR + warp * RW) * D, mine);
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(&empty[stg]);
+    if (!(d.flags & TD_LAST)) continue;
 
-    // publish this piece, then merge the pair if this CTA is the last to finish it
-    const int pair = pp.b * a.c.Hkv + pp.g;
-    const int64_t slot = (int64_t)blockIdx.x + pair;
+    // ---- end of a (chunk, pair) piece ----
+    const uint32_t par = np & 1;
+    ++np;
+    st.to_smem(sm, warp);  // this warp's (max, sum, accumulator) into sm[warp]
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(&sync_a);
+    if (!__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&sync_a, par, &abort_flag,
+                                                         kWaitLimitCycles)))
+      break;
+    // merge the warps straight into this piece's partial slot
+    const int64_t slot = (int64_t)blockIdx.x + d.pair;  // unique per (CTA range, pair)
     float* pml = a.part_ml + (size_t)slot * G * 2;
     float* po = a.part_o + (size_t)slot * G * D;
-    for (int idx = threadIdx.x; idx < G * D; idx += kCW * 32) po[idx] = sm.o[0][idx / D][idx % D];
-    if (threadIdx.x < G) {
-      pml[threadIdx.x * 2] = sm.m[0][threadIdx.x];
-      pml[threadIdx.x * 2 + 1] = sm.l[0][threadIdx.x];
+    for (int idx = threadIdx.x; idx < G * D; idx += kCW * 32) {
+      const int h = idx / D, e = idx % D;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kCW; ++w) mx = fmaxf(mx, sm.m[w][h]);
+      float l = 0.f, acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < kCW; ++w) {
+        const float wt = (mx == -INFINITY) ? 0.f : exp2f(sm.m[w][h] - mx);
+        l += sm.l[w][h] * wt;
+        acc += sm.o[w][h][e] * wt;
+      }
+      po[idx] = acc;
+      if (e == 0) {
+        pml[h * 2] = mx;
+        pml[h * 2 + 1] = l;
+      }
     }
     __threadfence();
-    cbar();
-    const int64_t first = cta_of_row(pp.start, R, NC);
-    const int64_t last = cta_of_row(pp.start + pp.n - 1, R, NC);
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(&sync_b);
+    if (!__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&sync_b, par, &abort_flag,
+                                                         kWaitLimitCycles)))
+      break;
+    const int64_t n = (a.cum[b + 1] - a.cum[b]) / Hkv;
+    const int64_t pstart = a.cum[b] + (int64_t)g * n;
+    const int64_t first = cta_of_row(pstart, R, NC), last = cta_of_row(pstart + n - 1, R, NC);
     if (threadIdx.x == 0) {
-      const int old = atomicAdd(&a.tick[pair], 1);
+      const int old = atomicAdd(&a.tick[d.pair], 1);
       is_last = (old == (int)(last - first));
+      ptx::mbar_arrive(&sync_c);
     }
-    cbar();
-    if (is_last) {
+    if (!__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&sync_c, par, &abort_flag,
+                                                         kWaitLimitCycles)))
+      break;
+    if (is_last) {  // every piece of the pair is published: merge them into the output
       __threadfence();
-      T* orow = (T*)a.out + ((size_t)pp.b * a.Hq + (size_t)pp.g * G) * D;
+      T* orow = (T*)a.out + ((size_t)b * a.Hq + (size_t)g * G) * D;
       for (int idx = threadIdx.x; idx < G * D; idx += kCW * 32) {
         const int h = idx / D, e = idx % D;
         // online merge of the pieces, kPieceBatch independent loads at a time
@@ -511,7 +536,7 @@ __global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8) 
           float mj[kPieceBatch], lj[kPieceBatch], oj[kPieceBatch];
 #pragma unroll
           for (int j = 0; j < kPieceBatch; ++j) {
-            const int64_t sl = c0 + j + pair;
+            const int64_t sl = c0 + j + d.pair;
             const bool in = c0 + j <= last;
             mj[j] = in ? __ldcg(a.part_ml + ((size_t)sl * G + h) * 2) : -INFINITY;
             lj[j] = in ? __ldcg(a.part_ml + ((size_t)sl * G + h) * 2 + 1) : 0.f;
@@ -534,9 +559,8 @@ __global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8) 
         }
         store_out<T>(orow + (size_t)h * D + e, A / L);
       }
-      if (threadIdx.x == 0) a.tick[pair] = 0;
+      if (threadIdx.x == 0) a.tick[d.pair] = 0;
     }
-    cbar();
   }
   if (threadIdx.x == 0 && abort_flag) atomicOr(a.c.err, ERR_TIMEOUT);
 }
@@ -576,13 +600,14 @@ cudaError_t dispatch_G(int G, int nctas, const DecodeArgs& a, cudaStream_t st) {
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 int max_ctas(int sm_count) { return sm_count * PS_DEC_CTAS_PER_SM; }
+constexpr int kMinRowsPerCta = 128;
 
 }  // namespace
 
 DecodeWs decode_ws_layout(void* ws, int B, int Hkv, int G, int d, int sm_count, size_t* bytes) {
   const int Bl = B < kMaxBatchPerLaunch ? B : kMaxBatchPerLaunch;  // launches run in turn
   const size_t pairs = (size_t)Bl * Hkv;
-  const size_t slots = (size_t)max_ctas(sm_count) + pairs;
+  const size_t slots = (size_t)max_ctas(sm_count) + pairs;  // (CTA range, pair) pieces
   const size_t tick = align256(pairs * sizeof(int32_t));
   const size_t ml = align256(slots * G * 2 * sizeof(float));
   const size_t o = align256(slots * G * d * sizeof(float));
