@@ -135,9 +135,13 @@ PS_API size_t ps_decode_workspace_bytes(const ps_cache* c, int B, int Hq);
  * out[b][h] = sum over visible p of softmax_p(scale * <q[b][h], k_p>) v_p,
  * computed in float32 (bf16 inputs are widened exactly; the bf16 output is
  * rounded to nearest even).  Evicted positions are never read.
- * workspace: device, >= ps_decode_workspace_bytes(c, B, Hq) bytes, zero-filled
- * before its first use; every call leaves it ready for the next.  Calls that
- * share a workspace must not overlap on the GPU.
+ * workspace: device, >= ps_decode_workspace_bytes(c, B, Hq) bytes, any
+ * contents (it holds split partial results within one call, no state between
+ * calls).  Calls that share a workspace must not overlap on the GPU.
+ * The ring state (P, head, count) of each entry is taken from the library's
+ * host bookkeeping at enqueue time; the kernel compares it with the device
+ * record and sets the device error bit 4 (see ps_device_error) if they differ,
+ * as happens when an append on another stream was not ordered before this call.
  * Hq must be a multiple of Hkv with Hq/Hkv in {1, 2, 4, 8}.
  * Errors: PS_EINVAL, PS_ESTATE, PS_EPOS, PS_ENOMEM, PS_EUNSUPPORTED. */
 PS_API int ps_attend_decode(ps_cache* c, const void* q, const int* seq_ids, const int64_t* t,
@@ -208,7 +212,13 @@ PS_API int ps_debug_visible(ps_cache* c, int seq, int64_t t, int64_t* pos_out, i
                      void* stream);
 
 /* Synchronise `stream` and read (then clear) the device error word:
- * *code = 0 when no kernel reported an inconsistency.  Errors: PS_ECUDA. */
+ * *code = 0 when no kernel reported an inconsistency, else an OR of
+ *   1  a split launch did not cover every visible row,
+ *   2  a ring no longer holds the window a query needs,
+ *   4  a batch entry's position or ring state disagrees with the device record,
+ *   8  a pipeline wait gave up and the kernel stopped early (outputs of that
+ *      call are undefined).
+ * Errors: PS_ECUDA. */
 PS_API int ps_device_error(ps_cache* c, int32_t* code, void* stream);
 
 /* Message of the last failed call in this thread ("" if none). */

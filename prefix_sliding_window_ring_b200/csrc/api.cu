@@ -309,7 +309,10 @@ int ps_attend_decode(ps_cache* c, const void* q, const int* seq_ids, const int64
     ps::BatchIds ids;
     memset(&ids, 0, sizeof(ids));
     for (int i = 0; i < nb; ++i) {
+      const SeqHost& s = c->seqs[seq_ids[b0 + i]];
       ids.seq[i] = seq_ids[b0 + i];
+      ids.P[i] = s.P;
+      ids.head[i] = s.head;
       ids.t[i] = t[b0 + i];
     }
     PS_CUDA(ps::launch_decode(c->dev, c->dtype, G, ids, rows.data() + b0, nb, Hq,

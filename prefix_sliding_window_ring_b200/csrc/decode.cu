@@ -4,10 +4,12 @@
 // launch are laid end to end and cut into `nctas` equal ranges, one per CTA
 // (two CTAs per SM), so every SM streams the same number of rows whatever the
 // batch shape.  For every (range, pair) piece a CTA emits one partial (max,
-// sum, accumulator) triple, and the last CTA to finish a pair -- an atomic
-// ticket, no spinning -- merges the pair's partials into the output.  The
+// sum, accumulator) triple; a small second grid, launched as a programmatic
+// dependent of the first, merges each pair's partials into the output.  The
 // producer hands each tile to the consumers with a small descriptor (pair,
-// rows, first/last of piece) next to the tile's data.
+// rows, first/last of piece) next to the tile's data.  The ring state of each
+// entry (P, head, count) comes with the launch from the host's bookkeeping, so
+// no copy waits on a metadata load; the device record is checked alongside.
 //
 // Streaming.  Warp kCW is the producer: one lane issues bulk async copies
 // (cp.async.bulk, no multicast) of contiguous K and V row tiles of 14 KiB each
@@ -23,8 +25,8 @@
 // each lane forms partial dot products for 8 (row, query head) scores, a
 // transpose-reduction leaves every lane with one complete score, the lane
 // exponentiates only that score, and the 8 weights are gathered back for the
-// weighted sum of the value rows.  Pairs of float32 lanes use the packed
-// fma.rn.f32x2 instruction (each half is an ordinary IEEE fma).
+// weighted sum of the value rows.  Pairs of float32 values use the packed
+// sm_100 FMA (each half is an ordinary IEEE fma).
 //
 // Every wait is bounded; a time-out stops the CTA, sets ERR_TIMEOUT and lets
 // the copies already issued land before the CTA exits.
@@ -68,6 +70,7 @@ constexpr int kThreadsDec = (kCW + 1) * 32;  // plus one producer warp
 constexpr int kStages = PS_DEC_STAGES;
 constexpr long long kWaitLimitCycles = 1ll << 30;  // about half a second
 constexpr int kPieceBatch = 8;  // partials read together by the pair merge
+constexpr int kMergeThreads = 128;
 
 template <typename T, int D> struct DecTile {
   static constexpr int RW = PS_DEC_WARP_BYTES / (D * (int)sizeof(T));  // rows per warp per tile
@@ -83,38 +86,38 @@ struct DecodeArgs {
   int64_t total;       // visible rows of all pairs of the launch
   float* part_ml;      // [nctas + B*Hkv][G][2]: per (CTA range, pair) piece (max, sum), base 2
   float* part_o;       // [nctas + B*Hkv][G][D]: per piece unnormalised accumulators
-  int32_t* tick;       // [B*Hkv] pieces finished per pair, 0 at rest
   int32_t seq[kMaxBatchPerLaunch];
+  int32_t P[kMaxBatchPerLaunch];     // prefix length of entry b
+  int32_t head[kMaxBatchPerLaunch];  // physical ring slot of entry b's oldest window row
   int64_t t[kMaxBatchPerLaunch];
   int64_t cum[kMaxBatchPerLaunch + 1];  // cum[b] = Hkv * (rows of entries before b)
 };
+static_assert(sizeof(DecodeArgs) <= 4096, "decode arguments fit the classic parameter space");
 
-__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0,
-                                      float b1) {
-  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\t"
-      "mov.b64 rb, {%4, %5};\n\t"
-      "mov.b64 rd, {%0, %1};\n\t"
-      "fma.rn.f32x2 rd, ra, rb, rd;\n\t"
-      "mov.b64 {%0, %1}, rd;\n\t}"
-      : "+f"(d0), "+f"(d1)
-      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
-}
+// bfloat16 pairs of a 16-byte vector as float2 (exact widening).
+template <typename T> struct Vec2;
+template <> struct Vec2<uint16_t> {
+  __device__ __forceinline__ static void unpack(const uint4& x, float2* f) {
+    f[0] = make_float2(bf16lo(x.x), bf16hi(x.x));
+    f[1] = make_float2(bf16lo(x.y), bf16hi(x.y));
+    f[2] = make_float2(bf16lo(x.z), bf16hi(x.z));
+    f[3] = make_float2(bf16lo(x.w), bf16hi(x.w));
+  }
+};
+template <> struct Vec2<float> {
+  __device__ __forceinline__ static void unpack(const uint4& x, float2* f) {
+    f[0] = make_float2(__uint_as_float(x.x), __uint_as_float(x.y));
+    f[1] = make_float2(__uint_as_float(x.z), __uint_as_float(x.w));
+  }
+};
 
-__device__ __forceinline__ void fmul2(float& d0, float& d1, float a) {
-  asm("{\n\t.reg .b64 ra, rd;\n\t"
-      "mov.b64 ra, {%2, %2};\n\t"
-      "mov.b64 rd, {%0, %1};\n\t"
-      "mul.rn.f32x2 rd, rd, ra;\n\t"
-      "mov.b64 {%0, %1}, rd;\n\t}"
-      : "+f"(d0), "+f"(d1)
-      : "f"(a));
-}
-
-// Online-softmax state of one lane (see the file comment).
+// Online-softmax state of one lane (see the file comment).  Pairs of values
+// are float2 so the packed sm_100 FMA/MUL (__ffma2_rn, __fmul2_rn: two IEEE
+// operations each) apply directly.
 template <typename T, int D, int G>
 struct DecState {
   static constexpr int VEC = Vec<T>::N;
+  static constexpr int V2 = VEC / 2;
   static constexpr int LPR = D / VEC;   // lanes per row
   static constexpr int RPI = 32 / LPR;  // rows per warp load instruction
   static constexpr int U = 8 / G;       // rows per row group per update
@@ -122,8 +125,9 @@ struct DecState {
   static constexpr int S1 = LPR / 2, S2 = LPR / 4, S3 = LPR / 8;
   static_assert(LPR >= 8, "the transpose-reduction needs at least 8 lanes per row");
 
-  float q[G][VEC];
-  float m[G], o[G][VEC];
+  float2 q[G][V2];
+  float2 o[G][V2];
+  float m[G];
   float mo, lpart;  // running max and partial sum of this lane's own head
   int c, rs, base, kown;
 
@@ -137,15 +141,17 @@ struct DecState {
     rs = lane / LPR;
     base = rs * LPR;
     kown = ((c & S1) ? 4 : 0) | ((c & S2) ? 2 : 0) | ((c & S3) ? 1 : 0);
+    const float2 s2 = make_float2(qscale, qscale);
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       uint4 raw = *(const uint4*)(qrow + (size_t)h * D + c * VEC);
-      Vec<T>::unpack(raw, q[h]);
+      Vec2<T>::unpack(raw, q[h]);
 #pragma unroll
-      for (int e = 0; e < VEC; ++e) q[h][e] *= qscale;
+      for (int e = 0; e < V2; ++e) {
+        q[h][e] = __fmul2_rn(q[h][e], s2);
+        o[h][e] = make_float2(0.f, 0.f);
+      }
       m[h] = -INFINITY;
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) o[h][e] = 0.f;
     }
     mo = -INFINITY;
     lpart = 0.f;
@@ -159,14 +165,14 @@ struct DecState {
     float v[8];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      float kf[VEC];
-      Vec<T>::unpack(kr[u], kf);
+      float2 kf[V2];
+      Vec2<T>::unpack(kr[u], kf);
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        float a0 = 0.f, a1 = 0.f;
+        float2 acc = __fmul2_rn(q[h][0], kf[0]);
 #pragma unroll
-        for (int e = 0; e < VEC; e += 2) ffma2(a0, a1, q[h][e], q[h][e + 1], kf[e], kf[e + 1]);
-        v[u * G + h] = a0 + a1;
+        for (int e = 1; e < V2; ++e) acc = __ffma2_rn(q[h][e], kf[e], acc);
+        v[u * G + h] = acc.x + acc.y;
       }
     }
     // transpose-reduction: 8 values -> 1 complete score per lane
@@ -174,21 +180,21 @@ struct DecState {
       const bool b1 = (lane & S1) != 0;
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        float send = b1 ? v[k] : v[k + 4];
-        float keep = b1 ? v[k + 4] : v[k];
+        const float send = b1 ? v[k] : v[k + 4];
+        const float keep = b1 ? v[k + 4] : v[k];
         v[k] = keep + __shfl_xor_sync(FULL, send, S1);
       }
       const bool b2 = (lane & S2) != 0;
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
-        float send = b2 ? v[k] : v[k + 2];
-        float keep = b2 ? v[k + 2] : v[k];
+        const float send = b2 ? v[k] : v[k + 2];
+        const float keep = b2 ? v[k + 2] : v[k];
         v[k] = keep + __shfl_xor_sync(FULL, send, S2);
       }
       const bool b3 = (lane & S3) != 0;
       {
-        float send = b3 ? v[0] : v[1];
-        float keep = b3 ? v[1] : v[0];
+        const float send = b3 ? v[0] : v[1];
+        const float keep = b3 ? v[1] : v[0];
         v[0] = keep + __shfl_xor_sync(FULL, send, S3);
       }
 #pragma unroll
@@ -222,18 +228,20 @@ struct DecState {
 #pragma unroll
     for (int k = 0; k < 8; ++k) pk[k] = __shfl_sync(FULL, p, base | lane_of(k));
 #pragma unroll
-    for (int h = 0; h < G; ++h)
+    for (int h = 0; h < G; ++h) {
+      const float2 a2 = make_float2(alpha[h], alpha[h]);
 #pragma unroll
-      for (int e = 0; e < VEC; e += 2) fmul2(o[h][e], o[h][e + 1], alpha[h]);
+      for (int e = 0; e < V2; ++e) o[h][e] = __fmul2_rn(o[h][e], a2);
+    }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      float vf[VEC];
-      Vec<T>::unpack(vr[u], vf);
+      float2 vf[V2];
+      Vec2<T>::unpack(vr[u], vf);
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const float w = pk[u * G + h];
+        const float2 w2 = make_float2(pk[u * G + h], pk[u * G + h]);
 #pragma unroll
-        for (int e = 0; e < VEC; e += 2) ffma2(o[h][e], o[h][e + 1], w, w, vf[e], vf[e + 1]);
+        for (int e = 0; e < V2; ++e) o[h][e] = __ffma2_rn(w2, vf[e], o[h][e]);
       }
     }
   }
@@ -277,9 +285,10 @@ struct DecState {
         float mm, ll, a1, a2;
         merge_ml(m[h], l[h], m2, l2, mm, ll, a1, a2);
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) {
-          const float o2 = __shfl_xor_sync(FULL, o[h][e], off);
-          o[h][e] = o[h][e] * a1 + o2 * a2;
+        for (int e = 0; e < V2; ++e) {
+          const float ox = __shfl_xor_sync(FULL, o[h][e].x, off);
+          const float oy = __shfl_xor_sync(FULL, o[h][e].y, off);
+          o[h][e] = make_float2(o[h][e].x * a1 + ox * a2, o[h][e].y * a1 + oy * a2);
         }
         m[h] = mm;
         l[h] = ll;
@@ -290,7 +299,10 @@ struct DecState {
       for (int h = 0; h < G; ++h) {
         if (c == 0) { sm.m[warp][h] = m[h]; sm.l[warp][h] = l[h]; }
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) sm.o[warp][h][c * VEC + e] = o[h][e];
+        for (int e = 0; e < V2; ++e) {
+          sm.o[warp][h][c * VEC + 2 * e] = o[h][e].x;
+          sm.o[warp][h][c * VEC + 2 * e + 1] = o[h][e].y;
+        }
       }
     }
   }
@@ -347,6 +359,7 @@ __device__ __forceinline__ PairPiece piece_at(const DecodeArgs& a, int64_t r, in
 // published by the mbarrier arrive that also carries the tile's bytes).
 struct TileDesc {
   int32_t pair, nrows, flags;
+  int32_t slot;  // partial-result slot of the tile's piece: CTA range + pair
 };
 
 // First flattened row of CTA c's range, and the CTA whose range holds row x.
@@ -356,6 +369,7 @@ __device__ __forceinline__ int64_t range_start(int64_t c, int64_t R, int64_t NC)
 __device__ __forceinline__ int64_t cta_of_row(int64_t x, int64_t R, int64_t NC) {
   return ((x + 1) * NC - 1) / R;
 }
+
 enum : int32_t { TD_FIRST = 1, TD_LAST = 2, TD_END = 4 };
 
 template <typename T, int D, int G>
@@ -366,11 +380,11 @@ __global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8)
   extern __shared__ __align__(128) unsigned char dsm[];
   T* ktile = (T*)dsm;                           // [kStages][TR][D]
   T* vtile = ktile + (size_t)kStages * TR * D;  // [kStages][TR][D]
+  T* qtile = vtile + (size_t)kStages * TR * D;  // [kStages][G][D]: q of a piece's first tile
   __shared__ __align__(8) uint64_t full[kStages], empty[kStages];
-  __shared__ __align__(8) uint64_t sync_a, sync_b, sync_c;
+  __shared__ __align__(8) uint64_t sync_a, sync_b;
   __shared__ TileDesc desc[kStages];
   __shared__ int abort_flag;
-  __shared__ int is_last;
   __shared__ MergeSmem<G, D, kCW> sm;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -383,11 +397,12 @@ __global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8)
     }
     ptx::mbar_init(&sync_a, kCW);
     ptx::mbar_init(&sync_b, kCW);
-    ptx::mbar_init(&sync_c, 1);
     abort_flag = 0;
     ptx::fence_mbar_init();
   }
   __syncthreads();
+  // The merge grid may be scheduled now; it waits for this grid's completion.
+  ptx::pdl_launch_dependents();
 
   if (warp == kCW) {
     if (lane != 0) return;
@@ -402,8 +417,16 @@ __global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8)
       if (d.flags & TD_END) {
         ptx::mbar_arrive(&full[st]);
       } else {
+        // The first tile of a piece also brings the piece's G query rows, so
+        // no consumer waits on a global load of q when a piece starts.
         const uint32_t bytes = (uint32_t)d.nrows * D * sizeof(T);
-        ptx::mbar_arrive_expect_tx(&full[st], 2 * bytes);
+        const uint32_t qbytes = (d.flags & TD_FIRST) ? (uint32_t)(G * D * sizeof(T)) : 0u;
+        ptx::mbar_arrive_expect_tx(&full[st], 2 * bytes + qbytes);
+        if (qbytes) {
+          const int b = d.pair / Hkv, g = d.pair % Hkv;
+          ptx::bulk_g2s(qtile + (size_t)st * G * D,
+                        (const T*)a.q + ((size_t)b * a.Hq + (size_t)g * G) * D, qbytes, &full[st]);
+        }
         ptx::bulk_g2s(ktile + (size_t)st * TR * D, ksrc, bytes, &full[st]);
         ptx::bulk_g2s(vtile + (size_t)st * TR * D, vsrc, bytes, &full[st]);
       }
@@ -411,38 +434,50 @@ __global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8)
       return true;
     };
     bool alive = true;
-    int64_t r = range_start(blockIdx.x, R, NC);
-    const int64_t r1 = range_start(blockIdx.x + 1, R, NC);
-    while (r < r1 && alive) {
-      const PairPiece pp = piece_at(a, r, r1);
-      r = pp.start + pp.hi;
-      const int s = a.seq[pp.b];
-      const DevMeta m = a.c.meta[s];
-      const int64_t t = m.next_pos - 1;
-      const SegSet segs = build_segments(m, a.c.W, a.c.P_max, t);
-      bool bad = false;
-      if (t != a.t[pp.b] || segs.total != pp.n || !segs.ring_ok) atomicOr(a.c.err, ERR_BATCH);
-      const size_t slab = ((size_t)s * Hkv + pp.g) * (size_t)a.c.slab_rows * D;
-      const int32_t hi = min(pp.hi, segs.total);
-      int ntiles = 0;
-      for_each_tile(segs, pp.lo, hi, TR, &bad, [&](int64_t, int) { ++ntiles; });
-      int k = 0;
-      const int pair = pp.b * Hkv + pp.g;
-      for_each_tile(segs, pp.lo, hi, TR, &bad, [&](int64_t row, int nr) {
-        if (!alive) return;
-        TileDesc d;
-        d.pair = pair;
-        d.nrows = nr;
-        d.flags = (k == 0 ? TD_FIRST : 0) | (k == ntiles - 1 ? TD_LAST : 0);
-        alive = put(d, (const T*)a.c.K + slab + (size_t)row * D,
-                    (const T*)a.c.V + slab + (size_t)row * D);
-        ++k;
-      });
-      if (bad) atomicOr(a.c.err, ERR_BATCH);
-    }
+    // Streams the pieces of the rows [r, r1) of CTA range u.
+    auto run = [&](int64_t r, const int64_t r1, const int64_t u) {
+      while (r < r1 && alive) {
+        const PairPiece pp = piece_at(a, r, r1);
+        r = pp.start + pp.hi;
+        const int s = a.seq[pp.b];
+        // The ring state comes with the launch (the host's bookkeeping), so the
+        // copies start without a dependent global load; the device's own record
+        // is loaded alongside and compared once the piece's copies are issued.
+        const DevMeta md = a.c.meta[s];
+        DevMeta m;
+        m.next_pos = a.t[pp.b] + 1;
+        m.P = a.P[pp.b];
+        m.head = a.head[pp.b];
+        m.count = pp.n - m.P;
+        const SegSet segs = build_segments(m, a.c.W, a.c.P_max, a.t[pp.b]);
+        bool bad = false;
+        const size_t slab = ((size_t)s * Hkv + pp.g) * (size_t)a.c.slab_rows * D;
+        const int32_t hi = min(pp.hi, segs.total);
+        int ntiles = 0;
+        for_each_tile(segs, pp.lo, hi, TR, &bad, [&](int64_t, int) { ++ntiles; });
+        int k = 0;
+        const int pair = pp.b * Hkv + pp.g;
+        for_each_tile(segs, pp.lo, hi, TR, &bad, [&](int64_t row, int nr) {
+          if (!alive) return;
+          TileDesc d;
+          d.pair = pair;
+          d.nrows = nr;
+          d.flags = (k == 0 ? TD_FIRST : 0) | (k == ntiles - 1 ? TD_LAST : 0);
+          d.slot = (int32_t)(u + pair);
+          alive = put(d, (const T*)a.c.K + slab + (size_t)row * D,
+                      (const T*)a.c.V + slab + (size_t)row * D);
+          ++k;
+        });
+        if (bad || segs.total != pp.n || md.next_pos != m.next_pos || md.P != m.P ||
+            md.head != m.head || md.count != m.count)
+          atomicOr(a.c.err, ERR_BATCH);
+        if (!segs.ring_ok) atomicOr(a.c.err, ERR_RING);
+      }
+    };
+    run(range_start(blockIdx.x, R, NC), range_start(blockIdx.x + 1, R, NC), blockIdx.x);
     if (alive) {
       TileDesc end;
-      end.pair = 0; end.nrows = 0; end.flags = TD_END;
+      end.pair = 0; end.nrows = 0; end.flags = TD_END; end.slot = 0;
       put(end, nullptr, nullptr);
     }
     if (abort_flag) {  // let the copies already issued land before the CTA exits
@@ -454,9 +489,15 @@ __global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8)
   }
 
   // -------------------------------------------------------------- consumers --
-  // The piece epilogue synchronises the consumer warps with three mbarriers
-  // (bounded waits, one phase per piece) rather than a named barrier, so a
-  // warp that gives up can never leave the others waiting for good.
+  // The consumer warps synchronise with mbarriers (bounded waits, one phase
+  // per piece) rather than a named barrier, so a warp that gives up can never
+  // leave the others waiting for good.
+  auto csync = [&](uint64_t* bar, int phase) -> bool {
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(bar);
+    return __all_sync(0xffffffffu,
+                      ptx::mbar_wait_bounded(bar, phase & 1, &abort_flag, kWaitLimitCycles));
+  };
   DecState<T, D, G> st;
   int np = 0;  // pieces finished by this CTA
   for (int i = 0;; ++i) {
@@ -466,9 +507,7 @@ __global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8)
     if (!__all_sync(0xffffffffu, ok)) break;
     const TileDesc d = desc[stg];
     if (d.flags & TD_END) break;
-    const int b = d.pair / Hkv, g = d.pair % Hkv;
-    if (d.flags & TD_FIRST)
-      st.init((const T*)a.q + ((size_t)b * a.Hq + (size_t)g * G) * D, a.qscale);
+    if (d.flags & TD_FIRST) st.init(qtile + (size_t)stg * G * D, a.qscale);
     const int mine = min(RW, d.nrows - warp * RW);  // this warp's rows of the tile
     if (mine > 0)
       st.tile(ktile + ((size_t)stg * TR + warp * RW) * D,
@@ -477,17 +516,10 @@ __global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8)
     if (lane == 0) ptx::mbar_arrive(&empty[stg]);
     if (!(d.flags & TD_LAST)) continue;
 
-    // ---- end of a (chunk, pair) piece ----
-    const uint32_t par = np & 1;
-    ++np;
+    // ---- end of a (CTA range, pair) piece: publish its partial ----
     st.to_smem(sm, warp);  // this warp's (max, sum, accumulator) into sm[warp]
-    __syncwarp();
-    if (lane == 0) ptx::mbar_arrive(&sync_a);
-    if (!__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&sync_a, par, &abort_flag,
-                                                         kWaitLimitCycles)))
-      break;
-    // merge the warps straight into this piece's partial slot
-    const int64_t slot = (int64_t)blockIdx.x + d.pair;  // unique per (CTA range, pair)
+    if (!csync(&sync_a, np)) break;
+    const int64_t slot = d.slot;  // unique per (CTA range, pair)
     float* pml = a.part_ml + (size_t)slot * G * 2;
     float* po = a.part_o + (size_t)slot * G * D;
     for (int idx = threadIdx.x; idx < G * D; idx += kCW * 32) {
@@ -508,66 +540,73 @@ __global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8)
         pml[h * 2 + 1] = l;
       }
     }
-    __threadfence();
-    __syncwarp();
-    if (lane == 0) ptx::mbar_arrive(&sync_b);
-    if (!__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&sync_b, par, &abort_flag,
-                                                         kWaitLimitCycles)))
-      break;
-    const int64_t n = (a.cum[b + 1] - a.cum[b]) / Hkv;
-    const int64_t pstart = a.cum[b] + (int64_t)g * n;
-    const int64_t first = cta_of_row(pstart, R, NC), last = cta_of_row(pstart + n - 1, R, NC);
-    if (threadIdx.x == 0) {
-      const int old = atomicAdd(&a.tick[d.pair], 1);
-      is_last = (old == (int)(last - first));
-      ptx::mbar_arrive(&sync_c);
-    }
-    if (!__all_sync(0xffffffffu, ptx::mbar_wait_bounded(&sync_c, par, &abort_flag,
-                                                         kWaitLimitCycles)))
-      break;
-    if (is_last) {  // every piece of the pair is published: merge them into the output
-      __threadfence();
-      T* orow = (T*)a.out + ((size_t)b * a.Hq + (size_t)g * G) * D;
-      for (int idx = threadIdx.x; idx < G * D; idx += kCW * 32) {
-        const int h = idx / D, e = idx % D;
-        // online merge of the pieces, kPieceBatch independent loads at a time
-        float M = -INFINITY, L = 0.f, A = 0.f;
-        for (int64_t c0 = first; c0 <= last; c0 += kPieceBatch) {
-          float mj[kPieceBatch], lj[kPieceBatch], oj[kPieceBatch];
-#pragma unroll
-          for (int j = 0; j < kPieceBatch; ++j) {
-            const int64_t sl = c0 + j + d.pair;
-            const bool in = c0 + j <= last;
-            mj[j] = in ? __ldcg(a.part_ml + ((size_t)sl * G + h) * 2) : -INFINITY;
-            lj[j] = in ? __ldcg(a.part_ml + ((size_t)sl * G + h) * 2 + 1) : 0.f;
-            oj[j] = in ? __ldcg(a.part_o + ((size_t)sl * G + h) * D + e) : 0.f;
-          }
-          float bm = M;
-#pragma unroll
-          for (int j = 0; j < kPieceBatch; ++j) bm = fmaxf(bm, mj[j]);
-          if (bm == -INFINITY) continue;
-          const float sc = exp2f(M - bm);  // M = -inf gives 0
-          L *= sc;
-          A *= sc;
-#pragma unroll
-          for (int j = 0; j < kPieceBatch; ++j) {
-            const float w = (mj[j] == -INFINITY) ? 0.f : exp2f(mj[j] - bm);
-            L += lj[j] * w;
-            A += oj[j] * w;
-          }
-          M = bm;
-        }
-        store_out<T>(orow + (size_t)h * D + e, A / L);
-      }
-      if (threadIdx.x == 0) a.tick[d.pair] = 0;
-    }
+    // sm is free for the next piece once every warp has read it
+    if (!csync(&sync_b, np)) break;
+    ++np;
   }
   if (threadIdx.x == 0 && abort_flag) atomicOr(a.c.err, ERR_TIMEOUT);
 }
 
+// Pair merge: one thread per four consecutive output elements of one pair.
+// It runs as a programmatic dependent launch after k_decode: its CTAs may be
+// scheduled while k_decode drains, and griddepcontrol.wait returns once every
+// k_decode CTA has finished and its partials are visible.  The pieces of a
+// pair sit in the slots of the consecutive CTA ranges [first, last] that hold
+// its rows; their (max, sum, accumulator) triples combine by the usual online
+// rescaling (base-2 exponents, the max subtracted before exponentiating).
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kMergeThreads) k_decode_merge(const __grid_constant__ DecodeArgs a) {
+  ptx::pdl_wait_primary();
+  constexpr int Q = G * D / 4;  // float4 groups per pair
+  const int Hkv = a.c.Hkv;
+  const int64_t gi = (int64_t)blockIdx.x * kMergeThreads + threadIdx.x;
+  if (gi >= (int64_t)a.B * Hkv * Q) return;
+  const int pair = (int)(gi / Q), qi = (int)(gi % Q);
+  const int h = qi * 4 / D, e0 = qi * 4 % D;
+  const int b = pair / Hkv, g = pair % Hkv;
+  const int64_t R = a.total, NC = a.nctas;
+  const int64_t n = (a.cum[b + 1] - a.cum[b]) / Hkv;
+  const int64_t pstart = a.cum[b] + (int64_t)g * n;
+  const int64_t first = cta_of_row(pstart, R, NC), last = cta_of_row(pstart + n - 1, R, NC);
+  float M = -INFINITY, L = 0.f;
+  float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int64_t c0 = first; c0 <= last; c0 += kPieceBatch) {
+    float2 ml[kPieceBatch];
+    float4 o[kPieceBatch];
+#pragma unroll
+    for (int j = 0; j < kPieceBatch; ++j) {
+      const int64_t sl = c0 + j + pair;
+      const bool in = c0 + j <= last;
+      ml[j] = in ? __ldcg((const float2*)(a.part_ml + ((size_t)sl * G + h) * 2))
+                 : make_float2(-INFINITY, 0.f);
+      o[j] = in ? __ldcg((const float4*)(a.part_o + ((size_t)sl * G + h) * D + e0))
+                : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    float bm = M;
+#pragma unroll
+    for (int j = 0; j < kPieceBatch; ++j) bm = fmaxf(bm, ml[j].x);
+    if (bm == -INFINITY) continue;
+    const float sc = exp2f(M - bm);  // M = -inf gives 0
+    L *= sc;
+    A.x *= sc; A.y *= sc; A.z *= sc; A.w *= sc;
+#pragma unroll
+    for (int j = 0; j < kPieceBatch; ++j) {
+      const float w = (ml[j].x == -INFINITY) ? 0.f : exp2f(ml[j].x - bm);
+      L += ml[j].y * w;
+      A.x += o[j].x * w; A.y += o[j].y * w; A.z += o[j].z * w; A.w += o[j].w * w;
+    }
+    M = bm;
+  }
+  T* orow = (T*)a.out + ((size_t)b * a.Hq + (size_t)g * G + h) * D + e0;
+  store_out<T>(orow + 0, A.x / L);
+  store_out<T>(orow + 1, A.y / L);
+  store_out<T>(orow + 2, A.z / L);
+  store_out<T>(orow + 3, A.w / L);
+}
+
 template <typename T, int D, int G>
 cudaError_t launch_kernel(int nctas, const DecodeArgs& a, cudaStream_t st) {
-  constexpr size_t dyn = (size_t)2 * kStages * DecTile<T, D>::TR * D * sizeof(T);
+  constexpr size_t dyn = (size_t)kStages * (2 * DecTile<T, D>::TR + G) * D * sizeof(T);
   static std::atomic<uint64_t> configured{0};  // one bit per device
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -583,7 +622,20 @@ cudaError_t launch_kernel(int nctas, const DecodeArgs& a, cudaStream_t st) {
     configured.fetch_or(bit);
   }
   k_decode<T, D, G><<<nctas, kThreadsDec, dyn, st>>>(a);
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  const int64_t groups = (int64_t)a.B * a.c.Hkv * (G * D / 4);
+  cfg.gridDim = dim3((unsigned)((groups + kMergeThreads - 1) / kMergeThreads));
+  cfg.blockDim = dim3(kMergeThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_decode_merge<T, D, G>, a);
 }
 
 template <typename T, int D>
@@ -607,16 +659,16 @@ constexpr int kMinRowsPerCta = 128;
 DecodeWs decode_ws_layout(void* ws, int B, int Hkv, int G, int d, int sm_count, size_t* bytes) {
   const int Bl = B < kMaxBatchPerLaunch ? B : kMaxBatchPerLaunch;  // launches run in turn
   const size_t pairs = (size_t)Bl * Hkv;
-  const size_t slots = (size_t)max_ctas(sm_count) + pairs;  // (CTA range, pair) pieces
-  const size_t tick = align256(pairs * sizeof(int32_t));
+  // one slot per (CTA range, pair) piece: range + pair, unique because
+  // both grow in row order
+  const size_t slots = (size_t)max_ctas(sm_count) + pairs;
   const size_t ml = align256(slots * G * 2 * sizeof(float));
   const size_t o = align256(slots * G * d * sizeof(float));
   DecodeWs w;
   char* p = (char*)ws;
-  w.tick = (int32_t*)p;
-  w.part_ml = (float*)(p + tick);
-  w.part_o = (float*)(p + tick + ml);
-  if (bytes) *bytes = tick + ml + o;
+  w.part_ml = (float*)p;
+  w.part_o = (float*)(p + ml);
+  if (bytes) *bytes = ml + o;
   return w;
 }
 
@@ -639,10 +691,11 @@ cudaError_t launch_decode(const CacheDev& c, int dtype, int G, const BatchIds& i
   a.B = B;
   a.part_ml = ws.part_ml;
   a.part_o = ws.part_o;
-  a.tick = ws.tick;
   a.cum[0] = 0;
   for (int b = 0; b < B; ++b) {
     a.seq[b] = ids.seq[b];
+    a.P[b] = ids.P[b];
+    a.head[b] = ids.head[b];
     a.t[b] = ids.t[b];
     a.cum[b + 1] = a.cum[b] + (int64_t)c.Hkv * rows[b];
   }

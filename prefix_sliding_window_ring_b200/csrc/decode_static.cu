@@ -29,10 +29,10 @@ std::mutex g_setup_mutex;
 void* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device.  The first call
-// on a device looks the address up and zero-fills the array (the split-merge
-// arrival counters must start at zero; every decode call leaves them at zero
-// again).  That set-up synchronises the device, so the first call on each
-// device must not be made while a stream is being captured.
+// on a device looks the address up and zero-fills the array (the decode keeps
+// no state in it between calls; the fill only gives it defined contents).
+// That set-up synchronises the device, so the first call on each device must
+// not be made while a stream is being captured.
 cudaError_t scratch_on_current_device(void** out, int* dev_out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);

@@ -11,6 +11,8 @@ constexpr int kMaxBatchPerLaunch = 128;  // batch entries passed by value per la
 
 struct BatchIds {
   int32_t seq[kMaxBatchPerLaunch];
+  int32_t P[kMaxBatchPerLaunch];     // host bookkeeping of each entry's ring state
+  int32_t head[kMaxBatchPerLaunch];
   int64_t t[kMaxBatchPerLaunch];
 };
 
@@ -29,7 +31,6 @@ cudaError_t launch_debug_visible(const CacheDev& c, int seq, int64_t t, int64_t*
 
 // decode.cu
 struct DecodeWs {
-  int32_t* tick;    // [B][Hkv] arrival counters (0 at rest)
   float* part_ml;   // per (pair, CTA) piece: (max, sum) per query head, base-2 domain
   float* part_o;    // per piece: unnormalised accumulators [G][d]
 };
@@ -37,7 +38,8 @@ struct DecodeWs {
 // entries run in turn and reuse it).
 DecodeWs decode_ws_layout(void* ws, int B, int Hkv, int G, int d, int sm_count, size_t* bytes);
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int sm_count);
-// rows[b]: visible rows of entry b (P + count), as the host bookkeeping has them.
+// rows[b]: visible rows of entry b (P + count), as the host bookkeeping has them;
+// ids.P / ids.head likewise.  The kernel checks them against the device record.
 cudaError_t launch_decode(const CacheDev& c, int dtype, int G, const BatchIds& ids,
                           const int32_t* rows, int B, int Hq, const void* q, void* out,
                           float scale, const DecodeWs& ws, int sm_count, cudaStream_t st);

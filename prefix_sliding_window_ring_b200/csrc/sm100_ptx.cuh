@@ -56,6 +56,18 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// ------------------------------------------- programmatic dependent launch --
+// Lets the grid launched after this one (with programmatic stream
+// serialization) be scheduled before this grid completes.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Waits until the preceding grid has completed and its memory is visible
+// (returns at once when the launch had no programmatic dependency).
+__device__ __forceinline__ void pdl_wait_primary() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ------------------------------------------------------- bulk async copies --
 // Global -> shared copy of `bytes` (multiple of 16, both addresses 16-byte
 // aligned) completing on `bar` as transaction bytes.  No multicast.
