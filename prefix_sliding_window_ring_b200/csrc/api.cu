@@ -282,7 +282,6 @@ int ps_attend_decode(ps_cache* c, const void* q, const int* seq_ids, const int64
   if (B == 0) return ok();
   if ((r = check_batch(c, seq_ids, B))) return r;
   if (!t) return fail(PS_EINVAL, "t is NULL");
-  std::vector<int32_t> rows(B);
   for (int b = 0; b < B; ++b) {
     const SeqHost& s = c->seqs[seq_ids[b]];
     if (t[b] != s.next_pos - 1)
@@ -291,7 +290,6 @@ int ps_attend_decode(ps_cache* c, const void* q, const int* seq_ids, const int64
     if (t[b] < s.P)
       return fail(PS_EPOS, "sequence %d: t=%lld lies inside the prefix (P=%d); append first",
                   seq_ids[b], (long long)t[b], s.P);
-    rows[b] = s.P + s.count;
   }
   if (!q || !out || !aligned16(q) || !aligned16(out))
     return fail(PS_EINVAL, "q/out must be non-NULL 16-byte aligned device pointers");
@@ -313,11 +311,11 @@ int ps_attend_decode(ps_cache* c, const void* q, const int* seq_ids, const int64
       ids.seq[i] = seq_ids[b0 + i];
       ids.P[i] = s.P;
       ids.head[i] = s.head;
+      ids.count[i] = s.count;
       ids.t[i] = t[b0 + i];
     }
-    PS_CUDA(ps::launch_decode(c->dev, c->dtype, G, ids, rows.data() + b0, nb, Hq,
-                              (const char*)q + b0 * per_entry, (char*)out + b0 * per_entry, scale,
-                              ws, c->sm_count, st));
+    PS_CUDA(ps::launch_decode(c->dev, c->dtype, G, ids, nb, Hq, (const char*)q + b0 * per_entry,
+                              (char*)out + b0 * per_entry, scale, ws, c->sm_count, st));
   }
   return ok();
 }

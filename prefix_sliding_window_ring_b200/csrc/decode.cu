@@ -83,14 +83,15 @@ struct DecodeArgs {
   void* out;
   float qscale;
   int Hq, B, nctas;
-  int64_t total;       // visible rows of all pairs of the launch
+  int32_t total;       // tiles of all pairs of the launch
   float* part_ml;      // [nctas + B*Hkv][G][2]: per (CTA range, pair) piece (max, sum), base 2
   float* part_o;       // [nctas + B*Hkv][G][D]: per piece unnormalised accumulators
   int32_t seq[kMaxBatchPerLaunch];
-  int32_t P[kMaxBatchPerLaunch];     // prefix length of entry b
-  int32_t head[kMaxBatchPerLaunch];  // physical ring slot of entry b's oldest window row
+  int32_t P[kMaxBatchPerLaunch];      // prefix length of entry b
+  int32_t head[kMaxBatchPerLaunch];   // physical ring slot of entry b's oldest window row
+  int32_t count[kMaxBatchPerLaunch];  // ring rows of entry b
   int64_t t[kMaxBatchPerLaunch];
-  int64_t cum[kMaxBatchPerLaunch + 1];  // cum[b] = Hkv * (rows of entries before b)
+  int32_t tcum[kMaxBatchPerLaunch + 1];  // tcum[b] = Hkv * (tiles per head of entries before b)
 };
 static_assert(sizeof(DecodeArgs) <= 4096, "decode arguments fit the classic parameter space");
 
@@ -308,51 +309,49 @@ struct DecState {
   }
 };
 
-// Calls f(slab_row, nrows) for the tiles of the logical rows [jb, je) of one
-// pair: split at visible-range boundaries and every TR rows.  Registers only.
-// Sets *bad if the range reaches block rows (a decode query never does).
+// Calls f(slab_row, dst_row, nrows) for the contiguous runs of the logical
+// rows [x0, x1) of one pair, dst_row counted from x0 (a tile may span the
+// prefix and both ring runs).  Sets *bad if the rows reach block rows (a
+// decode query never has them).
 template <typename F>
-__device__ __forceinline__ void for_each_tile(const SegSet& s, int32_t jb, int32_t je, int TR,
-                                              bool* bad, F&& f) {
+__device__ __forceinline__ void for_each_run(const SegSet& s, int32_t x0, int32_t x1, bool* bad,
+                                             F&& f) {
   int32_t L = 0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     if (i < s.n) {
-      const int32_t a = max(L, jb), b = min(L + s.len[i], je);
-      if (b > a) {
-        if (s.src[i] == 2) {
-          *bad = true;
-        } else {
-          for (int32_t x = a; x < b; x += TR) f(s.row0[i] + (x - L), min(TR, b - x));
-        }
+      const int32_t lo = max(L, x0), hi = min(L + s.len[i], x1);
+      if (hi > lo) {
+        if (s.src[i] == 2) *bad = true;
+        else f(s.row0[i] + (lo - L), lo - x0, hi - lo);
       }
       L += s.len[i];
     }
   }
 }
 
-// One pair (batch entry b, kv head g) restricted to local rows [lo, hi).
-struct PairPiece {
+// Tiles of the launch.  Pair (b, g) is cut into tph(b) = ceil(rows_b / TR)
+// tiles of TR consecutive logical rows (the last one ragged); the tiles of all
+// pairs are laid end to end (entry-major, then kv head) and CTA c streams the
+// tiles [T c / NC, T (c + 1) / NC).  So every CTA streams the same number of
+// tiles, and only a pair's last tile is ever short.
+struct PairTiles {
   int b, g;
-  int64_t start;  // first flattened row of the pair
-  int32_t n;      // rows of the pair
-  int32_t lo, hi;
+  int32_t tph;    // tiles of the pair
+  int32_t first;  // flattened index of the pair's first tile
 };
-
-__device__ __forceinline__ PairPiece piece_at(const DecodeArgs& a, int64_t r, int64_t r1) {
+__device__ __forceinline__ PairTiles pair_of_tile(const DecodeArgs& a, int32_t x) {
   int lo = 0, hi = a.B - 1;
-  while (lo < hi) {  // last entry with cum[b] <= r
+  while (lo < hi) {  // last entry with tcum[b] <= x
     const int mid = (lo + hi + 1) >> 1;
-    if (a.cum[mid] <= r) lo = mid; else hi = mid - 1;
+    if (a.tcum[mid] <= x) lo = mid; else hi = mid - 1;
   }
-  PairPiece pp;
-  pp.b = lo;
-  pp.n = (int32_t)((a.cum[lo + 1] - a.cum[lo]) / a.c.Hkv);
-  pp.g = (int)((r - a.cum[lo]) / pp.n);
-  pp.start = a.cum[lo] + (int64_t)pp.g * pp.n;
-  pp.lo = (int32_t)(r - pp.start);
-  pp.hi = (int32_t)min((int64_t)pp.n, r1 - pp.start);
-  return pp;
+  PairTiles pt;
+  pt.b = lo;
+  pt.tph = (a.tcum[lo + 1] - a.tcum[lo]) / a.c.Hkv;
+  pt.g = (x - a.tcum[lo]) / pt.tph;
+  pt.first = a.tcum[lo] + pt.g * pt.tph;
+  return pt;
 }
 
 // One tile as the producer hands it to the consumers (through shared memory,
@@ -362,12 +361,12 @@ struct TileDesc {
   int32_t slot;  // partial-result slot of the tile's piece: CTA range + pair
 };
 
-// First flattened row of CTA c's range, and the CTA whose range holds row x.
-__device__ __forceinline__ int64_t range_start(int64_t c, int64_t R, int64_t NC) {
-  return R * c / NC;
+// First flattened tile of CTA c's range, and the CTA whose range holds tile x.
+__device__ __forceinline__ int32_t range_start(int64_t c, int64_t T, int64_t NC) {
+  return (int32_t)(T * c / NC);
 }
-__device__ __forceinline__ int64_t cta_of_row(int64_t x, int64_t R, int64_t NC) {
-  return ((x + 1) * NC - 1) / R;
+__device__ __forceinline__ int32_t cta_of_tile(int64_t x, int64_t T, int64_t NC) {
+  return (int32_t)(((x + 1) * NC - 1) / T);
 }
 
 enum : int32_t { TD_FIRST = 1, TD_LAST = 2, TD_END = 4 };
@@ -408,77 +407,76 @@ __global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8)
     if (lane != 0) return;
     // ------------------------------------------------------------ producer --
     int i = 0;  // tiles handed out so far
-    auto put = [&](const TileDesc& d, const T* ksrc, const T* vsrc) -> bool {
-      const int st = i % kStages;
-      if (i >= kStages && !ptx::mbar_wait_bounded(&empty[st], ((i / kStages) - 1) & 1,
-                                                  &abort_flag, kWaitLimitCycles))
-        return false;
-      desc[st] = d;
-      if (d.flags & TD_END) {
-        ptx::mbar_arrive(&full[st]);
-      } else {
+    bool alive = true;
+    const int32_t x1 = range_start(blockIdx.x + 1, R, NC);
+    for (int32_t x = range_start(blockIdx.x, R, NC); x < x1 && alive;) {
+      // one piece: the tiles of one pair inside this CTA's range
+      const PairTiles pt = pair_of_tile(a, x);
+      const int32_t j0 = x - pt.first, j1 = min(pt.tph, x1 - pt.first);
+      x = pt.first + j1;
+      const int s = a.seq[pt.b];
+      // The ring state comes with the launch (the host's bookkeeping), so the
+      // copies start without a dependent global load; the device's own record
+      // is loaded alongside and compared once the piece's copies are issued.
+      const DevMeta md = a.c.meta[s];
+      DevMeta m;
+      m.next_pos = a.t[pt.b] + 1;
+      m.P = a.P[pt.b];
+      m.head = a.head[pt.b];
+      m.count = a.count[pt.b];
+      const SegSet segs = build_segments(m, a.c.W, a.c.P_max, a.t[pt.b]);
+      bool bad = segs.total != m.P + m.count || (segs.total + TR - 1) / TR != pt.tph;
+      const size_t slab = ((size_t)s * Hkv + pt.g) * (size_t)a.c.slab_rows * D;
+      const int pair = pt.b * Hkv + pt.g;
+      for (int32_t j = j0; j < j1 && alive; ++j) {
+        const int32_t r0 = j * TR, r1 = min(segs.total, r0 + TR);
+        const int st = i % kStages;
+        if (i >= kStages && !ptx::mbar_wait_bounded(&empty[st], ((i / kStages) - 1) & 1,
+                                                    &abort_flag, kWaitLimitCycles)) {
+          alive = false;
+          break;
+        }
+        TileDesc d;
+        d.pair = pair;
+        d.nrows = max(r1 - r0, 0);
+        d.flags = (j == j0 ? TD_FIRST : 0) | (j == j1 - 1 ? TD_LAST : 0);
+        d.slot = (int32_t)blockIdx.x + pair;
+        desc[st] = d;
         // The first tile of a piece also brings the piece's G query rows, so
         // no consumer waits on a global load of q when a piece starts.
         const uint32_t bytes = (uint32_t)d.nrows * D * sizeof(T);
         const uint32_t qbytes = (d.flags & TD_FIRST) ? (uint32_t)(G * D * sizeof(T)) : 0u;
         ptx::mbar_arrive_expect_tx(&full[st], 2 * bytes + qbytes);
-        if (qbytes) {
-          const int b = d.pair / Hkv, g = d.pair % Hkv;
+        if (qbytes)
           ptx::bulk_g2s(qtile + (size_t)st * G * D,
-                        (const T*)a.q + ((size_t)b * a.Hq + (size_t)g * G) * D, qbytes, &full[st]);
-        }
-        ptx::bulk_g2s(ktile + (size_t)st * TR * D, ksrc, bytes, &full[st]);
-        ptx::bulk_g2s(vtile + (size_t)st * TR * D, vsrc, bytes, &full[st]);
-      }
-      ++i;
-      return true;
-    };
-    bool alive = true;
-    // Streams the pieces of the rows [r, r1) of CTA range u.
-    auto run = [&](int64_t r, const int64_t r1, const int64_t u) {
-      while (r < r1 && alive) {
-        const PairPiece pp = piece_at(a, r, r1);
-        r = pp.start + pp.hi;
-        const int s = a.seq[pp.b];
-        // The ring state comes with the launch (the host's bookkeeping), so the
-        // copies start without a dependent global load; the device's own record
-        // is loaded alongside and compared once the piece's copies are issued.
-        const DevMeta md = a.c.meta[s];
-        DevMeta m;
-        m.next_pos = a.t[pp.b] + 1;
-        m.P = a.P[pp.b];
-        m.head = a.head[pp.b];
-        m.count = pp.n - m.P;
-        const SegSet segs = build_segments(m, a.c.W, a.c.P_max, a.t[pp.b]);
-        bool bad = false;
-        const size_t slab = ((size_t)s * Hkv + pp.g) * (size_t)a.c.slab_rows * D;
-        const int32_t hi = min(pp.hi, segs.total);
-        int ntiles = 0;
-        for_each_tile(segs, pp.lo, hi, TR, &bad, [&](int64_t, int) { ++ntiles; });
-        int k = 0;
-        const int pair = pp.b * Hkv + pp.g;
-        for_each_tile(segs, pp.lo, hi, TR, &bad, [&](int64_t row, int nr) {
-          if (!alive) return;
-          TileDesc d;
-          d.pair = pair;
-          d.nrows = nr;
-          d.flags = (k == 0 ? TD_FIRST : 0) | (k == ntiles - 1 ? TD_LAST : 0);
-          d.slot = (int32_t)(u + pair);
-          alive = put(d, (const T*)a.c.K + slab + (size_t)row * D,
-                      (const T*)a.c.V + slab + (size_t)row * D);
-          ++k;
+                        (const T*)a.q + ((size_t)pt.b * a.Hq + (size_t)pt.g * G) * D, qbytes,
+                        &full[st]);
+        T* kd = ktile + (size_t)st * TR * D;
+        T* vd = vtile + (size_t)st * TR * D;
+        for_each_run(segs, r0, r1, &bad, [&](int64_t row, int32_t dst, int32_t nr) {
+          const uint32_t nb = (uint32_t)nr * D * sizeof(T);
+          ptx::bulk_g2s(kd + (size_t)dst * D, (const T*)a.c.K + slab + (size_t)row * D, nb,
+                        &full[st]);
+          ptx::bulk_g2s(vd + (size_t)dst * D, (const T*)a.c.V + slab + (size_t)row * D, nb,
+                        &full[st]);
         });
-        if (bad || segs.total != pp.n || md.next_pos != m.next_pos || md.P != m.P ||
-            md.head != m.head || md.count != m.count)
-          atomicOr(a.c.err, ERR_BATCH);
-        if (!segs.ring_ok) atomicOr(a.c.err, ERR_RING);
+        ++i;
       }
-    };
-    run(range_start(blockIdx.x, R, NC), range_start(blockIdx.x + 1, R, NC), blockIdx.x);
-    if (alive) {
-      TileDesc end;
-      end.pair = 0; end.nrows = 0; end.flags = TD_END; end.slot = 0;
-      put(end, nullptr, nullptr);
+      if (bad || md.next_pos != m.next_pos || md.P != m.P || md.head != m.head ||
+          md.count != m.count)
+        atomicOr(a.c.err, ERR_BATCH);
+      if (!segs.ring_ok) atomicOr(a.c.err, ERR_RING);
+    }
+    if (alive) {  // end marker: a descriptor with no bytes
+      const int st = i % kStages;
+      if (i < kStages || ptx::mbar_wait_bounded(&empty[st], ((i / kStages) - 1) & 1, &abort_flag,
+                                                kWaitLimitCycles)) {
+        TileDesc end;
+        end.pair = 0; end.nrows = 0; end.flags = TD_END; end.slot = 0;
+        desc[st] = end;
+        ptx::mbar_arrive(&full[st]);
+        ++i;
+      }
     }
     if (abort_flag) {  // let the copies already issued land before the CTA exits
       int quiet = 0;
@@ -565,9 +563,9 @@ __global__ void __launch_bounds__(kMergeThreads) k_decode_merge(const __grid_con
   const int h = qi * 4 / D, e0 = qi * 4 % D;
   const int b = pair / Hkv, g = pair % Hkv;
   const int64_t R = a.total, NC = a.nctas;
-  const int64_t n = (a.cum[b + 1] - a.cum[b]) / Hkv;
-  const int64_t pstart = a.cum[b] + (int64_t)g * n;
-  const int64_t first = cta_of_row(pstart, R, NC), last = cta_of_row(pstart + n - 1, R, NC);
+  const int32_t tph = (a.tcum[b + 1] - a.tcum[b]) / Hkv;
+  const int32_t pfirst = a.tcum[b] + g * tph;
+  const int64_t first = cta_of_tile(pfirst, R, NC), last = cta_of_tile(pfirst + tph - 1, R, NC);
   float M = -INFINITY, L = 0.f;
   float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int64_t c0 = first; c0 <= last; c0 += kPieceBatch) {
@@ -604,8 +602,24 @@ __global__ void __launch_bounds__(kMergeThreads) k_decode_merge(const __grid_con
   store_out<T>(orow + 3, A.w / L);
 }
 
+int max_ctas(int sm_count) { return sm_count * PS_DEC_CTAS_PER_SM; }
+constexpr int kMinTilesPerCta = 2;
+
 template <typename T, int D, int G>
-cudaError_t launch_kernel(int nctas, const DecodeArgs& a, cudaStream_t st) {
+cudaError_t launch_kernel(DecodeArgs a, int sm_count, cudaStream_t st) {
+  // tiles per head of each entry, laid end to end, and the CTA count
+  constexpr int TR = DecTile<T, D>::TR;
+  a.tcum[0] = 0;
+  for (int b = 0; b < a.B; ++b) {
+    const int rows = a.P[b] + a.count[b];
+    a.tcum[b + 1] = a.tcum[b] + a.c.Hkv * ((rows + TR - 1) / TR);
+  }
+  a.total = a.tcum[a.B];
+  int64_t nc = ((int64_t)a.total + kMinTilesPerCta - 1) / kMinTilesPerCta;
+  if (nc > max_ctas(sm_count)) nc = max_ctas(sm_count);
+  if (nc < 1) nc = 1;
+  a.nctas = (int)nc;
+  const int nctas = a.nctas;
   constexpr size_t dyn = (size_t)kStages * (2 * DecTile<T, D>::TR + G) * D * sizeof(T);
   static std::atomic<uint64_t> configured{0};  // one bit per device
   int dev = 0;
@@ -639,20 +653,17 @@ cudaError_t launch_kernel(int nctas, const DecodeArgs& a, cudaStream_t st) {
 }
 
 template <typename T, int D>
-cudaError_t dispatch_G(int G, int nctas, const DecodeArgs& a, cudaStream_t st) {
+cudaError_t dispatch_G(int G, const DecodeArgs& a, int sm_count, cudaStream_t st) {
   switch (G) {
-    case 1: return launch_kernel<T, D, 1>(nctas, a, st);
-    case 2: return launch_kernel<T, D, 2>(nctas, a, st);
-    case 4: return launch_kernel<T, D, 4>(nctas, a, st);
-    case 8: return launch_kernel<T, D, 8>(nctas, a, st);
+    case 1: return launch_kernel<T, D, 1>(a, sm_count, st);
+    case 2: return launch_kernel<T, D, 2>(a, sm_count, st);
+    case 4: return launch_kernel<T, D, 4>(a, sm_count, st);
+    case 8: return launch_kernel<T, D, 8>(a, sm_count, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
-
-int max_ctas(int sm_count) { return sm_count * PS_DEC_CTAS_PER_SM; }
-constexpr int kMinRowsPerCta = 128;
 
 }  // namespace
 
@@ -660,7 +671,7 @@ DecodeWs decode_ws_layout(void* ws, int B, int Hkv, int G, int d, int sm_count, 
   const int Bl = B < kMaxBatchPerLaunch ? B : kMaxBatchPerLaunch;  // launches run in turn
   const size_t pairs = (size_t)Bl * Hkv;
   // one slot per (CTA range, pair) piece: range + pair, unique because
-  // both grow in row order
+  // both grow in tile order
   const size_t slots = (size_t)max_ctas(sm_count) + pairs;
   const size_t ml = align256(slots * G * 2 * sizeof(float));
   const size_t o = align256(slots * G * d * sizeof(float));
@@ -678,9 +689,9 @@ size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int sm_count) {
   return bytes;
 }
 
-cudaError_t launch_decode(const CacheDev& c, int dtype, int G, const BatchIds& ids,
-                          const int32_t* rows, int B, int Hq, const void* q, void* out,
-                          float scale, const DecodeWs& ws, int sm_count, cudaStream_t st) {
+cudaError_t launch_decode(const CacheDev& c, int dtype, int G, const BatchIds& ids, int B, int Hq,
+                          const void* q, void* out, float scale, const DecodeWs& ws, int sm_count,
+                          cudaStream_t st) {
   DecodeArgs a;
   memset(&a, 0, sizeof(a));
   a.c = c;
@@ -691,25 +702,19 @@ cudaError_t launch_decode(const CacheDev& c, int dtype, int G, const BatchIds& i
   a.B = B;
   a.part_ml = ws.part_ml;
   a.part_o = ws.part_o;
-  a.cum[0] = 0;
   for (int b = 0; b < B; ++b) {
     a.seq[b] = ids.seq[b];
     a.P[b] = ids.P[b];
     a.head[b] = ids.head[b];
+    a.count[b] = ids.count[b];
     a.t[b] = ids.t[b];
-    a.cum[b + 1] = a.cum[b] + (int64_t)c.Hkv * rows[b];
   }
-  a.total = a.cum[B];
-  int64_t nc = (a.total + kMinRowsPerCta - 1) / kMinRowsPerCta;
-  if (nc > max_ctas(sm_count)) nc = max_ctas(sm_count);
-  if (nc < 1) nc = 1;
-  a.nctas = (int)nc;
   if (dtype == 0) {
-    if (c.d == 64) return dispatch_G<float, 64>(G, a.nctas, a, st);
-    return dispatch_G<float, 128>(G, a.nctas, a, st);
+    if (c.d == 64) return dispatch_G<float, 64>(G, a, sm_count, st);
+    return dispatch_G<float, 128>(G, a, sm_count, st);
   }
-  if (c.d == 64) return dispatch_G<uint16_t, 64>(G, a.nctas, a, st);
-  return dispatch_G<uint16_t, 128>(G, a.nctas, a, st);
+  if (c.d == 64) return dispatch_G<uint16_t, 64>(G, a, sm_count, st);
+  return dispatch_G<uint16_t, 128>(G, a, sm_count, st);
 }
 
 }  // namespace ps

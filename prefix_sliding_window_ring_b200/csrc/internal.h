@@ -13,6 +13,7 @@ struct BatchIds {
   int32_t seq[kMaxBatchPerLaunch];
   int32_t P[kMaxBatchPerLaunch];     // host bookkeeping of each entry's ring state
   int32_t head[kMaxBatchPerLaunch];
+  int32_t count[kMaxBatchPerLaunch];
   int64_t t[kMaxBatchPerLaunch];
 };
 
@@ -38,11 +39,11 @@ struct DecodeWs {
 // entries run in turn and reuse it).
 DecodeWs decode_ws_layout(void* ws, int B, int Hkv, int G, int d, int sm_count, size_t* bytes);
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int sm_count);
-// rows[b]: visible rows of entry b (P + count), as the host bookkeeping has them;
-// ids.P / ids.head likewise.  The kernel checks them against the device record.
-cudaError_t launch_decode(const CacheDev& c, int dtype, int G, const BatchIds& ids,
-                          const int32_t* rows, int B, int Hq, const void* q, void* out,
-                          float scale, const DecodeWs& ws, int sm_count, cudaStream_t st);
+// ids.P / ids.head / ids.count: each entry's ring state as the host bookkeeping
+// has it.  The kernel checks them against the device record.
+cudaError_t launch_decode(const CacheDev& c, int dtype, int G, const BatchIds& ids, int B, int Hq,
+                          const void* q, void* out, float scale, const DecodeWs& ws, int sm_count,
+                          cudaStream_t st);
 
 // chunk_tc.cu (tcgen05 chunk kernel: bf16, head_dim 128)
 bool chunk_tc_supported(int dtype, int d, int G);
