@@ -216,7 +216,9 @@ class Workload:
         return list(range(r * B, (r + 1) * B))
 
     def step(self, i, stream=None, host=None):
-        """One hot-path step on batch group i % ROT (append + decode)."""
+        """One hot-path step on batch group i % ROT: append each sequence's token
+        and attend at it (ps_decode_step: ring append, visible ranges, split-K
+        decode and split merge in one streaming launch plus the merge launch)."""
         r = i % ROT
         v = self.visit[r]
         ids = self.ids(r)
@@ -225,8 +227,7 @@ class Workload:
             k, vv, q = self.k_pool[r][v], self.v_pool[r][v], self.q_pool[r][v]
         else:
             k, vv, q = host(r, v)
-        self.cache.append_kv(ids, k, vv, 1, stream)
-        self.cache.attend_decode(q, ids, ts, HQ, self.scale, self.out[r], self.ws, stream)
+        self.cache.decode_step(q, k, vv, ids, ts, HQ, self.scale, self.out[r], self.ws, stream)
         for s in ids:
             self.next_pos[s] += 1
         self.visit[r] += 1
@@ -428,7 +429,7 @@ def run_ours(args, rank, world, local_rank):
                      "traffic": decode_traffic()},
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": 3 * K,  # per step: ring append, decode stream, pair merge
+        "gpu_launches": 2 * K,  # per step: the decode-step stream launch and the pair merge
         "clocks": clk,
         "cpu_baseline": cpu,
         "prefill": prefill,

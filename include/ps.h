@@ -148,6 +148,20 @@ PS_API int ps_attend_decode(ps_cache* c, const void* q, const int* seq_ids, cons
                      int B, int Hq, float scale, void* out, void* workspace,
                      size_t workspace_bytes, void* stream);
 
+/* One whole decode step for B active sequences seq_ids[0..B) (host, distinct):
+ * append the token at t[b] == next_pos (k_new, v_new: [B][Hkv][d], device) to
+ * each ring, evicting as ps_append_kv does, then attend at t[b] as
+ * ps_attend_decode does (the digest's section 03 loop: append, then attend).
+ * The appended row is read once, from k_new/v_new, for the attention and
+ * written to its ring slot in the same pass; the ring contents, positions and
+ * bookkeeping afterwards, and the output, are exactly those of ps_append_kv
+ * (n = 1) followed by ps_attend_decode.  Requires t[b] >= P_s.
+ * q, out, workspace, Hq, scale: as ps_attend_decode.
+ * Errors: PS_EINVAL, PS_ESTATE, PS_EPOS, PS_ENOMEM, PS_EUNSUPPORTED. */
+PS_API int ps_decode_step(ps_cache* c, const void* q, const void* k_new, const void* v_new,
+                          const int* seq_ids, const int64_t* t, int B, int Hq, float scale,
+                          void* out, void* workspace, size_t workspace_bytes, void* stream);
+
 /* ------------------------------ decode for callers that cannot allocate --- */
 
 /* ps_attend_decode without a workspace argument, for callers that cannot give

@@ -40,6 +40,7 @@ SIGNATURES = {
     "ps_decode_workspace_bytes": (_sz, [_vp, _i, _i]),
     "ps_attend_decode": (_i, [_vp, _vp, _vp, _vp, _i, _i, _f, _vp, _vp, _sz, _vp]),
     "ps_attend_decode_static": (_i, [_vp, _vp, _vp, _vp, _i, _i, _f, _vp, _vp]),
+    "ps_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _f, _vp, _vp, _sz, _vp]),
     "ps_attend_chunk": (_i, [_vp, _i, _vp, _vp, _vp, _i64, _i, _i, _f, _vp, _i, _vp]),
     "ps_export_window": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp]),
     "ps_import_window": (_i, [_vp, _i, _i64, _vp, _vp, _i, _i, _vp]),
@@ -154,6 +155,18 @@ def ps_attend_decode(cache, q, seq_ids, t, Hq, scale, out, workspace, workspace_
     _check("ps_attend_decode", _lib.ps_attend_decode(cache, _ptr(q), ids, ts, B, Hq, scale,
                                                      _ptr(out), _ptr(workspace), workspace_bytes,
                                                      _stream(stream)))
+
+
+def ps_decode_step(cache, q, k_new, v_new, seq_ids, t, Hq, scale, out, workspace,
+                   workspace_bytes, stream=None) -> None:
+    """Append the token at t == next_pos of each sequence, then attend at t (one pass)."""
+    ids, B = _ints(seq_ids, ctypes.c_int)
+    ts, Bt = _ints(t, ctypes.c_int64)
+    if Bt != B:
+        raise ValueError("seq_ids and t differ in length")
+    _check("ps_decode_step", _lib.ps_decode_step(cache, _ptr(q), _ptr(k_new), _ptr(v_new), ids,
+                                                 ts, B, Hq, scale, _ptr(out), _ptr(workspace),
+                                                 workspace_bytes, _stream(stream)))
 
 
 def ps_attend_decode_static(cache, q, seq_ids, t, Hq, scale, out, stream=None) -> None:

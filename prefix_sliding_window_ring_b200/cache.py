@@ -61,6 +61,13 @@ class Cache:
         ws = workspace if workspace is not None else self.decode_workspace(B, Hq)
         abi.ps_attend_decode(self.handle, q, seq_ids, t, Hq, scale, out, ws, ws.numel(), stream)
 
+    def decode_step(self, q, k_new, v_new, seq_ids, t, Hq, scale, out, workspace=None,
+                    stream=None):
+        B = len(seq_ids)
+        ws = workspace if workspace is not None else self.decode_workspace(B, Hq)
+        abi.ps_decode_step(self.handle, q, k_new, v_new, seq_ids, t, Hq, scale, out, ws,
+                           ws.numel(), stream)
+
     def attend_chunk(self, seq, q, k_blk, v_blk, t0, n, Hq, scale, out, append_after=0, stream=None):
         abi.ps_attend_chunk(self.handle, seq, q, k_blk, v_blk, t0, n, Hq, scale, out, append_after,
                             stream)

@@ -315,8 +315,63 @@ int ps_attend_decode(ps_cache* c, const void* q, const int* seq_ids, const int64
       ids.t[i] = t[b0 + i];
     }
     PS_CUDA(ps::launch_decode(c->dev, c->dtype, G, ids, nb, Hq, (const char*)q + b0 * per_entry,
+                              nullptr, nullptr, (char*)out + b0 * per_entry, scale, ws,
+                              c->sm_count, st));
+  }
+  return ok();
+}
+
+int ps_decode_step(ps_cache* c, const void* q, const void* k_new, const void* v_new,
+                   const int* seq_ids, const int64_t* t, int B, int Hq, float scale, void* out,
+                   void* workspace, size_t workspace_bytes, void* stream) {
+  if (!c) return fail(PS_EINVAL, "cache is NULL");
+  if (B < 0) return fail(PS_EINVAL, "negative B=%d", B);
+  int G = 0;
+  int r = check_group(c, Hq, &G);
+  if (r) return r;
+  if (B == 0) return ok();
+  if ((r = check_batch(c, seq_ids, B))) return r;
+  if (!t) return fail(PS_EINVAL, "t is NULL");
+  for (int b = 0; b < B; ++b) {
+    const SeqHost& s = c->seqs[seq_ids[b]];
+    if (t[b] != s.next_pos)
+      return fail(PS_EPOS, "sequence %d: t=%lld is not the next position %lld", seq_ids[b],
+                  (long long)t[b], (long long)s.next_pos);
+    if (t[b] < s.P)
+      return fail(PS_EPOS, "sequence %d: t=%lld lies inside the prefix (P=%d)", seq_ids[b],
+                  (long long)t[b], s.P);
+  }
+  if (!q || !out || !k_new || !v_new || !aligned16(q) || !aligned16(out) || !aligned16(k_new) ||
+      !aligned16(v_new))
+    return fail(PS_EINVAL, "q/k_new/v_new/out must be non-NULL 16-byte aligned device pointers");
+  if (!workspace || ((uintptr_t)workspace & 255))
+    return fail(PS_EINVAL, "workspace must be a non-NULL 256-byte aligned device pointer");
+  size_t need = 0;
+  ps::DecodeWs ws = ps::decode_ws_layout(workspace, B, c->Hkv, G, c->d, c->sm_count, &need);
+  if (need > workspace_bytes)
+    return fail(PS_ENOMEM, "workspace holds %zu bytes, this call needs %zu", workspace_bytes, need);
+  if ((r = check_device(c))) return r;
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t per_entry = (size_t)Hq * c->d * c->esize;
+  const size_t per_row = (size_t)c->Hkv * c->d * c->esize;
+  for (int b0 = 0; b0 < B; b0 += ps::kMaxBatchPerLaunch) {
+    int nb = B - b0 < ps::kMaxBatchPerLaunch ? B - b0 : ps::kMaxBatchPerLaunch;
+    ps::BatchIds ids;
+    memset(&ids, 0, sizeof(ids));
+    for (int i = 0; i < nb; ++i) {
+      SeqHost s = c->seqs[seq_ids[b0 + i]];
+      advance(s, c->W, 1);  // the state the attention sees: the token appended
+      ids.seq[i] = seq_ids[b0 + i];
+      ids.P[i] = s.P;
+      ids.head[i] = s.head;
+      ids.count[i] = s.count;
+      ids.t[i] = t[b0 + i];
+    }
+    PS_CUDA(ps::launch_decode(c->dev, c->dtype, G, ids, nb, Hq, (const char*)q + b0 * per_entry,
+                              (const char*)k_new + b0 * per_row, (const char*)v_new + b0 * per_row,
                               (char*)out + b0 * per_entry, scale, ws, c->sm_count, st));
   }
+  for (int b = 0; b < B; ++b) advance(c->seqs[seq_ids[b]], c->W, 1);
   return ok();
 }
 

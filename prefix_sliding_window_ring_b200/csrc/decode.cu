@@ -80,6 +80,8 @@ template <typename T, int D> struct DecTile {
 struct DecodeArgs {
   CacheDev c;
   const void* q;
+  const void* knew;  // decode step: appended rows [B][Hkv][D] (NULL for a plain decode)
+  const void* vnew;
   void* out;
   float qscale;
   int Hq, B, nctas;
@@ -369,7 +371,12 @@ __device__ __forceinline__ int32_t cta_of_tile(int64_t x, int64_t T, int64_t NC)
   return (int32_t)(((x + 1) * NC - 1) / T);
 }
 
-enum : int32_t { TD_FIRST = 1, TD_LAST = 2, TD_END = 4 };
+enum : int32_t {
+  TD_FIRST = 1,  // first tile of a piece (brings the piece's q rows)
+  TD_LAST = 2,   // last tile of a piece
+  TD_END = 4,    // no more tiles
+  TD_NEW = 8,    // the tile's last row is the appended token (decode step)
+};
 
 template <typename T, int D, int G>
 __global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8)
@@ -426,6 +433,7 @@ __global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8)
       m.count = a.count[pt.b];
       const SegSet segs = build_segments(m, a.c.W, a.c.P_max, a.t[pt.b]);
       bool bad = segs.total != m.P + m.count || (segs.total + TR - 1) / TR != pt.tph;
+      const bool step = a.knew != nullptr;  // the pair's last row comes from knew/vnew
       const size_t slab = ((size_t)s * Hkv + pt.g) * (size_t)a.c.slab_rows * D;
       const int pair = pt.b * Hkv + pt.g;
       for (int32_t j = j0; j < j1 && alive; ++j) {
@@ -439,7 +447,8 @@ __global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8)
         TileDesc d;
         d.pair = pair;
         d.nrows = max(r1 - r0, 0);
-        d.flags = (j == j0 ? TD_FIRST : 0) | (j == j1 - 1 ? TD_LAST : 0);
+        const bool with_new = step && r1 == segs.total;
+        d.flags = (j == j0 ? TD_FIRST : 0) | (j == j1 - 1 ? TD_LAST : 0) | (with_new ? TD_NEW : 0);
         d.slot = (int32_t)blockIdx.x + pair;
         desc[st] = d;
         // The first tile of a piece also brings the piece's G query rows, so
@@ -453,17 +462,33 @@ __global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8)
                         &full[st]);
         T* kd = ktile + (size_t)st * TR * D;
         T* vd = vtile + (size_t)st * TR * D;
-        for_each_run(segs, r0, r1, &bad, [&](int64_t row, int32_t dst, int32_t nr) {
+        for_each_run(segs, r0, with_new ? r1 - 1 : r1, &bad,
+                     [&](int64_t row, int32_t dst, int32_t nr) {
           const uint32_t nb = (uint32_t)nr * D * sizeof(T);
           ptx::bulk_g2s(kd + (size_t)dst * D, (const T*)a.c.K + slab + (size_t)row * D, nb,
                         &full[st]);
           ptx::bulk_g2s(vd + (size_t)dst * D, (const T*)a.c.V + slab + (size_t)row * D, nb,
                         &full[st]);
         });
+        if (with_new) {  // the appended token, straight from the caller's rows
+          const size_t src = (size_t)pair * D;
+          const size_t dst = (size_t)(r1 - 1 - r0) * D;
+          ptx::bulk_g2s(kd + dst, (const T*)a.knew + src, D * sizeof(T), &full[st]);
+          ptx::bulk_g2s(vd + dst, (const T*)a.vnew + src, D * sizeof(T), &full[st]);
+        }
         ++i;
       }
-      if (bad || md.next_pos != m.next_pos || md.P != m.P || md.head != m.head ||
-          md.count != m.count)
+      // The device record is the state before this launch: for a decode step
+      // it must advance to m by the one appended token.
+      DevMeta me = md;
+      if (step) {
+        const int64_t W = a.c.W, cn = (int64_t)md.count + 1;
+        me.next_pos = md.next_pos + 1;
+        me.count = (int32_t)(cn < W ? cn : W);
+        me.head = (int32_t)((md.head + (cn > W ? 1 : 0)) % W);
+      }
+      if (bad || me.next_pos != m.next_pos || me.P != m.P || me.head != m.head ||
+          me.count != m.count)
         atomicOr(a.c.err, ERR_BATCH);
       if (!segs.ring_ok) atomicOr(a.c.err, ERR_RING);
     }
@@ -510,6 +535,22 @@ __global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8)
     if (mine > 0)
       st.tile(ktile + ((size_t)stg * TR + warp * RW) * D,
               vtile + ((size_t)stg * TR + warp * RW) * D, mine);
+    if ((d.flags & TD_NEW) && warp == (d.nrows - 1) / RW) {
+      // decode step: this warp holds the appended token; store it in its ring
+      // slot (the evicted row's, never visible to this step's queries)
+      const int b = d.pair / Hkv, g = d.pair % Hkv, s = a.seq[b];
+      const int64_t slot = ((int64_t)a.head[b] + a.count[b] - 1) % a.c.W;
+      const size_t row = (((size_t)s * Hkv + g) * (size_t)a.c.slab_rows + a.c.P_max + slot) * D;
+      const size_t so = ((size_t)stg * TR + d.nrows - 1) * D;
+      constexpr int V16 = D * (int)sizeof(T) / 16;  // 16-byte pieces per row
+      for (int x = lane; x < 2 * V16; x += 32) {
+        const bool isv = x >= V16;
+        const int xi = isv ? x - V16 : x;
+        const uint4 val = ((const uint4*)((isv ? vtile : ktile) + so))[xi];
+        ((uint4*)((T*)(isv ? a.c.V : a.c.K) + row))[xi] = val;
+      }
+      if (lane == 0 && g == 0) a.c.pos[(size_t)s * a.c.W + slot] = a.t[b];
+    }
     __syncwarp();
     if (lane == 0) ptx::mbar_arrive(&empty[stg]);
     if (!(d.flags & TD_LAST)) continue;
@@ -558,6 +599,15 @@ __global__ void __launch_bounds__(kMergeThreads) k_decode_merge(const __grid_con
   constexpr int Q = G * D / 4;  // float4 groups per pair
   const int Hkv = a.c.Hkv;
   const int64_t gi = (int64_t)blockIdx.x * kMergeThreads + threadIdx.x;
+  if (a.knew != nullptr && gi < a.B) {  // decode step: commit each entry's new bookkeeping
+    DevMeta m;
+    memset(&m, 0, sizeof(m));
+    m.next_pos = a.t[gi] + 1;
+    m.P = a.P[gi];
+    m.head = a.head[gi];
+    m.count = a.count[gi];
+    a.c.meta[a.seq[gi]] = m;
+  }
   if (gi >= (int64_t)a.B * Hkv * Q) return;
   const int pair = (int)(gi / Q), qi = (int)(gi % Q);
   const int h = qi * 4 / D, e0 = qi * 4 % D;
@@ -690,12 +740,14 @@ size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int sm_count) {
 }
 
 cudaError_t launch_decode(const CacheDev& c, int dtype, int G, const BatchIds& ids, int B, int Hq,
-                          const void* q, void* out, float scale, const DecodeWs& ws, int sm_count,
-                          cudaStream_t st) {
+                          const void* q, const void* k_new, const void* v_new, void* out,
+                          float scale, const DecodeWs& ws, int sm_count, cudaStream_t st) {
   DecodeArgs a;
   memset(&a, 0, sizeof(a));
   a.c = c;
   a.q = q;
+  a.knew = k_new;
+  a.vnew = v_new;
   a.out = out;
   a.qscale = scale * kLog2e;
   a.Hq = Hq;

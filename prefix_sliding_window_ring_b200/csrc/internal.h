@@ -41,9 +41,13 @@ DecodeWs decode_ws_layout(void* ws, int B, int Hkv, int G, int d, int sm_count, 
 size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int sm_count);
 // ids.P / ids.head / ids.count: each entry's ring state as the host bookkeeping
 // has it.  The kernel checks them against the device record.
+// k_new / v_new: NULL for a plain decode; for a decode step, the appended rows
+// [B][Hkv][d] at positions ids.t (ids then holds the state after the append),
+// which the launch reads for the attention, writes to their ring slots, and
+// after which it commits the new bookkeeping.
 cudaError_t launch_decode(const CacheDev& c, int dtype, int G, const BatchIds& ids, int B, int Hq,
-                          const void* q, void* out, float scale, const DecodeWs& ws, int sm_count,
-                          cudaStream_t st);
+                          const void* q, const void* k_new, const void* v_new, void* out,
+                          float scale, const DecodeWs& ws, int sm_count, cudaStream_t st);
 
 // chunk_tc.cu (tcgen05 chunk kernel: bf16, head_dim 128)
 bool chunk_tc_supported(int dtype, int d, int G);
