@@ -511,7 +511,60 @@ def prefill_measure(steps: int):
         c.close()
         del blocks
         torch.cuda.empty_cache()
+    res["prompt"] = prompt_measure(steps, peak)
     return res
+
+
+PR_P = 4096  # prompt length of the prompt-prefill measurement
+
+
+def prompt_measure(steps: int, peak: float):
+    """Prompt prefill (queries inside the pinned prefix, causal over it) on the
+    tensor-core kernel: 4 sequences with a 4096-token prompt each, one
+    ps_attend_prompt call per sequence.  Visible pairs only:
+    4 * d * Hq * sum over t < P of (t + 1) flops per sequence."""
+    import torch
+
+    import synth
+    from prefix_sliding_window_ring_b200 import PS_BF16, Cache
+
+    def dev(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+
+    c = Cache(W, PR_P, HKV, D, PS_BF16, PF_SEQS)
+    qs = []
+    for s in range(PF_SEQS):
+        c.prefill_prefix(s, dev(synth.rows(SEED, synth.TID_K, s, HKV, 0, PR_P, D, "bf16")),
+                         dev(synth.rows(SEED, synth.TID_V, s, HKV, 0, PR_P, D, "bf16")), PR_P)
+        q = dev(synth.rows(SEED, synth.TID_Q, s, HQ, 0, PR_P, D, "bf16"))
+        qs.append((q, torch.empty_like(q)))
+    scale = 1.0 / math.sqrt(D)
+    side = [torch.cuda.Stream() for _ in qs]
+
+    def step(i, st=None):
+        st = st or torch.cuda.current_stream()
+        for ss in side:
+            ss.wait_stream(st)
+        for s, (q, o) in enumerate(qs):
+            c.attend_prompt(s, q, 0, PR_P, HQ, scale, o, side[s])
+        for ss in side:
+            st.wait_stream(ss)
+
+    for i in range(3):
+        step(i)
+    torch.cuda.synchronize()
+    if c.device_error():
+        raise RuntimeError("device error word set by the prompt kernel")
+    ms = min(time_graph(torch, step, steps) for _ in range(2))
+    flops = 4.0 * D * HQ * (PR_P * (PR_P + 1) / 2) * PF_SEQS
+    tf = flops / (ms / 1e3) / 1e12
+    c.close()
+    del qs
+    torch.cuda.empty_cache()
+    return {"workload": f"{PF_SEQS} sequences x {PR_P}-token prompt (causal over the pinned prefix), "
+                        f"Hq={HQ} Hkv={HKV} d={D}, bf16",
+            "ms_per_step": round(ms, 4), "gflop_per_step": round(flops / 1e9, 1),
+            "achieved": round(tf, 1), "frac": round(tf / peak, 4)}
 
 
 # ------------------------------------------------------------ CPU oracle ----

@@ -108,6 +108,17 @@ PS_API int ps_seq_info_get(const ps_cache* c, int seq, ps_seq_info* out);
 PS_API int ps_prefill_prefix(ps_cache* c, int seq, const void* k, const void* v, int P_s,
                       void* stream);
 
+/* Attention of prompt tokens t0..t0+n-1 of active sequence `seq`, all inside
+ * its pinned prefix (0 <= t0, t0 + n <= P_s), over the prefix rows stored by
+ * ps_prefill_prefix: query t sees positions [0, t] (for t < P_s the
+ * visibility rule is plain causal attention; digest section 03 encodes the
+ * prefix once).  q: [n][Hq][d], out: [n][Hq][d] (device, cache dtype).  bf16
+ * with head_dim 128 runs on the tcgen05 tensor-core kernel, other
+ * configurations on the CUDA-core kernel.  The sequence's state is unchanged.
+ * Errors: PS_EINVAL, PS_ESTATE, PS_EPOS. */
+PS_API int ps_attend_prompt(ps_cache* c, int seq, const void* q, int64_t t0, int n, int Hq,
+                            float scale, void* out, void* stream);
+
 /* ---------------------------------------------------- a2 ring append ----- */
 
 /* Append n tokens to each of B active sequences seq_ids[0..B) (host array of

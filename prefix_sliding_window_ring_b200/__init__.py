@@ -5,7 +5,7 @@ The work happens in ``libps.so`` (hand-written CUDA, C ABI in include/ps.h);
 cache lives in.  Importing fails loudly if the library has not been built.
 """
 from .abi import (PS_BF16, PS_EINVAL, PS_ENOMEM, PS_EPOS, PS_ESTATE, PS_F32,  # noqa: F401
-                  PSError, ps_append_kv, ps_attend_chunk, ps_attend_decode,
+                  PSError, ps_append_kv, ps_attend_chunk, ps_attend_decode, ps_attend_prompt,
                   ps_attend_decode_static, ps_cache_bytes, ps_cache_create, ps_cache_destroy,
                   ps_debug_visible, ps_decode_step, ps_decode_workspace_bytes, ps_device_error,
                   ps_export_window, ps_import_window, ps_last_error, ps_prefill_prefix,

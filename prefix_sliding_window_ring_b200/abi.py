@@ -42,6 +42,7 @@ SIGNATURES = {
     "ps_attend_decode_static": (_i, [_vp, _vp, _vp, _vp, _i, _i, _f, _vp, _vp]),
     "ps_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _f, _vp, _vp, _sz, _vp]),
     "ps_attend_chunk": (_i, [_vp, _i, _vp, _vp, _vp, _i64, _i, _i, _f, _vp, _i, _vp]),
+    "ps_attend_prompt": (_i, [_vp, _i, _vp, _i64, _i, _i, _f, _vp, _vp]),
     "ps_export_window": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp]),
     "ps_import_window": (_i, [_vp, _i, _i64, _vp, _vp, _i, _i, _vp]),
     "ps_debug_visible": (_i, [_vp, _i, _i64, _vp, _vp, _vp]),
@@ -185,6 +186,12 @@ def ps_attend_chunk(cache, seq, q, k_blk, v_blk, t0, n, Hq, scale, out, append_a
     _check("ps_attend_chunk", _lib.ps_attend_chunk(cache, seq, _ptr(q), _ptr(k_blk), _ptr(v_blk),
                                                    t0, n, Hq, scale, _ptr(out), int(append_after),
                                                    _stream(stream)))
+
+
+def ps_attend_prompt(cache, seq, q, t0, n, Hq, scale, out, stream=None) -> None:
+    """Causal attention of prompt tokens t0..t0+n-1 (inside the pinned prefix)."""
+    _check("ps_attend_prompt", _lib.ps_attend_prompt(cache, seq, _ptr(q), t0, n, Hq, scale,
+                                                     _ptr(out), _stream(stream)))
 
 
 def ps_export_window(cache, seq, k, v, pos, count_out, stream=None) -> None:

@@ -72,6 +72,9 @@ class Cache:
         abi.ps_attend_chunk(self.handle, seq, q, k_blk, v_blk, t0, n, Hq, scale, out, append_after,
                             stream)
 
+    def attend_prompt(self, seq, q, t0, n, Hq, scale, out, stream=None):
+        abi.ps_attend_prompt(self.handle, seq, q, t0, n, Hq, scale, out, stream)
+
     def export_window(self, seq, stream=None):
         k = torch.empty((self.W, self.Hkv, self.d), dtype=self.torch_dtype, device=self.buf.device)
         v = torch.empty_like(k)

@@ -397,10 +397,10 @@ int ps_attend_chunk(ps_cache* c, int seq, const void* q, const void* k_blk, cons
   if ((r = check_device(c))) return r;
   cudaStream_t st = (cudaStream_t)stream;
   if (ps::chunk_tc_supported(c->dtype, c->d, G))
-    PS_CUDA(ps::launch_chunk_tc(c->dev, G, seq, t0, n, Hq, q, k_blk, v_blk, out, scale, st));
+    PS_CUDA(ps::launch_chunk_tc(c->dev, G, seq, t0, n, Hq, q, k_blk, v_blk, out, scale, 0, st));
   else
     PS_CUDA(ps::launch_chunk_cc(c->dev, c->dtype, G, seq, t0, n, Hq, q, k_blk, v_blk, out, scale,
-                                st));
+                                0, st));
   if (append_after) {
     ps::BatchIds ids;
     memset(&ids, 0, sizeof(ids));
@@ -408,6 +408,31 @@ int ps_attend_chunk(ps_cache* c, int seq, const void* q, const void* k_blk, cons
     PS_CUDA(ps::launch_ring_append(c->dev, c->esize, ids, 1, k_blk, v_blk, n, st));
     advance(c->seqs[seq], c->W, n);
   }
+  return ok();
+}
+
+int ps_attend_prompt(ps_cache* c, int seq, const void* q, int64_t t0, int n, int Hq, float scale,
+                     void* out, void* stream) {
+  if (!c) return fail(PS_EINVAL, "cache is NULL");
+  int r = check_seq(c, seq, true);
+  if (r) return r;
+  int G = 0;
+  if ((r = check_group(c, Hq, &G))) return r;
+  if (n < 0) return fail(PS_EINVAL, "negative n=%d", n);
+  const SeqHost& s = c->seqs[seq];
+  if (t0 < 0 || t0 + n > s.P)
+    return fail(PS_EPOS, "prompt queries [%lld, %lld) are not inside the prefix (P=%d)",
+                (long long)t0, (long long)(t0 + n), s.P);
+  if (n == 0) return ok();
+  if (!q || !out || !aligned16(q) || !aligned16(out))
+    return fail(PS_EINVAL, "q/out must be non-NULL 16-byte aligned device pointers");
+  if ((r = check_device(c))) return r;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (ps::chunk_tc_supported(c->dtype, c->d, G))
+    PS_CUDA(ps::launch_chunk_tc(c->dev, G, seq, t0, n, Hq, q, nullptr, nullptr, out, scale, 1, st));
+  else
+    PS_CUDA(ps::launch_chunk_cc(c->dev, c->dtype, G, seq, t0, n, Hq, q, nullptr, nullptr, out,
+                                scale, 1, st));
   return ok();
 }
 

@@ -238,6 +238,7 @@ struct AttnArgs {
   float* part_o;     // [B][Hkv][nsplit][G][D]
   int32_t* tick;     // [B][Hkv]
   int nsplit, chunk, Hq, b_off, seq;
+  int prompt;  // queries inside the prefix: causal over the prefix rows only
   int64_t t0;
   BatchIds ids;
 };
@@ -248,9 +249,17 @@ __global__ void __launch_bounds__(kThreadsAttn) k_chunk_cc(AttnArgs a) {
   const int i = blockIdx.x, g = blockIdx.y;
   const DevMeta m = a.c.meta[a.seq];
   const int64_t t = a.t0 + i;
-  const SegSet segs = build_segments(m, a.c.W, a.c.P_max, t);
+  SegSet segs = build_segments(m, a.c.W, a.c.P_max, t);
+  if (a.prompt) {  // t < P: the visible rows are the prefix rows [0, t]
+    segs.n = 1;
+    segs.len[0] = (int32_t)(t + 1);
+    segs.row0[0] = 0;
+    segs.src[0] = 0;
+    segs.total = (int32_t)(t + 1);
+    segs.ring_ok = 1;
+  }
   if (threadIdx.x == 0 && i == 0 && g == 0) {
-    if (m.next_pos != a.t0) atomicOr(a.c.err, ERR_BATCH);
+    if (a.prompt ? a.t0 + gridDim.x > m.P : m.next_pos != a.t0) atomicOr(a.c.err, ERR_BATCH);
     if (!segs.ring_ok) atomicOr(a.c.err, ERR_RING);
   }
   const size_t slab = ((size_t)a.seq * a.c.Hkv + g) * (size_t)a.c.slab_rows * D;
@@ -283,7 +292,7 @@ cudaError_t dispatch_chunk_G(int G, dim3 grid, const AttnArgs& a, cudaStream_t s
 
 cudaError_t launch_chunk_cc(const CacheDev& c, int dtype, int G, int seq, int64_t t0, int n,
                             int Hq, const void* q, const void* k_blk, const void* v_blk,
-                            void* out, float scale, cudaStream_t st) {
+                            void* out, float scale, int prompt, cudaStream_t st) {
   AttnArgs a;
   memset(&a, 0, sizeof(a));
   a.c = c;
@@ -294,6 +303,7 @@ cudaError_t launch_chunk_cc(const CacheDev& c, int dtype, int G, int seq, int64_
   a.qscale = scale * kLog2e;
   a.Hq = Hq;
   a.seq = seq;
+  a.prompt = prompt;
   a.t0 = t0;
   dim3 grid(n, c.Hkv);
   if (dtype == 0) {

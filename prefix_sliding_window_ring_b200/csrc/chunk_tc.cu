@@ -62,6 +62,7 @@ struct ChunkArgs {
   CacheDev c;
   void* out;
   int seq, n, Hq, G, PT;
+  int prompt;  // queries inside the prefix: causal over the prefix rows only
   int64_t t0;
   float sc;  // softmax scale * log2(e)
 };
@@ -102,12 +103,17 @@ __device__ __forceinline__ void add_range(KSched& s, int src, int64_t row0, int6
 }
 
 // Query positions [plo, phi]; the ring holds [next_pos - count, next_pos - 1] = [.., t0 - 1].
+// Prompt queries (phi < P) read only the prefix rows [0, phi].
 __device__ __forceinline__ KSched make_sched(const DevMeta& m, int W, int P_max, int64_t t0,
-                                             int64_t plo, int64_t phi) {
+                                             int64_t plo, int64_t phi, bool prompt) {
   KSched s;
   s.n = 0;
   s.ntiles = 0;
   for (int i = 0; i < 4; ++i) { s.src[i] = 0; s.row0[i] = 0; s.pos0[i] = 0; s.len[i] = 0; s.tbase[i] = 0; }
+  if (prompt) {
+    add_range(s, 0, 0, 0, phi + 1 < m.P ? phi + 1 : m.P);
+    return s;
+  }
   add_range(s, 0, 0, 0, m.P);  // pinned prefix
   int64_t lo = plo - W + 1;
   if (lo < m.P) lo = m.P;
@@ -179,7 +185,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
   const DevMeta m = a.c.meta[a.seq];
   const int64_t plo = a.t0 + i0;
   const int64_t phi = a.t0 + min(i0 + PT, a.n) - 1;
-  const KSched ks = make_sched(m, a.c.W, a.c.P_max, a.t0, plo, phi);
+  const KSched ks = make_sched(m, a.c.W, a.c.P_max, a.t0, plo, phi, a.prompt != 0);
   const int T = ks.ntiles;
 
   if (threadIdx.x == 0) {
@@ -196,7 +202,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
     ptx::mbar_init(&mma_done, 1);
     abort_flag = 0;
     ptx::fence_mbar_init();
-    if (m.next_pos != a.t0 && blockIdx.x == 0 && g == 0) atomicOr(a.c.err, ERR_BATCH);
+    const bool bad = a.prompt ? a.t0 + a.n > m.P : m.next_pos != a.t0;
+    if (bad && blockIdx.x == 0 && g == 0) atomicOr(a.c.err, ERR_BATCH);
   }
   if (warp == 2) {
     ptx::tmem_alloc(&tmem_slot, kTmemCols);
@@ -300,7 +307,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
     const int64_t tq = a.t0 + i;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     const int cbase = half * 64;          // first S/O column of this thread
-    const int W = a.c.W, P = m.P;
+    // A prompt query t sees [0, t]: the mask below with the prefix taken as [0, t].
+    const int W = a.c.W, P = a.prompt ? (int)(tq + 1) : m.P;
     const float sc = a.sc;
     const int pair_bar = 2 + quad;        // named barrier of the two warps of this quadrant
     auto pair_sync = [&]() { asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory"); };
@@ -477,7 +485,7 @@ bool chunk_tc_supported(int dtype, int d, int G) {
 
 cudaError_t launch_chunk_tc(const CacheDev& c, int G, int seq, int64_t t0, int n, int Hq,
                             const void* q, const void* k_blk, const void* v_blk, void* out,
-                            float scale, cudaStream_t st) {
+                            float scale, int prompt, cudaStream_t st) {
   ChunkArgs a;
   memset(&a, 0, sizeof(a));
   const uint64_t row = kHD * 2;  // bytes per head row
@@ -487,8 +495,12 @@ cudaError_t launch_chunk_tc(const CacheDev& c, int G, int seq, int64_t t0, int n
                    (uint64_t)c.slab_rows * row, 64, kBN, 1);
   ok = ok && map3d(&a.vslab, c.V, kHD, c.slab_rows, (uint64_t)c.S * c.Hkv, row,
                    (uint64_t)c.slab_rows * row, 64, kBN, 1);
-  ok = ok && map3d(&a.kblk, k_blk, kHD, c.Hkv, n, row, (uint64_t)c.Hkv * row, 64, 1, kBN);
-  ok = ok && map3d(&a.vblk, v_blk, kHD, c.Hkv, n, row, (uint64_t)c.Hkv * row, 64, 1, kBN);
+  // a prompt launch loads no block rows; its block maps describe the cache
+  // K/V (never used) so that every map is well formed
+  ok = ok && map3d(&a.kblk, prompt ? c.K : k_blk, kHD, c.Hkv, n, row, (uint64_t)c.Hkv * row, 64,
+                   1, kBN);
+  ok = ok && map3d(&a.vblk, prompt ? c.V : v_blk, kHD, c.Hkv, n, row, (uint64_t)c.Hkv * row, 64,
+                   1, kBN);
   if (!ok) return cudaErrorInvalidValue;
   a.c = c;
   a.out = out;
@@ -497,6 +509,7 @@ cudaError_t launch_chunk_tc(const CacheDev& c, int G, int seq, int64_t t0, int n
   a.Hq = Hq;
   a.G = G;
   a.PT = PT;
+  a.prompt = prompt;
   a.t0 = t0;
   a.sc = scale * 1.4426950408889634f;
   const size_t dyn = sizeof(TcSmem) + 1024;

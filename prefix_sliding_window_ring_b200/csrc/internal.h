@@ -51,14 +51,16 @@ cudaError_t launch_decode(const CacheDev& c, int dtype, int G, const BatchIds& i
 
 // chunk_tc.cu (tcgen05 chunk kernel: bf16, head_dim 128)
 bool chunk_tc_supported(int dtype, int d, int G);
+// prompt != 0: queries t0..t0+n-1 inside the prefix attend causally to the
+// prefix rows [0, t] (k_blk / v_blk unused); otherwise a chunk at t0 == next_pos.
 cudaError_t launch_chunk_tc(const CacheDev& c, int G, int seq, int64_t t0, int n, int Hq,
                             const void* q, const void* k_blk, const void* v_blk, void* out,
-                            float scale, cudaStream_t st);
+                            float scale, int prompt, cudaStream_t st);
 
 // attend.cu (CUDA-core chunk kernel)
 cudaError_t launch_chunk_cc(const CacheDev& c, int dtype, int G, int seq, int64_t t0, int n,
                             int Hq, const void* q, const void* k_blk, const void* v_blk,
-                            void* out, float scale, cudaStream_t st);
+                            void* out, float scale, int prompt, cudaStream_t st);
 
 // api.cu: error message of the calling thread, and cache accessors.
 int set_error(int code, const char* fmt, ...);

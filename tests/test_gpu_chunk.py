@@ -82,6 +82,10 @@ SMALL = [
     (64, 5, 3, 1, "f32", 64, 8),
     (300, 40, 700, 260, "bf16", 128, 2),
     (256, 128, 256, 384, "bf16", 128, 2),
+    # window not yet full before, and inside, the block (tensor-core kernel)
+    (512, 64, 0, 700, "bf16", 128, 4),
+    (4096, 256, 100, 2048, "bf16", 128, 2),
+    (4096, 128, 3000, 2048, "bf16", 128, 2),
 ]
 
 
