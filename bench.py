@@ -405,6 +405,9 @@ def run_ours(args, rank, world, local_rank):
     prefill = None
     if rank == 0 and not args.no_prefill:
         prefill = prefill_measure(max(3, min(args.steps, 10)))
+    ragged = None
+    if rank == 0 and not args.no_prefill:
+        ragged = ragged_measure(max(3, min(args.steps, 10)))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -434,6 +437,7 @@ def run_ours(args, rank, world, local_rank):
         "cpu_baseline": cpu,
         "prefill": prefill,
         "prefix_overhead": overhead,
+        "ragged": ragged,
     }
     print(json.dumps(line), flush=True)
 
@@ -565,6 +569,73 @@ def prompt_measure(steps: int, peak: float):
                         f"Hq={HQ} Hkv={HKV} d={D}, bf16",
             "ms_per_step": round(ms, 4), "gflop_per_step": round(flops / 1e9, 1),
             "achieved": round(tf, 1), "frac": round(tf / peak, 4)}
+
+
+def ragged_measure(steps: int):
+    """The ragged serving batch: 64 sequences with their own prefix lengths
+    P_s ~ U[64, 512], positions t_s ~ U[P_s, 131072] and ring head offsets, one
+    ps_decode_step per step (about 1.13 GB of visible K/V: larger than L2)."""
+    import torch
+
+    import synth
+    from prefix_sliding_window_ring_b200 import PS_BF16, Cache
+    from synth import workloads
+
+    def dev(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+
+    draws = workloads.ragged_draws(0)
+    S = len(draws)
+    Pm = workloads.RAGGED_P_RANGE[1]
+    c = Cache(W, Pm, HKV, D, PS_BF16, S)
+    for s, r in enumerate(draws):
+        c.seq_reset(s, 0)
+        c.prefill_prefix(s, dev(synth.rows(SEED, synth.TID_K, s, HKV, 0, r.P, D, "bf16")),
+                         dev(synth.rows(SEED, synth.TID_V, s, HKV, 0, r.P, D, "bf16")), r.P)
+        n = min(W, r.t - r.P)
+        if n > 0:
+            c.import_window(s, r.t,
+                            dev(synth.rows(SEED, synth.TID_K, s, HKV, r.t - n, n, D, "bf16")),
+                            dev(synth.rows(SEED, synth.TID_V, s, HKV, r.t - n, n, D, "bf16")),
+                            n, r.h0)
+    total = 3 + 2 * steps
+    q = dev(np.stack([synth.rows(SEED, synth.TID_Q, s, HQ, r.t, total, D, "bf16")
+                      for s, r in enumerate(draws)], axis=1))
+    kn = dev(np.stack([synth.rows(SEED, synth.TID_K, s, HKV, r.t, total, D, "bf16")
+                       for s, r in enumerate(draws)], axis=1))
+    vn = dev(np.stack([synth.rows(SEED, synth.TID_V, s, HKV, r.t, total, D, "bf16")
+                       for s, r in enumerate(draws)], axis=1))
+    out = torch.empty((S, HQ, D), dtype=torch.bfloat16, device="cuda")
+    ws = c.decode_workspace(S, HQ)
+    ids = list(range(S))
+    pos = [r.t for r in draws]
+    scale = 1.0 / math.sqrt(D)
+    rows = []
+
+    def step(i, st=None):
+        c.decode_step(q[i], kn[i], vn[i], ids, pos, HQ, scale, out, ws, st)
+        rows.append(sum(r.P + min(W, p + 1 - r.P) for r, p in zip(draws, pos)))
+        for s in range(S):
+            pos[s] += 1
+
+    for i in range(3):
+        step(i)
+    torch.cuda.synchronize()
+    if c.device_error():
+        raise RuntimeError("device error word set by the ragged decode")
+    n0 = len(rows)
+    ms = time_graph(torch, lambda i, st: step(3 + i, st), steps)
+    kv = HKV * D * 2 * 2 * (sum(rows[n0:]) / steps)
+    if c.device_error():
+        raise RuntimeError("device error word set by the ragged decode")
+    c.close()
+    del q, kn, vn
+    torch.cuda.empty_cache()
+    return {"workload": f"{S} sequences, P_s~U[64,512], t_s~U[P_s,131072], W={W}, "
+                        f"Hq={HQ} Hkv={HKV} d={D}, bf16 (ps_decode_step)",
+            "ms_per_step": round(ms, 5), "tokens_per_s": round(S / (ms / 1e3), 1),
+            "kv_bytes_per_step": int(kv), "kv_gbs": round(kv / (ms / 1e3) / 1e9, 1),
+            "frac": round(kv / (ms / 1e3) / 1e9 / load_peaks()[0], 4)}
 
 
 # ------------------------------------------------------------ CPU oracle ----

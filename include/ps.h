@@ -236,6 +236,14 @@ PS_API int ps_import_window(ps_cache* c, int seq, int64_t next_pos, const void* 
 PS_API int ps_debug_visible(ps_cache* c, int seq, int64_t t, int64_t* pos_out, int32_t* n_out,
                      void* stream);
 
+/* Test hook for the bounded waits of every kernel pipeline: one GPU thread
+ * waits on a barrier that nothing ever arrives at, gives up after about
+ * limit_cycles SM clock cycles (1 <= limit_cycles <= 2^31, about a second at
+ * most) with the same helper the kernels use, and sets bit 8 (time-out) of
+ * the device error word.  No memory but that word is touched and the context
+ * stays usable.  Errors: PS_EINVAL. */
+PS_API int ps_debug_wait_timeout(ps_cache* c, long long limit_cycles, void* stream);
+
 /* Synchronise `stream` and read (then clear) the device error word:
  * *code = 0 when no kernel reported an inconsistency, else an OR of
  *   1  a split launch did not cover every visible row,

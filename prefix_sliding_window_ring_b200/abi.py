@@ -43,6 +43,7 @@ SIGNATURES = {
     "ps_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _f, _vp, _vp, _sz, _vp]),
     "ps_attend_chunk": (_i, [_vp, _i, _vp, _vp, _vp, _i64, _i, _i, _f, _vp, _i, _vp]),
     "ps_attend_prompt": (_i, [_vp, _i, _vp, _i64, _i, _i, _f, _vp, _vp]),
+    "ps_debug_wait_timeout": (_i, [_vp, ctypes.c_longlong, _vp]),
     "ps_export_window": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp]),
     "ps_import_window": (_i, [_vp, _i, _i64, _vp, _vp, _i, _i, _vp]),
     "ps_debug_visible": (_i, [_vp, _i, _i64, _vp, _vp, _vp]),
@@ -192,6 +193,12 @@ def ps_attend_prompt(cache, seq, q, t0, n, Hq, scale, out, stream=None) -> None:
     """Causal attention of prompt tokens t0..t0+n-1 (inside the pinned prefix)."""
     _check("ps_attend_prompt", _lib.ps_attend_prompt(cache, seq, _ptr(q), t0, n, Hq, scale,
                                                      _ptr(out), _stream(stream)))
+
+
+def ps_debug_wait_timeout(cache, limit_cycles, stream=None) -> None:
+    """Run one bounded wait that nothing satisfies (sets the time-out bit)."""
+    _check("ps_debug_wait_timeout", _lib.ps_debug_wait_timeout(cache, limit_cycles,
+                                                               _stream(stream)))
 
 
 def ps_export_window(cache, seq, k, v, pos, count_out, stream=None) -> None:

@@ -495,6 +495,16 @@ int ps_debug_visible(ps_cache* c, int seq, int64_t t, int64_t* pos_out, int32_t*
   return ok();
 }
 
+int ps_debug_wait_timeout(ps_cache* c, long long limit_cycles, void* stream) {
+  if (!c) return fail(PS_EINVAL, "cache is NULL");
+  if (limit_cycles < 1 || limit_cycles > (1ll << 31))
+    return fail(PS_EINVAL, "limit_cycles=%lld outside [1, 2^31]", limit_cycles);
+  int r = check_device(c);
+  if (r) return r;
+  PS_CUDA(ps::launch_debug_wait_timeout(c->dev, limit_cycles, (cudaStream_t)stream));
+  return ok();
+}
+
 int ps_device_error(ps_cache* c, int32_t* code, void* stream) {
   if (!c || !code) return fail(PS_EINVAL, "NULL argument");
   int r = check_device(c);

@@ -407,7 +407,10 @@ __global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8)
     ptx::fence_mbar_init();
   }
   __syncthreads();
-  // The merge grid may be scheduled now; it waits for this grid's completion.
+  // Launched as a programmatic dependent of the previous kernel on the stream:
+  // everything above overlapped its tail; no memory is touched before it has
+  // completed.  Then the merge grid may be scheduled (it waits for this one).
+  ptx::pdl_wait_primary();
   ptx::pdl_launch_dependents();
 
   if (warp == kCW) {
@@ -595,6 +598,7 @@ __global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8)
 // rescaling (base-2 exponents, the max subtracted before exponentiating).
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kMergeThreads) k_decode_merge(const __grid_constant__ DecodeArgs a) {
+  ptx::pdl_launch_dependents();  // the next call's streaming grid may be scheduled
   ptx::pdl_wait_primary();
   constexpr int Q = G * D / 4;  // float4 groups per pair
   const int Hkv = a.c.Hkv;
@@ -685,13 +689,20 @@ cudaError_t launch_kernel(DecodeArgs a, int sm_count, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
-  k_decode<T, D, G><<<nctas, kThreadsDec, dyn, st>>>(a);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
+  // Both grids are programmatic dependent launches of the kernel before them.
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t dcfg = {};
+  dcfg.gridDim = dim3((unsigned)nctas);
+  dcfg.blockDim = dim3(kThreadsDec);
+  dcfg.dynamicSmemBytes = dyn;
+  dcfg.stream = st;
+  dcfg.attrs = attr;
+  dcfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&dcfg, k_decode<T, D, G>, a);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
   const int64_t groups = (int64_t)a.B * a.c.Hkv * (G * D / 4);
   cfg.gridDim = dim3((unsigned)((groups + kMergeThreads - 1) / kMergeThreads));
   cfg.blockDim = dim3(kMergeThreads);

@@ -27,6 +27,7 @@ cudaError_t launch_ring_import(const CacheDev& c, int esize, int seq, const DevM
                                const void* k, const void* v, int n, cudaStream_t st);
 cudaError_t launch_ring_export(const CacheDev& c, int esize, int seq, void* k, void* v,
                                int64_t* pos, int32_t* count_out, cudaStream_t st);
+cudaError_t launch_debug_wait_timeout(const CacheDev& c, long long limit_cycles, cudaStream_t st);
 cudaError_t launch_debug_visible(const CacheDev& c, int seq, int64_t t, int64_t* pos_out,
                                  int32_t* n_out, cudaStream_t st);
 

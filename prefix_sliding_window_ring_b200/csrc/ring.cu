@@ -9,6 +9,7 @@
 // (mod W), and position p always lands in slot (head + p - base) mod W with
 // base = next_pos - count the oldest held position.
 #include "internal.h"
+#include "sm100_ptx.cuh"
 
 namespace ps {
 
@@ -165,6 +166,20 @@ __global__ void k_debug_visible(CacheDev c, int seq, int64_t t, int64_t* __restr
   if (threadIdx.x == 0) *n_out = s.total;
 }
 
+// Test hook for the bounded waits every pipeline uses: one thread waits on an
+// mbarrier that nothing ever arrives at, with the same helper and a short limit,
+// and reports the time-out in the error word as the kernels do.
+__global__ void k_debug_wait_timeout(CacheDev c, long long limit_cycles) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&bar, 1);
+    abort_flag = 0;
+    ptx::fence_mbar_init();
+    if (!ptx::mbar_wait_bounded(&bar, 0, &abort_flag, limit_cycles)) atomicOr(c.err, ERR_TIMEOUT);
+  }
+}
+
 int grid_for(int64_t work, int cap) {
   int64_t g = (work + kThreads - 1) / kThreads;
   if (g < 1) g = 1;
@@ -220,6 +235,11 @@ cudaError_t launch_ring_export(const CacheDev& c, int esize, int seq, void* k, v
 cudaError_t launch_debug_visible(const CacheDev& c, int seq, int64_t t, int64_t* pos_out,
                                  int32_t* n_out, cudaStream_t st) {
   k_debug_visible<<<1, kThreads, 0, st>>>(c, seq, t, pos_out, n_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_debug_wait_timeout(const CacheDev& c, long long limit_cycles, cudaStream_t st) {
+  k_debug_wait_timeout<<<1, 32, 0, st>>>(c, limit_cycles);
   return cudaGetLastError();
 }
 

@@ -68,3 +68,24 @@ def test_decode_inside_prefix_rejected():
     c.prefill_prefix(0, to_torch(sd.k(0, 4)), to_torch(sd.v(0, 4)), 4)
     q = to_torch(sd.q(3, 1))
     assert code_of(c.attend_decode, q, [0], [3], 1, 0.1, torch.empty_like(q)) == abi.PS_EPOS
+
+
+def test_bounded_wait_times_out_and_reports():
+    """A pipeline wait that nothing satisfies gives up after its limit, sets the
+    time-out bit of the device error word, and leaves the context usable: a
+    decode right after it runs and reports no error."""
+    from prefix_sliding_window_ring_b200 import abi
+    W, P, Hq, Hkv, d = 8, 2, 2, 1, 64
+    c = Cache(W, P, Hkv, d, ps_dtype("f32"), 1)
+    sd = SeqData(9, 0, Hq, Hkv, d, "f32")
+    c.prefill_prefix(0, to_torch(sd.k(0, P)), to_torch(sd.v(0, P)), P)
+    abi.ps_debug_wait_timeout(c.handle, 1 << 20)   # about half a millisecond
+    assert c.device_error() == 8                  # the time-out bit, then cleared
+    assert c.device_error() == 0
+    q = to_torch(sd.q(P, 1))
+    out = torch.empty((1, Hq, d), device="cuda")
+    c.decode_step(q, to_torch(sd.k(P, 1)), to_torch(sd.v(P, 1)), [0], [P], Hq, 0.125, out)
+    assert c.device_error() == 0
+    assert torch.isfinite(out).all()
+    with pytest.raises(PSError):
+        abi.ps_debug_wait_timeout(c.handle, 0)
