@@ -405,9 +405,10 @@ def run_ours(args, rank, world, local_rank):
     prefill = None
     if rank == 0 and not args.no_prefill:
         prefill = prefill_measure(max(3, min(args.steps, 10)))
-    ragged = None
+    ragged = shared = None
     if rank == 0 and not args.no_prefill:
         ragged = ragged_measure(max(3, min(args.steps, 10)))
+        shared = shared_prefix_measure(max(3, min(args.steps, 10)))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -438,6 +439,7 @@ def run_ours(args, rank, world, local_rank):
         "prefill": prefill,
         "prefix_overhead": overhead,
         "ragged": ragged,
+        "shared_prefix": shared,
     }
     print(json.dumps(line), flush=True)
 
@@ -636,6 +638,73 @@ def ragged_measure(steps: int):
             "ms_per_step": round(ms, 5), "tokens_per_s": round(S / (ms / 1e3), 1),
             "kv_bytes_per_step": int(kv), "kv_gbs": round(kv / (ms / 1e3) / 1e9, 1),
             "frac": round(kv / (ms / 1e3) / 1e9 / load_peaks()[0], 4)}
+
+
+SP_P = 4096  # system-prompt length of the shared-prefix measurement
+
+
+def shared_prefix_measure(steps: int):
+    """Prompt reuse (ps_share_prefix): B=8 sequences with the same 4096-token
+    pinned prefix, W=4096, t >= 65536, decoded by ps_decode_step -- once with
+    the prefix held once and shared, once with a private copy per sequence.
+    The visible K/V per step is the same (268 MB); the shared prefix is read
+    from HBM once per step instead of eight times."""
+    import torch
+
+    import synth
+    from prefix_sliding_window_ring_b200 import PS_BF16, Cache
+
+    def dev(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+
+    kp = dev(synth.rows(SEED, synth.TID_K, 0, HKV, 0, SP_P, D, "bf16"))
+    vp = dev(synth.rows(SEED, synth.TID_V, 0, HKV, 0, SP_P, D, "bf16"))
+    total = 3 + steps
+    t0 = [T_START + 31 * s for s in range(B)]
+    q = dev(np.stack([synth.rows(SEED, synth.TID_Q, s, HQ, t0[s], total, D, "bf16")
+                      for s in range(B)], axis=1))
+    kn = dev(np.stack([synth.rows(SEED, synth.TID_K, s, HKV, t0[s], total, D, "bf16")
+                       for s in range(B)], axis=1))
+    vn = dev(np.stack([synth.rows(SEED, synth.TID_V, s, HKV, t0[s], total, D, "bf16")
+                       for s in range(B)], axis=1))
+    scale = 1.0 / math.sqrt(D)
+    res = {"workload": f"B={B} sequences sharing a {SP_P}-token pinned prefix, W={W}, "
+                       f"t>=65536, Hq={HQ} Hkv={HKV} d={D}, bf16 (ps_decode_step)",
+           "kv_bytes_per_step": B * HKV * (SP_P + W) * D * 2 * 2}
+    for mode in ("private", "shared"):
+        c = Cache(W, SP_P, HKV, D, PS_BF16, B)
+        for s in range(B):
+            c.seq_reset(s, (s * 613) % W)
+            if mode == "shared" and s > 0:
+                c.share_prefix(s, 0)
+            else:
+                c.prefill_prefix(s, kp, vp, SP_P)
+            c.import_window(s, t0[s],
+                            dev(synth.rows(SEED, synth.TID_K, s, HKV, t0[s] - W, W, D, "bf16")),
+                            dev(synth.rows(SEED, synth.TID_V, s, HKV, t0[s] - W, W, D, "bf16")),
+                            W, (s * 613) % W)
+        out = torch.empty((B, HQ, D), dtype=torch.bfloat16, device="cuda")
+        ws = c.decode_workspace(B, HQ)
+        ids = list(range(B))
+        pos = list(t0)
+
+        def step(i, st=None):
+            c.decode_step(q[i], kn[i], vn[i], ids, pos, HQ, scale, out, ws, st)
+            for s in range(B):
+                pos[s] += 1
+
+        for i in range(3):
+            step(i)
+        torch.cuda.synchronize()
+        ms = time_graph(torch, lambda i, st: step(3 + i, st), steps)
+        if c.device_error():
+            raise RuntimeError("device error word set by the shared-prefix decode")
+        res[f"{mode}_ms_per_step"] = round(ms, 5)
+        res[f"{mode}_tokens_per_s"] = round(B / (ms / 1e3), 1)
+        c.close()
+        torch.cuda.empty_cache()
+    res["speedup"] = round(res["private_ms_per_step"] / res["shared_ms_per_step"], 3)
+    return res
 
 
 # ------------------------------------------------------------ CPU oracle ----

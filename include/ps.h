@@ -92,7 +92,7 @@ PS_API void ps_cache_destroy(ps_cache* c);
 /* Return sequence `seq` to the empty state; its ring head starts at slot
  * ring_head_offset (0 <= offset < W).  Results do not depend on the offset
  * beyond float32 rounding order.
- * Errors: PS_EINVAL. */
+ * Errors: PS_EINVAL, PS_ESTATE (other sequences share this one's prefix). */
 PS_API int ps_seq_reset(ps_cache* c, int seq, int ring_head_offset, void* stream);
 
 /* Host mirror of a sequence's state (no device access). Errors: PS_EINVAL. */
@@ -107,6 +107,17 @@ PS_API int ps_seq_info_get(const ps_cache* c, int seq, ps_seq_info* out);
  * empty window.  Errors: PS_EINVAL, PS_ESTATE (sequence not empty). */
 PS_API int ps_prefill_prefix(ps_cache* c, int seq, const void* k, const void* v, int P_s,
                       void* stream);
+
+/* Let empty sequence `seq` use the pinned prefix of active sequence `src`
+ * instead of a copy of its own (prompt reuse, as in prefix caching): `seq`
+ * becomes active with the same P_s, next_pos = P_s and an empty window, and
+ * every kernel reads its prefix rows from the slab that holds src's prefix,
+ * so sequences sharing a prompt stream its keys and values from HBM once per
+ * L2 residency.  Results are exactly those of a private copy of the same rows.
+ * While any sequence shares a prefix, the sequence holding it cannot be reset
+ * (PS_ESTATE); resetting a sharer releases it.
+ * Errors: PS_EINVAL, PS_ESTATE (seq not empty, or src has no prefix). */
+PS_API int ps_share_prefix(ps_cache* c, int seq, int src, void* stream);
 
 /* Attention of prompt tokens t0..t0+n-1 of active sequence `seq`, all inside
  * its pinned prefix (0 <= t0, t0 + n <= P_s), over the prefix rows stored by

@@ -43,6 +43,7 @@ SIGNATURES = {
     "ps_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _f, _vp, _vp, _sz, _vp]),
     "ps_attend_chunk": (_i, [_vp, _i, _vp, _vp, _vp, _i64, _i, _i, _f, _vp, _i, _vp]),
     "ps_attend_prompt": (_i, [_vp, _i, _vp, _i64, _i, _i, _f, _vp, _vp]),
+    "ps_share_prefix": (_i, [_vp, _i, _i, _vp]),
     "ps_debug_wait_timeout": (_i, [_vp, ctypes.c_longlong, _vp]),
     "ps_export_window": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp]),
     "ps_import_window": (_i, [_vp, _i, _i64, _vp, _vp, _i, _i, _vp]),
@@ -187,6 +188,11 @@ def ps_attend_chunk(cache, seq, q, k_blk, v_blk, t0, n, Hq, scale, out, append_a
     _check("ps_attend_chunk", _lib.ps_attend_chunk(cache, seq, _ptr(q), _ptr(k_blk), _ptr(v_blk),
                                                    t0, n, Hq, scale, _ptr(out), int(append_after),
                                                    _stream(stream)))
+
+
+def ps_share_prefix(cache, seq, src, stream=None) -> None:
+    """Empty sequence `seq` reads the pinned prefix of sequence `src`."""
+    _check("ps_share_prefix", _lib.ps_share_prefix(cache, seq, src, _stream(stream)))
 
 
 def ps_attend_prompt(cache, seq, q, t0, n, Hq, scale, out, stream=None) -> None:

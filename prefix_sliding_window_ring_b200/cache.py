@@ -72,6 +72,9 @@ class Cache:
         abi.ps_attend_chunk(self.handle, seq, q, k_blk, v_blk, t0, n, Hq, scale, out, append_after,
                             stream)
 
+    def share_prefix(self, seq, src, stream=None):
+        abi.ps_share_prefix(self.handle, seq, src, stream)
+
     def attend_prompt(self, seq, q, t0, n, Hq, scale, out, stream=None):
         abi.ps_attend_prompt(self.handle, seq, q, t0, n, Hq, scale, out, stream)
 

@@ -46,6 +46,8 @@ struct SeqHost {
   int64_t next_pos;
   int32_t head;
   int32_t count;
+  int32_t owner = -1;   // sequence whose slab holds the prefix rows (itself unless shared)
+  int32_t sharers = 0;  // other sequences reading this one's prefix rows
 };
 
 struct Layout {
@@ -140,6 +142,7 @@ ps::DevMeta to_dev(const SeqHost& s) {
   m.P = s.P;
   m.head = s.head;
   m.count = s.count;
+  m.owner = s.owner;
   return m;
 }
 
@@ -216,9 +219,15 @@ int ps_seq_reset(ps_cache* c, int seq, int ring_head_offset, void* stream) {
   if (r) return r;
   if (ring_head_offset < 0 || ring_head_offset >= c->W)
     return fail(PS_EINVAL, "ring_head_offset %d not in [0,%d)", ring_head_offset, c->W);
+  const SeqHost cur = c->seqs[seq];
+  if (cur.sharers > 0)
+    return fail(PS_ESTATE, "sequence %d's prefix is read by %d other sequences (reset them first)",
+                seq, cur.sharers);
   if ((r = check_device(c))) return r;
   SeqHost s{0, 0, 0, ring_head_offset, 0};
+  s.owner = seq;
   PS_CUDA(ps::launch_meta_set(c->dev, seq, to_dev(s), (cudaStream_t)stream));
+  if (cur.state == 1 && cur.owner >= 0 && cur.owner != seq) c->seqs[cur.owner].sharers--;
   c->seqs[seq] = s;
   return ok();
 }
@@ -236,9 +245,28 @@ int ps_prefill_prefix(ps_cache* c, int seq, const void* k, const void* v, int P_
   cudaStream_t st = (cudaStream_t)stream;
   PS_CUDA(ps::launch_prefix_store(c->dev, c->esize, seq, k, v, P_s, st));
   SeqHost s = c->seqs[seq];
-  s.state = 1; s.P = P_s; s.next_pos = P_s; s.count = 0;
+  s.state = 1; s.P = P_s; s.next_pos = P_s; s.count = 0; s.owner = seq;
   PS_CUDA(ps::launch_meta_set(c->dev, seq, to_dev(s), st));
   c->seqs[seq] = s;
+  return ok();
+}
+
+int ps_share_prefix(ps_cache* c, int seq, int src, void* stream) {
+  if (!c) return fail(PS_EINVAL, "cache is NULL");
+  int r = check_seq(c, seq, false);
+  if (r) return r;
+  if ((r = check_seq(c, src, true))) return r;
+  if (seq == src) return fail(PS_EINVAL, "sequence %d cannot share its own prefix", seq);
+  if (c->seqs[seq].state != 0)
+    return fail(PS_ESTATE, "sequence %d already has a prefix (reset it first)", seq);
+  if ((r = check_device(c))) return r;
+  const int owner = c->seqs[src].owner;
+  SeqHost s = c->seqs[seq];
+  s.state = 1; s.P = c->seqs[src].P; s.next_pos = s.P; s.count = 0; s.owner = owner;
+  s.sharers = 0;
+  PS_CUDA(ps::launch_meta_set(c->dev, seq, to_dev(s), (cudaStream_t)stream));
+  c->seqs[seq] = s;
+  c->seqs[owner].sharers++;
   return ok();
 }
 
@@ -312,6 +340,7 @@ int ps_attend_decode(ps_cache* c, const void* q, const int* seq_ids, const int64
       ids.P[i] = s.P;
       ids.head[i] = s.head;
       ids.count[i] = s.count;
+      ids.owner[i] = s.owner;
       ids.t[i] = t[b0 + i];
     }
     PS_CUDA(ps::launch_decode(c->dev, c->dtype, G, ids, nb, Hq, (const char*)q + b0 * per_entry,
@@ -365,6 +394,7 @@ int ps_decode_step(ps_cache* c, const void* q, const void* k_new, const void* v_
       ids.P[i] = s.P;
       ids.head[i] = s.head;
       ids.count[i] = s.count;
+      ids.owner[i] = s.owner;
       ids.t[i] = t[b0 + i];
     }
     PS_CUDA(ps::launch_decode(c->dev, c->dtype, G, ids, nb, Hq, (const char*)q + b0 * per_entry,

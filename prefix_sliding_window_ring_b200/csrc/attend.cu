@@ -186,7 +186,9 @@ __device__ __forceinline__ void merge_warps(MergeSmem<G, D>& sm) {
 // Stream logical rows [j_begin, j_end) of `segs` straight from global memory
 // (warp w takes row groups w, w+kNW, ...); leave the CTA state in sm slot 0.
 template <typename T, int D, int G>
-__device__ __forceinline__ void stream_rows(const SegSet& segs, const T* __restrict__ kslab,
+__device__ __forceinline__ void stream_rows(const SegSet& segs, const T* __restrict__ kpre,
+                                            const T* __restrict__ vpre,
+                                            const T* __restrict__ kslab,
                                             const T* __restrict__ vslab,
                                             const T* __restrict__ kblk,
                                             const T* __restrict__ vblk, int64_t blk_stride,
@@ -213,9 +215,10 @@ __device__ __forceinline__ void stream_rows(const SegSet& segs, const T* __restr
         if (segs.src[si] == 2) {
           size_t r = (size_t)(segs.row0[si] + off) * blk_stride;
           kp = kblk + r; vp = vblk + r;
-        } else {
+        } else {  // prefix rows from the owner's slab, ring rows from the sequence's own
           size_t r = (size_t)(segs.row0[si] + off) * D;
-          kp = kslab + r; vp = vslab + r;
+          kp = (segs.src[si] == 0 ? kpre : kslab) + r;
+          vp = (segs.src[si] == 0 ? vpre : vslab) + r;
         }
         kr[u] = __ldcs((const uint4*)(kp + st.c * S::VEC));
         vr[u] = __ldcs((const uint4*)(vp + st.c * S::VEC));
@@ -263,9 +266,11 @@ __global__ void __launch_bounds__(kThreadsAttn) k_chunk_cc(AttnArgs a) {
     if (!segs.ring_ok) atomicOr(a.c.err, ERR_RING);
   }
   const size_t slab = ((size_t)a.seq * a.c.Hkv + g) * (size_t)a.c.slab_rows * D;
+  const size_t pslab = ((size_t)m.owner * a.c.Hkv + g) * (size_t)a.c.slab_rows * D;
   const int64_t bstride = (int64_t)a.c.Hkv * D;
   const T* qrow = (const T*)a.q + ((size_t)i * a.Hq + (size_t)g * G) * D;
-  stream_rows<T, D, G>(segs, (const T*)a.c.K + slab, (const T*)a.c.V + slab,
+  stream_rows<T, D, G>(segs, (const T*)a.c.K + pslab, (const T*)a.c.V + pslab,
+                       (const T*)a.c.K + slab, (const T*)a.c.V + slab,
                        (const T*)a.kb + (size_t)g * D, (const T*)a.vb + (size_t)g * D, bstride,
                        qrow, a.qscale, 0, segs.total, sm);
   T* orow = (T*)a.out + ((size_t)i * a.Hq + (size_t)g * G) * D;

@@ -77,7 +77,7 @@ struct __align__(1024) TcSmem {
 struct KSched {
   int n;
   int ntiles;
-  int src[4];       // 0: cache slab row, 1: block row
+  int src[4];       // 0: ring row of the sequence's slab, 1: block row, 2: prefix row (owner's slab)
   int64_t row0[4];  // first slab row / block row of the range
   int64_t pos0[4];  // position of that row
   int32_t len[4];
@@ -111,10 +111,10 @@ __device__ __forceinline__ KSched make_sched(const DevMeta& m, int W, int P_max,
   s.ntiles = 0;
   for (int i = 0; i < 4; ++i) { s.src[i] = 0; s.row0[i] = 0; s.pos0[i] = 0; s.len[i] = 0; s.tbase[i] = 0; }
   if (prompt) {
-    add_range(s, 0, 0, 0, phi + 1 < m.P ? phi + 1 : m.P);
+    add_range(s, 2, 0, 0, phi + 1 < m.P ? phi + 1 : m.P);
     return s;
   }
-  add_range(s, 0, 0, 0, m.P);  // pinned prefix
+  add_range(s, 2, 0, 0, m.P);  // pinned prefix
   int64_t lo = plo - W + 1;
   if (lo < m.P) lo = m.P;
   const int64_t base = m.next_pos - m.count;
@@ -218,6 +218,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
     // ------------------------------------------------------------ producer --
     if (lane == 0) {
       const int slab_z = a.seq * a.c.Hkv + g;
+      const int prefix_z = m.owner * a.c.Hkv + g;  // prefix rows live in the owner's slab
       int issued_k = 0, issued_v = 0;
       ptx::mbar_arrive_expect_tx(&q_full, 2 * kBM * 128);
       for (int hh = 0; hh < a.G; ++hh)
@@ -229,8 +230,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
         if (j >= 2 && !wait_bar(&k_empty[st], ((j >> 1) - 1) & 1, &abort_flag)) break;
         ptx::mbar_arrive_expect_tx(&k_full[st], kTileBytes);
         for (int b = 0; b < 2; ++b) {
-          if (kt.src == 0)
-            ptx::tma_load_3d(sm.k[st][b], &a.kslab, b * 64, (int32_t)kt.row, slab_z, &k_full[st]);
+          if (kt.src != 1)
+            ptx::tma_load_3d(sm.k[st][b], &a.kslab, b * 64, (int32_t)kt.row,
+                             kt.src == 2 ? prefix_z : slab_z, &k_full[st]);
           else
             ptx::tma_load_3d(sm.k[st][b], &a.kblk, b * 64, g, (int32_t)kt.row, &k_full[st]);
         }
@@ -238,8 +240,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
         if (j >= 2 && !wait_bar(&v_empty[st], ((j >> 1) - 1) & 1, &abort_flag)) break;
         ptx::mbar_arrive_expect_tx(&v_full[st], kTileBytes);
         for (int b = 0; b < 2; ++b) {
-          if (kt.src == 0)
-            ptx::tma_load_3d(sm.v[st][b], &a.vslab, b * 64, (int32_t)kt.row, slab_z, &v_full[st]);
+          if (kt.src != 1)
+            ptx::tma_load_3d(sm.v[st][b], &a.vslab, b * 64, (int32_t)kt.row,
+                             kt.src == 2 ? prefix_z : slab_z, &v_full[st]);
           else
             ptx::tma_load_3d(sm.v[st][b], &a.vblk, b * 64, g, (int32_t)kt.row, &v_full[st]);
         }
@@ -335,7 +338,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
         const KTile kt = tile_of(ks, j);
         // element masks only for tiles on a window or causal edge
         const bool full = kt.valid == kBN &&
-                          (kt.src == 0 && kt.pos0 + kBN <= P
+                          (kt.src == 2 && kt.pos0 + kBN <= P
                                ? true
                                : (kt.pos0 >= phi - W + 1 && kt.pos0 + kBN - 1 <= plo));
         if (!full) {

@@ -16,7 +16,8 @@ struct DevMeta {
   int32_t P;
   int32_t head;
   int32_t count;
-  int32_t pad[3];
+  int32_t owner;  // sequence whose slab holds the pinned prefix rows (itself unless shared)
+  int32_t pad[2];
 };
 static_assert(sizeof(DevMeta) == 32, "DevMeta layout");
 

@@ -92,10 +92,12 @@ struct DecodeArgs {
   int32_t P[kMaxBatchPerLaunch];      // prefix length of entry b
   int32_t head[kMaxBatchPerLaunch];   // physical ring slot of entry b's oldest window row
   int32_t count[kMaxBatchPerLaunch];  // ring rows of entry b
+  int32_t owner[kMaxBatchPerLaunch];  // sequence whose slab holds entry b's prefix rows
   int64_t t[kMaxBatchPerLaunch];
   int32_t tcum[kMaxBatchPerLaunch + 1];  // tcum[b] = Hkv * (tiles per head of entries before b)
 };
-static_assert(sizeof(DecodeArgs) <= 4096, "decode arguments fit the classic parameter space");
+// Kernel parameters above 4 KB need CUDA 12.1 and sm_70 or later (limit 32764 bytes).
+static_assert(sizeof(DecodeArgs) <= 32764, "decode arguments fit the kernel parameter space");
 
 // bfloat16 pairs of a 16-byte vector as float2 (exact widening).
 template <typename T> struct Vec2;
@@ -311,10 +313,10 @@ struct DecState {
   }
 };
 
-// Calls f(slab_row, dst_row, nrows) for the contiguous runs of the logical
-// rows [x0, x1) of one pair, dst_row counted from x0 (a tile may span the
-// prefix and both ring runs).  Sets *bad if the rows reach block rows (a
-// decode query never has them).
+// Calls f(src, slab_row, dst_row, nrows) for the contiguous runs of the
+// logical rows [x0, x1) of one pair (src 0: prefix rows, 1: ring rows),
+// dst_row counted from x0 (a tile may span the prefix and both ring runs).
+// Sets *bad if the rows reach block rows (a decode query never has them).
 template <typename F>
 __device__ __forceinline__ void for_each_run(const SegSet& s, int32_t x0, int32_t x1, bool* bad,
                                              F&& f) {
@@ -325,7 +327,7 @@ __device__ __forceinline__ void for_each_run(const SegSet& s, int32_t x0, int32_
       const int32_t lo = max(L, x0), hi = min(L + s.len[i], x1);
       if (hi > lo) {
         if (s.src[i] == 2) *bad = true;
-        else f(s.row0[i] + (lo - L), lo - x0, hi - lo);
+        else f(s.src[i], s.row0[i] + (lo - L), lo - x0, hi - lo);
       }
       L += s.len[i];
     }
@@ -434,10 +436,13 @@ __global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8)
       m.P = a.P[pt.b];
       m.head = a.head[pt.b];
       m.count = a.count[pt.b];
+      m.owner = a.owner[pt.b];
       const SegSet segs = build_segments(m, a.c.W, a.c.P_max, a.t[pt.b]);
       bool bad = segs.total != m.P + m.count || (segs.total + TR - 1) / TR != pt.tph;
       const bool step = a.knew != nullptr;  // the pair's last row comes from knew/vnew
       const size_t slab = ((size_t)s * Hkv + pt.g) * (size_t)a.c.slab_rows * D;
+      // prefix rows come from the slab of the sequence that owns them
+      const size_t pslab = ((size_t)a.owner[pt.b] * Hkv + pt.g) * (size_t)a.c.slab_rows * D;
       const int pair = pt.b * Hkv + pt.g;
       for (int32_t j = j0; j < j1 && alive; ++j) {
         const int32_t r0 = j * TR, r1 = min(segs.total, r0 + TR);
@@ -466,12 +471,11 @@ __global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8)
         T* kd = ktile + (size_t)st * TR * D;
         T* vd = vtile + (size_t)st * TR * D;
         for_each_run(segs, r0, with_new ? r1 - 1 : r1, &bad,
-                     [&](int64_t row, int32_t dst, int32_t nr) {
+                     [&](int src, int64_t row, int32_t dst, int32_t nr) {
           const uint32_t nb = (uint32_t)nr * D * sizeof(T);
-          ptx::bulk_g2s(kd + (size_t)dst * D, (const T*)a.c.K + slab + (size_t)row * D, nb,
-                        &full[st]);
-          ptx::bulk_g2s(vd + (size_t)dst * D, (const T*)a.c.V + slab + (size_t)row * D, nb,
-                        &full[st]);
+          const size_t base = (src == 0 ? pslab : slab) + (size_t)row * D;
+          ptx::bulk_g2s(kd + (size_t)dst * D, (const T*)a.c.K + base, nb, &full[st]);
+          ptx::bulk_g2s(vd + (size_t)dst * D, (const T*)a.c.V + base, nb, &full[st]);
         });
         if (with_new) {  // the appended token, straight from the caller's rows
           const size_t src = (size_t)pair * D;
@@ -491,7 +495,7 @@ __global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8)
         me.head = (int32_t)((md.head + (cn > W ? 1 : 0)) % W);
       }
       if (bad || me.next_pos != m.next_pos || me.P != m.P || me.head != m.head ||
-          me.count != m.count)
+          me.count != m.count || me.owner != m.owner)
         atomicOr(a.c.err, ERR_BATCH);
       if (!segs.ring_ok) atomicOr(a.c.err, ERR_RING);
     }
@@ -610,6 +614,7 @@ __global__ void __launch_bounds__(kMergeThreads) k_decode_merge(const __grid_con
     m.P = a.P[gi];
     m.head = a.head[gi];
     m.count = a.count[gi];
+    m.owner = a.owner[gi];
     a.c.meta[a.seq[gi]] = m;
   }
   if (gi >= (int64_t)a.B * Hkv * Q) return;
@@ -770,6 +775,7 @@ cudaError_t launch_decode(const CacheDev& c, int dtype, int G, const BatchIds& i
     a.P[b] = ids.P[b];
     a.head[b] = ids.head[b];
     a.count[b] = ids.count[b];
+    a.owner[b] = ids.owner[b];
     a.t[b] = ids.t[b];
   }
   if (dtype == 0) {

@@ -14,6 +14,7 @@ struct BatchIds {
   int32_t P[kMaxBatchPerLaunch];     // host bookkeeping of each entry's ring state
   int32_t head[kMaxBatchPerLaunch];
   int32_t count[kMaxBatchPerLaunch];
+  int32_t owner[kMaxBatchPerLaunch];  // sequence whose slab holds the prefix rows
   int64_t t[kMaxBatchPerLaunch];
 };
 
