@@ -28,7 +28,8 @@
  *    available from ps_last_error() in the calling thread.
  *  - The library owns only the opaque host object.  All device storage lives
  *    in the caller's buffer passed to ps_cache_create; decode scratch lives in
- *    the caller's workspace passed to ps_attend_decode.
+ *    the caller's workspace passed to ps_attend_decode / ps_decode_step (or in
+ *    the library's fixed array for ps_attend_decode_static).
  *  - Kernels never trap.  An internal inconsistency detected on the device sets
  *    an error word that ps_device_error() reads back.
  */
@@ -257,7 +258,6 @@ PS_API int ps_debug_wait_timeout(ps_cache* c, long long limit_cycles, void* stre
 
 /* Synchronise `stream` and read (then clear) the device error word:
  * *code = 0 when no kernel reported an inconsistency, else an OR of
- *   1  a split launch did not cover every visible row,
  *   2  a ring no longer holds the window a query needs,
  *   4  a batch entry's position or ring state disagrees with the device record,
  *   8  a pipeline wait gave up and the kernel stopped early (outputs of that

@@ -237,13 +237,9 @@ struct AttnArgs {
   const void* kb;
   const void* vb;
   float qscale;
-  float* part_ml;    // [B][Hkv][nsplit][G][2]
-  float* part_o;     // [B][Hkv][nsplit][G][D]
-  int32_t* tick;     // [B][Hkv]
-  int nsplit, chunk, Hq, b_off, seq;
+  int Hq, seq;
   int prompt;  // queries inside the prefix: causal over the prefix rows only
   int64_t t0;
-  BatchIds ids;
 };
 
 template <typename T, int D, int G>

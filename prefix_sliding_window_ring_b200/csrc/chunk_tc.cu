@@ -1,8 +1,12 @@
-// Chunked prefill/extend on the tcgen05 tensor cores (bf16, head_dim 128).
+// Chunked prefill/extend and prompt prefill on the tcgen05 tensor cores
+// (bf16, head_dim 128).
 //
 // A block of n queries at positions t0..t0+n-1 attends to the pinned prefix,
 // the ring entries of each query's window and the block itself, causally
-// ("Prefix Sliding" digest, sections 03 and 06).  One CTA takes a 128-row
+// ("Prefix Sliding" digest, sections 03 and 06); prompt queries (t < P)
+// attend to the prefix rows [0, t].  Prefix rows are read from the slab of the
+// sequence that owns them (itself, or the sequence whose prefix it shares).
+// One CTA takes a 128-row
 // query tile: 128/G consecutive positions of each of the G query heads that
 // share one key/value head, so every key tile feeds all G heads at once.
 //
@@ -11,12 +15,12 @@
 // the block rows -- so no evicted row is ever loaded; only tiles on a window
 // or causal edge are masked element by element.
 //
-// Roles (8 warps):
+// Roles (12 warps):
 //   warp 0   TMA producer: Q once, then K and V tiles into 2-stage rings
 //            (tensor-map tiled loads with 128-byte swizzle, no multicast);
 //   warp 1   MMA issuer: S_j = Q K_j^T into one of two TMEM buffers, then
 //            O += P_j V_j with P_j read from TMEM (kind::f16, f32 accumulate);
-//   warp 2   owns the TMEM allocation;
+//   warp 2   owns the TMEM allocation (S in two 128-column buffers, O);
 //   warps 4-11 softmax: each query row is shared by two threads (same TMEM
 //            lane, one half of the columns each), which exchange row maxima
 //            and sums through shared memory.  They load S_j from TMEM, mask,

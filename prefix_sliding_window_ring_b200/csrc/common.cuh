@@ -37,7 +37,6 @@ struct CacheDev {
 };
 
 enum : int32_t {
-  ERR_COVERAGE = 1,  // a split-K launch did not cover every visible row
   ERR_RING = 2,      // the ring does not hold the window a query needs
   ERR_BATCH = 4,     // a batch entry's position disagrees with the bookkeeping
   ERR_TIMEOUT = 8,   // a pipeline wait gave up (the kernel stopped early)

@@ -1,25 +1,33 @@
-// Decode attention (visible-range derivation, split streaming, split merge).
+// Decode attention (visible-range derivation, split streaming, split merge),
+// and the decode step that appends the token in the same pass.
 //
-// Work division.  The visible rows of all (batch entry, kv head) pairs of a
-// launch are laid end to end and cut into `nctas` equal ranges, one per CTA
-// (two CTAs per SM), so every SM streams the same number of rows whatever the
-// batch shape.  For every (range, pair) piece a CTA emits one partial (max,
-// sum, accumulator) triple; a small second grid, launched as a programmatic
-// dependent of the first, merges each pair's partials into the output.  The
-// producer hands each tile to the consumers with a small descriptor (pair,
-// rows, first/last of piece) next to the tile's data.  The ring state of each
-// entry (P, head, count) comes with the launch from the host's bookkeeping, so
-// no copy waits on a metadata load; the device record is checked alongside.
+// Work division.  Each (batch entry, kv head) pair's visible rows -- the
+// pinned prefix, then the ring window as at most two runs split at the
+// physical wrap -- are cut into tiles of TR consecutive rows (only a pair's
+// last tile is short; a tile may span the prefix/ring boundary or the wrap and
+// is then assembled from several bulk copies).  The tiles of all pairs are
+// laid end to end and CTA c of nctas (two per SM) streams tiles
+// [T c / nctas, T (c + 1) / nctas), so every CTA streams the same number of
+// tiles whatever the batch shape.  For every (CTA range, pair) piece a CTA
+// emits one partial (max, sum, accumulator) triple; a small second grid
+// merges each pair's partials into the output.  Both grids are programmatic
+// dependent launches of the kernel before them.  No evicted row is ever
+// fetched ("Prefix Sliding" digest, section 06: iterate the prefix blocks and
+// the window blocks separately).
 //
 // Streaming.  Warp kCW is the producer: one lane issues bulk async copies
-// (cp.async.bulk, no multicast) of contiguous K and V row tiles of 14 KiB each
-// into a kStages-deep shared-memory ring (bulk copies much smaller than that
-// leave HBM bandwidth unused).  A tile never crosses a visible range (prefix
-// rows, or one contiguous run of ring slots split at the physical wrap), so no
-// evicted row is ever fetched ("Prefix Sliding" digest, section 06: iterate
-// the prefix blocks and the window blocks separately).  Each of the kCW
-// consumer warps takes its own share of every tile and keeps its own
-// online-softmax state; a stage is refilled once all of them have released it.
+// (cp.async.bulk, no multicast) of K and V tiles of 14 KiB each into a
+// kStages-deep shared-memory ring (much smaller copies leave HBM bandwidth
+// unused), with a small descriptor per tile (pair, rows, first/last of piece,
+// partial slot); the first tile of a piece also brings the pair's q rows.
+// Each entry's ring state comes with the launch from the host's bookkeeping,
+// so no copy waits on a metadata load; the device record is checked alongside.
+// Prefix rows come from the slab of the sequence that owns them (a shared
+// prefix); in a decode step the pair's last row, the appended token, comes
+// from the caller's buffer and is stored to its ring slot by the consumer warp
+// that holds it.  Each of the kCW consumer warps takes its own share of every
+// tile and keeps its own online-softmax state; a stage is refilled once all of
+// them have released it.
 //
 // Consumer arithmetic (per warp, LPR lanes per row, 8 scores per update):
 // each lane forms partial dot products for 8 (row, query head) scores, a
