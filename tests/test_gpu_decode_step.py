@@ -146,3 +146,70 @@ def test_step_rejects_wrong_positions_without_side_effects():
     assert (info.next_pos, info.count) == (P, 0)
     c.decode_step(q, kn, vn, [0], [P], Hq, 0.125, out)
     assert c.seq_info(0).next_pos == P + 1 and c.device_error() == 0
+
+
+SHAPES = [("f32", 64, 1, 1), ("bf16", 64, 4, 2), ("bf16", 128, 8, 2), ("f32", 128, 2, 2),
+          ("bf16", 128, 1, 4)]
+
+
+@pytest.mark.parametrize("dtype,d,G,Hkv", SHAPES,
+                         ids=[f"{dt}-d{d}-G{G}-Hkv{h}" for dt, d, G, h in SHAPES])
+def test_step_every_head_shape(dtype, d, G, Hkv):
+    """Every head_dim / GQA group size the decode kernel is built for: a few
+    steps across the just-full boundary, fused vs split bit-exact, oracle."""
+    W, P = 40, 7
+    Hq = G * Hkv
+    sd = SeqData(12, 3, Hq, Hkv, d, dtype)
+    scale = default_scale(d)
+    T = P + W + 6
+    kall, vall = to_torch(sd.k(0, T)), to_torch(sd.v(0, T))
+    qall = to_torch(sd.q(0, T))
+    fused = Cache(W, P, Hkv, d, ps_dtype(dtype), 1)
+    split = Cache(W, P, Hkv, d, ps_dtype(dtype), 1)
+    for c in (fused, split):
+        c.seq_reset(0, 11)
+        c.prefill_prefix(0, kall[:P], vall[:P], P)
+        c.append_kv([0], kall[P:P + W - 3], vall[P:P + W - 3], W - 3)
+    steps = list(range(P + W - 3, T))
+    out_f = torch.empty((len(steps), Hq, d), dtype=kall.dtype, device="cuda")
+    out_s = torch.empty_like(out_f)
+    for i, t in enumerate(steps):
+        fused.decode_step(qall[t:t + 1], kall[t:t + 1], vall[t:t + 1], [0], [t], Hq, scale,
+                          out_f[i:i + 1])
+        split.append_kv([0], kall[t:t + 1], vall[t:t + 1], 1)
+        split.attend_decode(qall[t:t + 1], [0], [t], Hq, scale, out_s[i:i + 1])
+    assert fused.device_error() == 0 and split.device_error() == 0
+    assert torch.equal(_bits(out_f), _bits(out_s))
+    _same_state(fused, split, [0], "every-shape")
+    batch = oracle.Batch()
+    exp = [oracle_decode(batch, sd, P, W, t, scale, to_f64(qall[t])) for t in steps]
+    batch.run()
+    exp = np.stack([np.concatenate(e, axis=0) for e in exp])
+    check_close(to_f64(out_f), exp, dtype, f"step {dtype} d={d} G={G}")
+
+
+def test_step_batch_larger_than_one_launch():
+    """150 sequences in one call (two launches of at most 128 entries)."""
+    W, P, Hq, Hkv, d, B = 16, 3, 4, 2, 64, 150
+    scale = default_scale(d)
+    sds = [SeqData(13, b, Hq, Hkv, d, "f32") for b in range(B)]
+    ts = [P + 5 + (b % 23) for b in range(B)]
+    fused = Cache(W, P, Hkv, d, ps_dtype("f32"), B)
+    split = Cache(W, P, Hkv, d, ps_dtype("f32"), B)
+    for c in (fused, split):
+        for b, (sd, t) in enumerate(zip(sds, ts)):
+            c.seq_reset(b, b % W)
+            c.prefill_prefix(b, to_torch(sd.k(0, P)), to_torch(sd.v(0, P)), P)
+            n = min(W, t - P)
+            c.import_window(b, t, to_torch(sd.k(t - n, n)), to_torch(sd.v(t - n, n)), n, (5 * b) % W)
+    q = torch.stack([to_torch(sd.q(t, 1))[0] for sd, t in zip(sds, ts)])
+    kn = torch.stack([to_torch(sd.k(t, 1))[0] for sd, t in zip(sds, ts)])
+    vn = torch.stack([to_torch(sd.v(t, 1))[0] for sd, t in zip(sds, ts)])
+    ids = list(range(B))
+    out_f, out_s = torch.empty_like(q), torch.empty_like(q)
+    fused.decode_step(q, kn, vn, ids, ts, Hq, scale, out_f)
+    split.append_kv(ids, kn, vn, 1)
+    split.attend_decode(q, ids, ts, Hq, scale, out_s)
+    assert fused.device_error() == 0 and split.device_error() == 0
+    assert torch.equal(_bits(out_f), _bits(out_s))
+    _same_state(fused, split, [0, 127, 128, 149], "B=150")
