@@ -365,21 +365,22 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.empty_cache()
 
     # ---- end to end through the public API with host buffers ----
-    def host_inputs(r, v):
-        return hk[r][v], hv[r][v], hq[r][v]
-    hk = [wl.k_pool[r].cpu().pin_memory() for r in range(ROT)]
-    hv = [wl.v_pool[r].cpu().pin_memory() for r in range(ROT)]
-    hq = [wl.q_pool[r].cpu().pin_memory() for r in range(ROT)]
+    # Each step's inputs sit in one pinned host record [q | k | v] and cross
+    # to the device in one copy; the call gets views of the device copy.
+    nq, nk = B * HQ * D, B * HKV * D
+    hin = [torch.cat([wl.q_pool[r].reshape(wl.visits, -1), wl.k_pool[r].reshape(wl.visits, -1),
+                      wl.v_pool[r].reshape(wl.visits, -1)], dim=1).cpu().pin_memory()
+           for r in range(ROT)]
     hout = torch.empty((B, HQ, D), dtype=torch.bfloat16).pin_memory()
-    dk = torch.empty((B, HKV, D), dtype=torch.bfloat16, device="cuda")
-    dv, dq = torch.empty_like(dk), torch.empty((B, HQ, D), dtype=torch.bfloat16, device="cuda")
+    din = torch.empty(nq + 2 * nk, dtype=torch.bfloat16, device="cuda")
+    dq = din[:nq].view(B, HQ, D)
+    dk = din[nq:nq + nk].view(B, HKV, D)
+    dv = din[nq + nk:].view(B, HKV, D)
 
     def e2e_step(i):
         r = i % ROT
         v = wl.visit[r]
-        dk.copy_(hk[r][v], non_blocking=True)
-        dv.copy_(hv[r][v], non_blocking=True)
-        dq.copy_(hq[r][v], non_blocking=True)
+        din.copy_(hin[r][v], non_blocking=True)
         out = wl.step(i, host=lambda r_, v_: (dk, dv, dq))
         hout.copy_(out, non_blocking=True)
 
