@@ -409,10 +409,11 @@ def run_ours(args, rank, world, local_rank):
     prefill = None
     if rank == 0 and not args.no_prefill:
         prefill = prefill_measure(max(3, min(args.steps, 10)))
-    ragged = shared = None
+    ragged = shared = paged = None
     if rank == 0 and not args.no_prefill:
         ragged = ragged_measure(max(3, min(args.steps, 10)))
         shared = shared_prefix_measure(max(3, min(args.steps, 10)))
+        paged = paged_measure(max(3, min(args.steps, 10)))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -446,6 +447,7 @@ def run_ours(args, rank, world, local_rank):
         "prefix_overhead": overhead,
         "ragged": ragged,
         "shared_prefix": shared,
+        "paged": paged,
     }
     print(json.dumps(line), flush=True)
 
@@ -710,6 +712,68 @@ def shared_prefix_measure(steps: int):
         c.close()
         torch.cuda.empty_cache()
     res["speedup"] = round(res["private_ms_per_step"] / res["shared_ms_per_step"], 3)
+    return res
+
+
+def paged_measure(steps: int):
+    """Paged ring (block-table indirection): the decode step of the headline
+    workload (B=8, Hq=16, Hkv=8, d=128, P=128, W=4096, bf16, window full) on an
+    unpaged cache and on paged caches with 256- and 16-row pages.  Every cache
+    is filled the same way -- the prefix, then the window appended to all eight
+    sequences one page-sized piece at a time -- so a paged cache's pages are
+    interleaved across sequences in the pool, as they are when sequences grow
+    side by side.  The visible K/V per step is the same in every mode."""
+    import torch
+
+    import synth
+    from prefix_sliding_window_ring_b200 import PS_BF16, Cache
+
+    def dev(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+
+    total = 3 + steps
+    kp = [synth.rows(SEED, synth.TID_K, s, HKV, 0, P + W + total, D, "bf16") for s in range(B)]
+    vp = [synth.rows(SEED, synth.TID_V, s, HKV, 0, P + W + total, D, "bf16") for s in range(B)]
+    kall = dev(np.stack(kp))  # [B][P + W + total][Hkv][d]
+    vall = dev(np.stack(vp))
+    q = dev(np.stack([synth.rows(SEED, synth.TID_Q, s, HQ, P + W, total, D, "bf16")
+                      for s in range(B)], axis=1))
+    scale = 1.0 / math.sqrt(D)
+    res = {"workload": f"B={B}, Hq={HQ} Hkv={HKV} d={D}, P={P}, W={W}, window full, bf16 "
+                       "(ps_decode_step); pages interleaved across sequences",
+           "kv_bytes_per_step": kv_bytes_per_step()}
+    ids = list(range(B))
+    for page in (0, 256, 16):
+        c = Cache(W, P, HKV, D, PS_BF16, B, page_rows=page, num_pages=B * W // page if page else 0)
+        piece = page if page else 256
+        for s in range(B):
+            c.seq_reset(s, (s * 613) % W)
+            c.prefill_prefix(s, kall[s, :P], vall[s, :P], P)
+        for p0 in range(P, P + W, piece):
+            c.append_kv(ids, kall[:, p0:p0 + piece].contiguous(), vall[:, p0:p0 + piece].contiguous(),
+                        piece)
+        out = torch.empty((B, HQ, D), dtype=torch.bfloat16, device="cuda")
+        ws = c.decode_workspace(B, HQ)
+        pos = [P + W] * B
+        kn = kall[:, P + W:].transpose(0, 1).contiguous()  # [total][B][Hkv][d]
+        vn = vall[:, P + W:].transpose(0, 1).contiguous()
+
+        def step(i, st=None):
+            c.decode_step(q[i], kn[i], vn[i], ids, pos, HQ, scale, out, ws, st)
+            for s in range(B):
+                pos[s] += 1
+
+        for i in range(3):
+            step(i)
+        torch.cuda.synchronize()
+        ms = time_graph(torch, lambda i, st: step(3 + i, st), steps)
+        if c.device_error():
+            raise RuntimeError("device error word set by the paged decode")
+        key = f"page_rows_{page}" if page else "unpaged"
+        res[key] = {"us_per_step": round(ms * 1e3, 2),
+                    "GBps": round(kv_bytes_per_step() / (ms / 1e3) / 1e9, 1)}
+        c.close()
+        torch.cuda.empty_cache()
     return res
 
 

@@ -87,6 +87,28 @@ PS_API size_t ps_cache_bytes(int W, int P_max, int Hkv, int d, int dtype, int ma
 PS_API int ps_cache_create(int W, int P_max, int Hkv, int d, int dtype, int max_seqs,
                     void* dev_buf, size_t dev_bytes, void* stream, ps_cache** out);
 
+/* Paged ring (block-table indirection, vLLM-style): the same cache with each
+ * sequence's W ring slots split into W / page_rows pages that live in a pool
+ * of num_pages physical pages shared by all sequences, mapped through a page
+ * table.  A page is taken from the pool when an append, decode step, chunk
+ * append or window import first writes one of its slots, and returns to the
+ * pool when the sequence is reset; so memory follows the tokens actually held
+ * rather than max_seqs * W.  Every call behaves exactly as on an unpaged cache
+ * (same results, bit for bit), except that a write needing a page when the
+ * pool is empty fails with PS_ENOMEM and changes nothing.  Requires
+ * 1 <= page_rows <= W, W % page_rows == 0, num_pages >= 1; the tensor-core
+ * chunk kernel needs page_rows % 128 == 0 (other page sizes use the CUDA-core
+ * chunk kernel).  ps_cache_bytes_paged returns 0 for an invalid shape. */
+PS_API size_t ps_cache_bytes_paged(int W, int P_max, int Hkv, int d, int dtype, int max_seqs,
+                                   int page_rows, int num_pages);
+PS_API int ps_cache_create_paged(int W, int P_max, int Hkv, int d, int dtype, int max_seqs,
+                                 int page_rows, int num_pages, void* dev_buf, size_t dev_bytes,
+                                 void* stream, ps_cache** out);
+
+/* Physical ring pages left in the pool of a paged cache (host bookkeeping, no
+ * device access).  Errors: PS_EINVAL (NULL or unpaged cache). */
+PS_API int ps_ring_pages_free(const ps_cache* c);
+
 /* Free the host object (the device buffer stays the caller's). NULL is a no-op. */
 PS_API void ps_cache_destroy(ps_cache* c);
 

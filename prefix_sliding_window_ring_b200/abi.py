@@ -31,6 +31,10 @@ class SeqInfo(ctypes.Structure):
 
 SIGNATURES = {
     "ps_cache_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "ps_cache_bytes_paged": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i]),
+    "ps_cache_create_paged": (_i, [_i, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp,
+                                   ctypes.POINTER(_vp)]),
+    "ps_ring_pages_free": (_i, [_vp]),
     "ps_cache_create": (_i, [_i, _i, _i, _i, _i, _i, _vp, _sz, _vp, ctypes.POINTER(_vp)]),
     "ps_cache_destroy": (None, [_vp]),
     "ps_seq_reset": (_i, [_vp, _i, _i, _vp]),
@@ -119,6 +123,26 @@ def ps_cache_create(W, P_max, Hkv, d, dtype, max_seqs, dev_buf, dev_bytes, strea
     _check("ps_cache_create", _lib.ps_cache_create(W, P_max, Hkv, d, dtype, max_seqs, _ptr(dev_buf),
                                                    dev_bytes, _stream(stream), ctypes.byref(h)))
     return h
+
+
+def ps_cache_bytes_paged(W, P_max, Hkv, d, dtype, max_seqs, page_rows, num_pages) -> int:
+    return int(_lib.ps_cache_bytes_paged(W, P_max, Hkv, d, dtype, max_seqs, page_rows, num_pages))
+
+
+def ps_cache_create_paged(W, P_max, Hkv, d, dtype, max_seqs, page_rows, num_pages, dev_buf,
+                          dev_bytes, stream=None):
+    h = _vp()
+    _check("ps_cache_create_paged",
+           _lib.ps_cache_create_paged(W, P_max, Hkv, d, dtype, max_seqs, page_rows, num_pages,
+                                      _ptr(dev_buf), dev_bytes, _stream(stream), ctypes.byref(h)))
+    return h
+
+
+def ps_ring_pages_free(cache) -> int:
+    r = int(_lib.ps_ring_pages_free(cache))
+    if r < 0:
+        _check("ps_ring_pages_free", r)
+    return r
 
 
 def ps_cache_destroy(cache) -> None:

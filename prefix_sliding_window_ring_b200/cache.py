@@ -12,16 +12,28 @@ class Cache:
     """Owns the device buffer of one ps_cache and forwards calls to the C ABI."""
 
     def __init__(self, W: int, P_max: int, Hkv: int, d: int, dtype: int, max_seqs: int,
-                 device="cuda", stream=None):
+                 device="cuda", stream=None, page_rows: int = 0, num_pages: int = 0):
+        """page_rows > 0 makes a paged ring (num_pages physical pages of page_rows slots)."""
         self.W, self.P_max, self.Hkv, self.d, self.dtype, self.max_seqs = W, P_max, Hkv, d, dtype, max_seqs
         self.torch_dtype = TORCH_DTYPE[dtype]
-        self.nbytes = abi.ps_cache_bytes(W, P_max, Hkv, d, dtype, max_seqs)
+        if page_rows > 0:
+            self.nbytes = abi.ps_cache_bytes_paged(W, P_max, Hkv, d, dtype, max_seqs, page_rows,
+                                                   num_pages)
+        else:
+            self.nbytes = abi.ps_cache_bytes(W, P_max, Hkv, d, dtype, max_seqs)
         if self.nbytes == 0:
             raise abi.PSError("ps_cache_bytes", abi.PS_EINVAL, "invalid cache shape")
         self.buf = torch.empty(self.nbytes, dtype=torch.uint8, device=device)
-        self.handle = abi.ps_cache_create(W, P_max, Hkv, d, dtype, max_seqs, self.buf, self.nbytes,
-                                          stream)
+        if page_rows > 0:
+            self.handle = abi.ps_cache_create_paged(W, P_max, Hkv, d, dtype, max_seqs, page_rows,
+                                                    num_pages, self.buf, self.nbytes, stream)
+        else:
+            self.handle = abi.ps_cache_create(W, P_max, Hkv, d, dtype, max_seqs, self.buf,
+                                              self.nbytes, stream)
         self._ws = {}
+
+    def ring_pages_free(self) -> int:
+        return abi.ps_ring_pages_free(self.handle)
 
     def close(self) -> None:
         if getattr(self, "handle", None) is not None:

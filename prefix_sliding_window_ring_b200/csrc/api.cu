@@ -48,30 +48,42 @@ struct SeqHost {
   int32_t count;
   int32_t owner = -1;   // sequence whose slab holds the prefix rows (itself unless shared)
   int32_t sharers = 0;  // other sequences reading this one's prefix rows
+  std::vector<int32_t> pages;  // paged cache: physical page of each ring page (-1: none yet)
 };
 
 struct Layout {
-  size_t meta, tickets, err, pos, K, V, total;
+  size_t meta, tickets, err, pos, ptab, K, V, total;
 };
 
 size_t al(size_t x) { return (x + 255) & ~(size_t)255; }
 
 int esize_of(int dtype) { return dtype == PS_F32 ? 4 : (dtype == PS_BF16 ? 2 : 0); }
 
-bool make_layout(int W, int P_max, int Hkv, int d, int dtype, int S, Layout* L) {
+// page_rows == 0: unpaged, each sequence's ring inside its own slab
+// [Hkv][P_max + W]; otherwise ring pages of page_rows slots come from a pool of
+// nphys pages after the prefix slabs [S][Hkv][P_max].
+bool make_layout(int W, int P_max, int Hkv, int d, int dtype, int S, int page_rows, int nphys,
+                 Layout* L) {
   int es = esize_of(dtype);
   if (W < 1 || W > (1 << 28) || P_max < 0 || P_max > (1 << 28) || Hkv < 1 || Hkv > 1024 ||
       S < 1 || S > (1 << 20) || es == 0)
     return false;
   if (d != 64 && d != 128) return false;
+  const bool paged = page_rows > 0;
+  if (paged && (page_rows > W || W % page_rows != 0 || nphys < 1 || nphys > (1 << 24)))
+    return false;
+  const size_t pr = paged ? (size_t)page_rows : (size_t)W;
+  const size_t np = paged ? (size_t)nphys : (size_t)S;
   size_t off = 0;
   L->meta = off; off += al((size_t)S * sizeof(ps::DevMeta));
   L->tickets = off; off += al((size_t)S * sizeof(int32_t));
   L->err = off; off += 256;
-  L->pos = off; off += al((size_t)S * W * sizeof(int64_t));
-  size_t slab = (size_t)S * Hkv * ((size_t)P_max + W) * d * es;
-  L->K = off; off += al(slab);
-  L->V = off; off += al(slab);
+  L->pos = off; off += al(np * pr * sizeof(int64_t));
+  L->ptab = off; off += paged ? al((size_t)S * (W / page_rows) * sizeof(int32_t)) : 0;
+  const size_t rows = paged ? (size_t)S * Hkv * P_max + np * Hkv * pr
+                            : (size_t)S * Hkv * ((size_t)P_max + W);
+  L->K = off; off += al(rows * d * es);
+  L->V = off; off += al(rows * d * es);
   L->total = off;
   return true;
 }
@@ -82,6 +94,8 @@ bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
 
 struct ps_cache {
   int W, P_max, Hkv, d, dtype, S, esize;
+  bool paged;
+  std::vector<int32_t> free_pages;  // paged: physical ring pages not held by any sequence
   char* base;
   size_t bytes;
   int device;
@@ -127,6 +141,33 @@ int check_group(const ps_cache* c, int Hq, int* G) {
   return PS_OK;
 }
 
+// Paged cache: ring slots [slot0, slot0 + n) (mod W) of sequence `seq` are
+// about to be written.  Assigns a physical page to every ring page they touch
+// that has none yet, taking pages from `avail` and recording the page-table
+// entries to set; `pages` is the sequence's page list to update.  Returns
+// false if the pool runs out (the caller then changes nothing).
+bool plan_pages(const ps_cache* c, int seq, std::vector<int32_t>& pages, int64_t slot0, int64_t n,
+                std::vector<int32_t>& avail, std::vector<int32_t>& idx,
+                std::vector<int32_t>& phys) {
+  if (!c->paged || n <= 0) return true;
+  const int64_t W = c->W, pr = c->dev.page_rows;
+  int64_t s = ((slot0 % W) + W) % W;
+  for (int64_t left = n < W ? n : W; left > 0;) {
+    const int64_t page = s / pr;
+    const int64_t chunk = pr - s % pr < left ? pr - s % pr : left;
+    if (pages[page] < 0) {
+      if (avail.empty()) return false;
+      pages[page] = avail.back();
+      avail.pop_back();
+      idx.push_back((int32_t)(seq * (int64_t)c->dev.npg + page));
+      phys.push_back(pages[page]);
+    }
+    left -= chunk;
+    s = (s + chunk) % W;
+  }
+  return true;
+}
+
 void advance(SeqHost& s, int W, int64_t n) {
   int64_t cn = (int64_t)s.count + n;
   int64_t adv = cn - W > 0 ? cn - W : 0;
@@ -154,21 +195,21 @@ const char* ps_last_error(void) { return g_err.c_str(); }
 
 const char* ps_version(void) { return "prefix_sliding_window_ring_b200 0.1 (sm_100a)"; }
 
-size_t ps_cache_bytes(int W, int P_max, int Hkv, int d, int dtype, int max_seqs) {
-  Layout L;
-  if (!make_layout(W, P_max, Hkv, d, dtype, max_seqs, &L)) return 0;
-  return L.total;
-}
+}  // extern "C"
 
-int ps_cache_create(int W, int P_max, int Hkv, int d, int dtype, int max_seqs, void* dev_buf,
-                    size_t dev_bytes, void* stream, ps_cache** out) {
+namespace {
+
+int create_cache(int W, int P_max, int Hkv, int d, int dtype, int max_seqs, int page_rows,
+                 int num_pages, void* dev_buf, size_t dev_bytes, void* stream, ps_cache** out) {
   if (!out) return fail(PS_EINVAL, "out is NULL");
   *out = nullptr;
   if (d != 64 && d != 128) return fail(PS_EUNSUPPORTED, "head_dim %d not in {64,128}", d);
   Layout L;
-  if (!make_layout(W, P_max, Hkv, d, dtype, max_seqs, &L))
-    return fail(PS_EINVAL, "invalid cache shape W=%d P_max=%d Hkv=%d d=%d dtype=%d seqs=%d", W,
-                P_max, Hkv, d, dtype, max_seqs);
+  if (!make_layout(W, P_max, Hkv, d, dtype, max_seqs, page_rows, num_pages, &L))
+    return fail(PS_EINVAL,
+                "invalid cache shape W=%d P_max=%d Hkv=%d d=%d dtype=%d seqs=%d page_rows=%d "
+                "pages=%d",
+                W, P_max, Hkv, d, dtype, max_seqs, page_rows, num_pages);
   if (!dev_buf || ((uintptr_t)dev_buf & 255))
     return fail(PS_EINVAL, "dev_buf must be a non-NULL 256-byte aligned device pointer");
   if (dev_bytes < L.total)
@@ -181,9 +222,11 @@ int ps_cache_create(int W, int P_max, int Hkv, int d, int dtype, int max_seqs, v
   PS_CUDA(cudaDeviceGetAttribute(&sm, cudaDevAttrMultiProcessorCount, attr.device));
   cudaStream_t st = (cudaStream_t)stream;
   PS_CUDA(cudaMemsetAsync(dev_buf, 0, L.total, st));
+  const bool paged = page_rows > 0;
   ps_cache* c = new ps_cache();
   c->W = W; c->P_max = P_max; c->Hkv = Hkv; c->d = d; c->dtype = dtype; c->S = max_seqs;
   c->esize = esize_of(dtype);
+  c->paged = paged;
   c->base = (char*)dev_buf;
   c->bytes = dev_bytes;
   c->device = attr.device;
@@ -194,11 +237,62 @@ int ps_cache_create(int W, int P_max, int Hkv, int d, int dtype, int max_seqs, v
   c->dev.pos = (int64_t*)(c->base + L.pos);
   c->dev.K = c->base + L.K;
   c->dev.V = c->base + L.V;
+  c->dev.page_table = paged ? (int32_t*)(c->base + L.ptab) : nullptr;
   c->dev.W = W; c->dev.P_max = P_max; c->dev.Hkv = Hkv; c->dev.d = d; c->dev.S = max_seqs;
-  c->dev.slab_rows = (int64_t)P_max + W;
-  c->seqs.assign(max_seqs, SeqHost{0, 0, 0, 0, 0});
+  c->dev.page_rows = paged ? page_rows : W;
+  c->dev.npg = paged ? W / page_rows : 1;
+  c->dev.nphys = paged ? num_pages : max_seqs;
+  c->dev.pstride = paged ? P_max : (int64_t)P_max + W;
+  c->dev.rstride = paged ? page_rows : (int64_t)P_max + W;
+  c->dev.rbase = paged ? (int64_t)max_seqs * Hkv * P_max : P_max;
+  SeqHost empty{0, 0, 0, 0, 0};
+  if (paged) {
+    empty.pages.assign(c->dev.npg, -1);
+    for (int p = num_pages - 1; p >= 0; --p) c->free_pages.push_back(p);  // page 0 first
+  }
+  c->seqs.assign(max_seqs, empty);
   *out = c;
   return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ps_cache_bytes(int W, int P_max, int Hkv, int d, int dtype, int max_seqs) {
+  Layout L;
+  if (!make_layout(W, P_max, Hkv, d, dtype, max_seqs, 0, 0, &L)) return 0;
+  return L.total;
+}
+
+size_t ps_cache_bytes_paged(int W, int P_max, int Hkv, int d, int dtype, int max_seqs,
+                            int page_rows, int num_pages) {
+  Layout L;
+  if (page_rows < 1 || !make_layout(W, P_max, Hkv, d, dtype, max_seqs, page_rows, num_pages, &L))
+    return 0;
+  return L.total;
+}
+
+int ps_cache_create(int W, int P_max, int Hkv, int d, int dtype, int max_seqs, void* dev_buf,
+                    size_t dev_bytes, void* stream, ps_cache** out) {
+  return create_cache(W, P_max, Hkv, d, dtype, max_seqs, 0, 0, dev_buf, dev_bytes, stream, out);
+}
+
+int ps_cache_create_paged(int W, int P_max, int Hkv, int d, int dtype, int max_seqs,
+                          int page_rows, int num_pages, void* dev_buf, size_t dev_bytes,
+                          void* stream, ps_cache** out) {
+  if (page_rows < 1) {
+    if (out) *out = nullptr;
+    return fail(PS_EINVAL, "page_rows=%d must be at least 1", page_rows);
+  }
+  return create_cache(W, P_max, Hkv, d, dtype, max_seqs, page_rows, num_pages, dev_buf,
+                      dev_bytes, stream, out);
+}
+
+int ps_ring_pages_free(const ps_cache* c) {
+  if (!c) return fail(PS_EINVAL, "cache is NULL");
+  if (!c->paged) return fail(PS_EINVAL, "the cache is not paged");
+  return (int)c->free_pages.size();
 }
 
 void ps_cache_destroy(ps_cache* c) { delete c; }
@@ -228,6 +322,11 @@ int ps_seq_reset(ps_cache* c, int seq, int ring_head_offset, void* stream) {
   s.owner = seq;
   PS_CUDA(ps::launch_meta_set(c->dev, seq, to_dev(s), (cudaStream_t)stream));
   if (cur.state == 1 && cur.owner >= 0 && cur.owner != seq) c->seqs[cur.owner].sharers--;
+  if (c->paged) {  // its ring pages go back to the pool
+    for (int32_t p : cur.pages)
+      if (p >= 0) c->free_pages.push_back(p);
+    s.pages.assign(c->dev.npg, -1);
+  }
   c->seqs[seq] = s;
   return ok();
 }
@@ -280,7 +379,20 @@ int ps_append_kv(ps_cache* c, const int* seq_ids, int B, const void* k, const vo
   if (!k || !v || !aligned16(k) || !aligned16(v))
     return fail(PS_EINVAL, "k/v must be non-NULL 16-byte aligned device pointers");
   if ((r = check_device(c))) return r;
+  // paged: ring pages for the slots the appends write (the last min(n, W) tokens)
+  std::vector<int32_t> avail = c->free_pages, idx, phys;
+  std::vector<std::vector<int32_t>> pages(B);
+  for (int b = 0; b < B; ++b) {
+    const SeqHost& s = c->seqs[seq_ids[b]];
+    pages[b] = s.pages;
+    const int64_t n_eff = n < c->W ? n : c->W;
+    if (!plan_pages(c, seq_ids[b], pages[b], (int64_t)s.head + s.count + (n - n_eff), n_eff,
+                    avail, idx, phys))
+      return fail(PS_ENOMEM, "the ring page pool has no free page left");
+  }
   cudaStream_t st = (cudaStream_t)stream;
+  if (!idx.empty())
+    PS_CUDA(ps::launch_page_set(c->dev, idx.data(), phys.data(), (int)idx.size(), st));
   size_t per_entry = (size_t)n * c->Hkv * c->d * c->esize;
   for (int b0 = 0; b0 < B; b0 += ps::kMaxBatchPerLaunch) {
     int nb = B - b0 < ps::kMaxBatchPerLaunch ? B - b0 : ps::kMaxBatchPerLaunch;
@@ -290,7 +402,11 @@ int ps_append_kv(ps_cache* c, const int* seq_ids, int B, const void* k, const vo
     PS_CUDA(ps::launch_ring_append(c->dev, c->esize, ids, nb, (const char*)k + b0 * per_entry,
                                    (const char*)v + b0 * per_entry, n, st));
   }
-  for (int b = 0; b < B; ++b) advance(c->seqs[seq_ids[b]], c->W, n);
+  c->free_pages = avail;
+  for (int b = 0; b < B; ++b) {
+    c->seqs[seq_ids[b]].pages = pages[b];
+    advance(c->seqs[seq_ids[b]], c->W, n);
+  }
   return ok();
 }
 
@@ -380,7 +496,18 @@ int ps_decode_step(ps_cache* c, const void* q, const void* k_new, const void* v_
   if (need > workspace_bytes)
     return fail(PS_ENOMEM, "workspace holds %zu bytes, this call needs %zu", workspace_bytes, need);
   if ((r = check_device(c))) return r;
+  // paged: a ring page for each appended token's slot
+  std::vector<int32_t> avail = c->free_pages, idx, phys;
+  std::vector<std::vector<int32_t>> pages(B);
+  for (int b = 0; b < B; ++b) {
+    const SeqHost& s = c->seqs[seq_ids[b]];
+    pages[b] = s.pages;
+    if (!plan_pages(c, seq_ids[b], pages[b], (int64_t)s.head + s.count, 1, avail, idx, phys))
+      return fail(PS_ENOMEM, "the ring page pool has no free page left");
+  }
   cudaStream_t st = (cudaStream_t)stream;
+  if (!idx.empty())
+    PS_CUDA(ps::launch_page_set(c->dev, idx.data(), phys.data(), (int)idx.size(), st));
   const size_t per_entry = (size_t)Hq * c->d * c->esize;
   const size_t per_row = (size_t)c->Hkv * c->d * c->esize;
   for (int b0 = 0; b0 < B; b0 += ps::kMaxBatchPerLaunch) {
@@ -401,7 +528,11 @@ int ps_decode_step(ps_cache* c, const void* q, const void* k_new, const void* v_
                               (const char*)k_new + b0 * per_row, (const char*)v_new + b0 * per_row,
                               (char*)out + b0 * per_entry, scale, ws, c->sm_count, st));
   }
-  for (int b = 0; b < B; ++b) advance(c->seqs[seq_ids[b]], c->W, 1);
+  c->free_pages = avail;
+  for (int b = 0; b < B; ++b) {
+    c->seqs[seq_ids[b]].pages = pages[b];
+    advance(c->seqs[seq_ids[b]], c->W, 1);
+  }
   return ok();
 }
 
@@ -425,17 +556,29 @@ int ps_attend_chunk(ps_cache* c, int seq, const void* q, const void* k_blk, cons
       !aligned16(v_blk))
     return fail(PS_EINVAL, "q/k_blk/v_blk/out must be non-NULL 16-byte aligned device pointers");
   if ((r = check_device(c))) return r;
+  // paged: ring pages for the block's appended slots, planned before anything runs
+  std::vector<int32_t> avail = c->free_pages, idx, phys, pages = s.pages;
+  if (append_after) {
+    const int64_t n_eff = n < c->W ? n : c->W;
+    if (!plan_pages(c, seq, pages, (int64_t)s.head + s.count + (n - n_eff), n_eff, avail, idx,
+                    phys))
+      return fail(PS_ENOMEM, "the ring page pool has no free page left");
+  }
   cudaStream_t st = (cudaStream_t)stream;
-  if (ps::chunk_tc_supported(c->dtype, c->d, G))
+  if (ps::chunk_tc_supported(c->dev, c->dtype, c->d, G))
     PS_CUDA(ps::launch_chunk_tc(c->dev, G, seq, t0, n, Hq, q, k_blk, v_blk, out, scale, 0, st));
   else
     PS_CUDA(ps::launch_chunk_cc(c->dev, c->dtype, G, seq, t0, n, Hq, q, k_blk, v_blk, out, scale,
                                 0, st));
   if (append_after) {
+    if (!idx.empty())
+      PS_CUDA(ps::launch_page_set(c->dev, idx.data(), phys.data(), (int)idx.size(), st));
     ps::BatchIds ids;
     memset(&ids, 0, sizeof(ids));
     ids.seq[0] = seq;
     PS_CUDA(ps::launch_ring_append(c->dev, c->esize, ids, 1, k_blk, v_blk, n, st));
+    c->free_pages = avail;
+    c->seqs[seq].pages = pages;
     advance(c->seqs[seq], c->W, n);
   }
   return ok();
@@ -458,7 +601,7 @@ int ps_attend_prompt(ps_cache* c, int seq, const void* q, int64_t t0, int n, int
     return fail(PS_EINVAL, "q/out must be non-NULL 16-byte aligned device pointers");
   if ((r = check_device(c))) return r;
   cudaStream_t st = (cudaStream_t)stream;
-  if (ps::chunk_tc_supported(c->dtype, c->d, G))
+  if (ps::chunk_tc_supported(c->dev, c->dtype, c->d, G))
     PS_CUDA(ps::launch_chunk_tc(c->dev, G, seq, t0, n, Hq, q, nullptr, nullptr, out, scale, 1, st));
   else
     PS_CUDA(ps::launch_chunk_cc(c->dev, c->dtype, G, seq, t0, n, Hq, q, nullptr, nullptr, out,
@@ -497,11 +640,18 @@ int ps_import_window(ps_cache* c, int seq, int64_t next_pos, const void* k, cons
   if (n > 0 && (!k || !v || !aligned16(k) || !aligned16(v)))
     return fail(PS_EINVAL, "k/v must be non-NULL 16-byte aligned device pointers");
   if ((r = check_device(c))) return r;
+  std::vector<int32_t> avail = c->free_pages, idx, phys;
+  if (!plan_pages(c, seq, s.pages, ring_head_offset, n, avail, idx, phys))
+    return fail(PS_ENOMEM, "the ring page pool has no free page left");
+  if (!idx.empty())
+    PS_CUDA(ps::launch_page_set(c->dev, idx.data(), phys.data(), (int)idx.size(),
+                                (cudaStream_t)stream));
   s.next_pos = next_pos;
   s.head = ring_head_offset;
   s.count = n;
   PS_CUDA(ps::launch_ring_import(c->dev, c->esize, seq, to_dev(s), k, v, n,
                                  (cudaStream_t)stream));
+  c->free_pages = avail;
   c->seqs[seq] = s;
   return ok();
 }

@@ -185,12 +185,11 @@ __device__ __forceinline__ void merge_warps(MergeSmem<G, D>& sm) {
 
 // Stream logical rows [j_begin, j_end) of `segs` straight from global memory
 // (warp w takes row groups w, w+kNW, ...); leave the CTA state in sm slot 0.
+// Prefix rows come from the slab of sequence `owner`, ring slots from the
+// pages of sequence `seq`, block rows from kblk / vblk.
 template <typename T, int D, int G>
-__device__ __forceinline__ void stream_rows(const SegSet& segs, const T* __restrict__ kpre,
-                                            const T* __restrict__ vpre,
-                                            const T* __restrict__ kslab,
-                                            const T* __restrict__ vslab,
-                                            const T* __restrict__ kblk,
+__device__ __forceinline__ void stream_rows(const SegSet& segs, const CacheDev& c, int seq,
+                                            int owner, int g, const T* __restrict__ kblk,
                                             const T* __restrict__ vblk, int64_t blk_stride,
                                             const T* __restrict__ qrow, float qscale,
                                             int32_t j_begin, int32_t j_end,
@@ -215,10 +214,12 @@ __device__ __forceinline__ void stream_rows(const SegSet& segs, const T* __restr
         if (segs.src[si] == 2) {
           size_t r = (size_t)(segs.row0[si] + off) * blk_stride;
           kp = kblk + r; vp = vblk + r;
-        } else {  // prefix rows from the owner's slab, ring rows from the sequence's own
-          size_t r = (size_t)(segs.row0[si] + off) * D;
-          kp = (segs.src[si] == 0 ? kpre : kslab) + r;
-          vp = (segs.src[si] == 0 ? vpre : vslab) + r;
+        } else {
+          const int32_t x = (int32_t)segs.row0[si] + off;  // prefix row or ring slot
+          const size_t r = (size_t)(segs.src[si] == 0 ? prefix_row(c, owner, g, x)
+                                                      : ring_row(c, ring_page(c, seq, x), g, x)) *
+                           D;
+          kp = (const T*)c.K + r; vp = (const T*)c.V + r;
         }
         kr[u] = __ldcs((const uint4*)(kp + st.c * S::VEC));
         vr[u] = __ldcs((const uint4*)(vp + st.c * S::VEC));
@@ -248,7 +249,7 @@ __global__ void __launch_bounds__(kThreadsAttn) k_chunk_cc(AttnArgs a) {
   const int i = blockIdx.x, g = blockIdx.y;
   const DevMeta m = a.c.meta[a.seq];
   const int64_t t = a.t0 + i;
-  SegSet segs = build_segments(m, a.c.W, a.c.P_max, t);
+  SegSet segs = build_segments(m, a.c.W, t);
   if (a.prompt) {  // t < P: the visible rows are the prefix rows [0, t]
     segs.n = 1;
     segs.len[0] = (int32_t)(t + 1);
@@ -261,13 +262,9 @@ __global__ void __launch_bounds__(kThreadsAttn) k_chunk_cc(AttnArgs a) {
     if (a.prompt ? a.t0 + gridDim.x > m.P : m.next_pos != a.t0) atomicOr(a.c.err, ERR_BATCH);
     if (!segs.ring_ok) atomicOr(a.c.err, ERR_RING);
   }
-  const size_t slab = ((size_t)a.seq * a.c.Hkv + g) * (size_t)a.c.slab_rows * D;
-  const size_t pslab = ((size_t)m.owner * a.c.Hkv + g) * (size_t)a.c.slab_rows * D;
   const int64_t bstride = (int64_t)a.c.Hkv * D;
   const T* qrow = (const T*)a.q + ((size_t)i * a.Hq + (size_t)g * G) * D;
-  stream_rows<T, D, G>(segs, (const T*)a.c.K + pslab, (const T*)a.c.V + pslab,
-                       (const T*)a.c.K + slab, (const T*)a.c.V + slab,
-                       (const T*)a.kb + (size_t)g * D, (const T*)a.vb + (size_t)g * D, bstride,
+  stream_rows<T, D, G>(segs, a.c, a.seq, m.owner, g, (const T*)a.kb + (size_t)g * D, (const T*)a.vb + (size_t)g * D, bstride,
                        qrow, a.qscale, 0, segs.total, sm);
   T* orow = (T*)a.out + ((size_t)i * a.Hq + (size_t)g * G) * D;
   for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {

@@ -59,8 +59,10 @@ __host__ __device__ __forceinline__ uint32_t col_s(int st) { return st ? 128u : 
 
 struct ChunkArgs {
   CUtensorMap qmap;   // q [n][Hq][128]: box (64, 1, PT)
-  CUtensorMap kslab;  // cache K [S*Hkv][slab_rows][128]: box (64, 128, 1)
-  CUtensorMap vslab;
+  CUtensorMap kpre;   // cache K prefix rows [S*Hkv][pstride][128]: box (64, 128, 1)
+  CUtensorMap vpre;
+  CUtensorMap kring;  // cache K ring pages [nphys*Hkv][page_rows][128]: box (64, 128, 1)
+  CUtensorMap vring;
   CUtensorMap kblk;   // k_blk [n][Hkv][128]: box (64, 1, 128)
   CUtensorMap vblk;
   CacheDev c;
@@ -77,14 +79,18 @@ struct __align__(1024) TcSmem {
   uint8_t v[2][2][kBN * 128];
 };
 
-// The key tiles of one query tile: up to 4 ranges, each tiled from its start.
+// The key tiles of one query tile: up to 4 ranges, each tiled from its start;
+// a ring range of a paged cache is also cut where it crosses into a new page
+// (the first `first` rows, then 128-row tiles from that page boundary on).
 struct KSched {
   int n;
   int ntiles;
-  int src[4];       // 0: ring row of the sequence's slab, 1: block row, 2: prefix row (owner's slab)
-  int64_t row0[4];  // first slab row / block row of the range
+  int src[4];       // 0: ring slot, 1: block row, 2: prefix row (owner's slab)
+  int64_t row0[4];  // first ring slot / block row / prefix row of the range
   int64_t pos0[4];  // position of that row
   int32_t len[4];
+  int32_t first[4];   // rows before the range's first page boundary (len if none)
+  int32_t tfirst[4];  // tiles over those rows
   int32_t tbase[4];
 };
 
@@ -94,26 +100,38 @@ struct KTile {
   int valid;
 };
 
+// page: ring page size for a ring range of a paged cache (0: no page cuts)
 __device__ __forceinline__ void add_range(KSched& s, int src, int64_t row0, int64_t pos0,
-                                          int64_t len) {
+                                          int64_t len, int64_t page = 0) {
   if (len <= 0) return;
+  int64_t first = len;
+  if (page > 0) {
+    const int64_t to_edge = page - row0 % page;
+    first = to_edge < len ? to_edge : len;
+  }
   s.src[s.n] = src;
   s.row0[s.n] = row0;
   s.pos0[s.n] = pos0;
   s.len[s.n] = (int32_t)len;
+  s.first[s.n] = (int32_t)first;
+  s.tfirst[s.n] = (int32_t)((first + kBN - 1) / kBN);
   s.tbase[s.n] = s.ntiles;
-  s.ntiles += (int32_t)((len + kBN - 1) / kBN);
+  s.ntiles += s.tfirst[s.n] + (int32_t)((len - first + kBN - 1) / kBN);
   s.n++;
 }
 
 // Query positions [plo, phi]; the ring holds [next_pos - count, next_pos - 1] = [.., t0 - 1].
 // Prompt queries (phi < P) read only the prefix rows [0, phi].
-__device__ __forceinline__ KSched make_sched(const DevMeta& m, int W, int P_max, int64_t t0,
+// page: ring page size of a paged cache (0 when unpaged).
+__device__ __forceinline__ KSched make_sched(const DevMeta& m, int W, int page, int64_t t0,
                                              int64_t plo, int64_t phi, bool prompt) {
   KSched s;
   s.n = 0;
   s.ntiles = 0;
-  for (int i = 0; i < 4; ++i) { s.src[i] = 0; s.row0[i] = 0; s.pos0[i] = 0; s.len[i] = 0; s.tbase[i] = 0; }
+  for (int i = 0; i < 4; ++i) {
+    s.src[i] = 0; s.row0[i] = 0; s.pos0[i] = 0; s.len[i] = 0;
+    s.first[i] = 0; s.tfirst[i] = 0; s.tbase[i] = 0;
+  }
   if (prompt) {
     add_range(s, 2, 0, 0, phi + 1 < m.P ? phi + 1 : m.P);
     return s;
@@ -127,8 +145,8 @@ __device__ __forceinline__ KSched make_sched(const DevMeta& m, int W, int P_max,
     const int64_t nw = t0 - rlo;
     const int64_t s0 = ((int64_t)m.head + (rlo - base)) % W;
     const int64_t lenA = nw < W - s0 ? nw : W - s0;
-    add_range(s, 0, P_max + s0, rlo, lenA);
-    add_range(s, 0, P_max, rlo + lenA, nw - lenA);
+    add_range(s, 0, s0, rlo, lenA, page);
+    add_range(s, 0, 0, rlo + lenA, nw - lenA, page);
   }
   const int64_t blo = lo > t0 ? lo : t0;
   add_range(s, 1, blo - t0, blo, phi - blo + 1);
@@ -142,17 +160,23 @@ __device__ __forceinline__ KTile tile_of(const KSched& s, int j) {
 #pragma unroll
   for (int q = 1; q < 4; ++q)
     if (q < s.n && j >= s.tbase[q]) k = q;
-  int64_t off = 0, len = 0;
+  int64_t off = 0, end = 0;
 #pragma unroll
   for (int q = 0; q < 4; ++q)
     if (q == k) {
       t.src = s.src[q];
-      off = (int64_t)(j - s.tbase[q]) * kBN;
+      const int u = j - s.tbase[q];
+      if (u < s.tfirst[q]) {  // before the range's first page boundary
+        off = (int64_t)u * kBN;
+        end = s.first[q];
+      } else {
+        off = s.first[q] + (int64_t)(u - s.tfirst[q]) * kBN;
+        end = s.len[q];
+      }
       t.row = s.row0[q] + off;
       t.pos0 = s.pos0[q] + off;
-      len = s.len[q];
     }
-  t.valid = (int)(len - off < kBN ? len - off : kBN);
+  t.valid = (int)(end - off < kBN ? end - off : kBN);
   return t;
 }
 
@@ -189,7 +213,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
   const DevMeta m = a.c.meta[a.seq];
   const int64_t plo = a.t0 + i0;
   const int64_t phi = a.t0 + min(i0 + PT, a.n) - 1;
-  const KSched ks = make_sched(m, a.c.W, a.c.P_max, a.t0, plo, phi, a.prompt != 0);
+  const KSched ks = make_sched(m, a.c.W, a.c.page_table ? a.c.page_rows : 0, a.t0, plo, phi,
+                               a.prompt != 0);
   const int T = ks.ntiles;
 
   if (threadIdx.x == 0) {
@@ -221,7 +246,6 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
   if (warp == 0) {
     // ------------------------------------------------------------ producer --
     if (lane == 0) {
-      const int slab_z = a.seq * a.c.Hkv + g;
       const int prefix_z = m.owner * a.c.Hkv + g;  // prefix rows live in the owner's slab
       int issued_k = 0, issued_v = 0;
       ptx::mbar_arrive_expect_tx(&q_full, 2 * kBM * 128);
@@ -232,11 +256,16 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
         const int st = j & 1;
         const KTile kt = tile_of(ks, j);
         if (j >= 2 && !wait_bar(&k_empty[st], ((j >> 1) - 1) & 1, &abort_flag)) break;
+        // a ring tile lies within one page: (slot within the page, page's slab)
+        const int32_t kslot = (int32_t)kt.row;  // ring slot (ring tiles)
+        const int ring_z = kt.src == 0 ? ring_page(a.c, a.seq, kslot) * a.c.Hkv + g : 0;
+        const int32_t ring_y = kt.src == 0 ? kslot % a.c.page_rows : 0;
         ptx::mbar_arrive_expect_tx(&k_full[st], kTileBytes);
         for (int b = 0; b < 2; ++b) {
-          if (kt.src != 1)
-            ptx::tma_load_3d(sm.k[st][b], &a.kslab, b * 64, (int32_t)kt.row,
-                             kt.src == 2 ? prefix_z : slab_z, &k_full[st]);
+          if (kt.src == 2)
+            ptx::tma_load_3d(sm.k[st][b], &a.kpre, b * 64, (int32_t)kt.row, prefix_z, &k_full[st]);
+          else if (kt.src == 0)
+            ptx::tma_load_3d(sm.k[st][b], &a.kring, b * 64, ring_y, ring_z, &k_full[st]);
           else
             ptx::tma_load_3d(sm.k[st][b], &a.kblk, b * 64, g, (int32_t)kt.row, &k_full[st]);
         }
@@ -244,9 +273,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
         if (j >= 2 && !wait_bar(&v_empty[st], ((j >> 1) - 1) & 1, &abort_flag)) break;
         ptx::mbar_arrive_expect_tx(&v_full[st], kTileBytes);
         for (int b = 0; b < 2; ++b) {
-          if (kt.src != 1)
-            ptx::tma_load_3d(sm.v[st][b], &a.vslab, b * 64, (int32_t)kt.row,
-                             kt.src == 2 ? prefix_z : slab_z, &v_full[st]);
+          if (kt.src == 2)
+            ptx::tma_load_3d(sm.v[st][b], &a.vpre, b * 64, (int32_t)kt.row, prefix_z, &v_full[st]);
+          else if (kt.src == 0)
+            ptx::tma_load_3d(sm.v[st][b], &a.vring, b * 64, ring_y, ring_z, &v_full[st]);
           else
             ptx::tma_load_3d(sm.v[st][b], &a.vblk, b * 64, g, (int32_t)kt.row, &v_full[st]);
         }
@@ -486,8 +516,10 @@ bool map3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t 
 
 }  // namespace
 
-bool chunk_tc_supported(int dtype, int d, int G) {
-  return dtype == 1 && d == kHD && (G == 1 || G == 2 || G == 4 || G == 8);
+bool chunk_tc_supported(const CacheDev& c, int dtype, int d, int G) {
+  // ring tiles of a paged cache must not straddle pages: 128-row multiples
+  const bool pages_ok = !c.page_table || c.page_rows % kBN == 0;
+  return pages_ok && dtype == 1 && d == kHD && (G == 1 || G == 2 || G == 4 || G == 8);
 }
 
 cudaError_t launch_chunk_tc(const CacheDev& c, int G, int seq, int64_t t0, int n, int Hq,
@@ -498,10 +530,17 @@ cudaError_t launch_chunk_tc(const CacheDev& c, int G, int seq, int64_t t0, int n
   const uint64_t row = kHD * 2;  // bytes per head row
   const int PT = kBM / G;
   bool ok = map3d(&a.qmap, q, kHD, Hq, n, row, (uint64_t)Hq * row, 64, 1, PT);
-  ok = ok && map3d(&a.kslab, c.K, kHD, c.slab_rows, (uint64_t)c.S * c.Hkv, row,
-                   (uint64_t)c.slab_rows * row, 64, kBN, 1);
-  ok = ok && map3d(&a.vslab, c.V, kHD, c.slab_rows, (uint64_t)c.S * c.Hkv, row,
-                   (uint64_t)c.slab_rows * row, 64, kBN, 1);
+  // prefix rows: [S*Hkv][pstride] rows from the buffer start; ring pages:
+  // [nphys*Hkv][page_rows] slabs rstride rows apart from row rbase
+  const uint64_t prows = c.pstride > 0 ? (uint64_t)c.pstride : 1;
+  const char* kring = (const char*)c.K + (size_t)c.rbase * row;
+  const char* vring = (const char*)c.V + (size_t)c.rbase * row;
+  ok = ok && map3d(&a.kpre, c.K, kHD, prows, (uint64_t)c.S * c.Hkv, row, prows * row, 64, kBN, 1);
+  ok = ok && map3d(&a.vpre, c.V, kHD, prows, (uint64_t)c.S * c.Hkv, row, prows * row, 64, kBN, 1);
+  ok = ok && map3d(&a.kring, kring, kHD, (uint64_t)c.page_rows, (uint64_t)c.nphys * c.Hkv, row,
+                   (uint64_t)c.rstride * row, 64, kBN, 1);
+  ok = ok && map3d(&a.vring, vring, kHD, (uint64_t)c.page_rows, (uint64_t)c.nphys * c.Hkv, row,
+                   (uint64_t)c.rstride * row, 64, kBN, 1);
   // a prompt launch loads no block rows; its block maps describe the cache
   // K/V (never used) so that every map is well formed
   ok = ok && map3d(&a.kblk, prompt ? c.K : k_blk, kHD, c.Hkv, n, row, (uint64_t)c.Hkv * row, 64,

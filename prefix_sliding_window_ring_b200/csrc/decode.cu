@@ -445,12 +445,9 @@ __global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8)
       m.head = a.head[pt.b];
       m.count = a.count[pt.b];
       m.owner = a.owner[pt.b];
-      const SegSet segs = build_segments(m, a.c.W, a.c.P_max, a.t[pt.b]);
+      const SegSet segs = build_segments(m, a.c.W, a.t[pt.b]);
       bool bad = segs.total != m.P + m.count || (segs.total + TR - 1) / TR != pt.tph;
       const bool step = a.knew != nullptr;  // the pair's last row comes from knew/vnew
-      const size_t slab = ((size_t)s * Hkv + pt.g) * (size_t)a.c.slab_rows * D;
-      // prefix rows come from the slab of the sequence that owns them
-      const size_t pslab = ((size_t)a.owner[pt.b] * Hkv + pt.g) * (size_t)a.c.slab_rows * D;
       const int pair = pt.b * Hkv + pt.g;
       for (int32_t j = j0; j < j1 && alive; ++j) {
         const int32_t r0 = j * TR, r1 = min(segs.total, r0 + TR);
@@ -478,12 +475,26 @@ __global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8)
                         &full[st]);
         T* kd = ktile + (size_t)st * TR * D;
         T* vd = vtile + (size_t)st * TR * D;
+        auto copy = [&](int64_t crow, int32_t cdst, int32_t cn) {
+          const uint32_t nb = (uint32_t)cn * D * sizeof(T);
+          ptx::bulk_g2s(kd + (size_t)cdst * D, (const T*)a.c.K + (size_t)crow * D, nb, &full[st]);
+          ptx::bulk_g2s(vd + (size_t)cdst * D, (const T*)a.c.V + (size_t)crow * D, nb, &full[st]);
+        };
         for_each_run(segs, r0, with_new ? r1 - 1 : r1, &bad,
                      [&](int src, int64_t row, int32_t dst, int32_t nr) {
-          const uint32_t nb = (uint32_t)nr * D * sizeof(T);
-          const size_t base = (src == 0 ? pslab : slab) + (size_t)row * D;
-          ptx::bulk_g2s(kd + (size_t)dst * D, (const T*)a.c.K + base, nb, &full[st]);
-          ptx::bulk_g2s(vd + (size_t)dst * D, (const T*)a.c.V + base, nb, &full[st]);
+          if (src == 0) {  // prefix rows, from the slab of the sequence that owns them
+            copy(prefix_row(a.c, a.owner[pt.b], pt.g, row), dst, nr);
+            return;
+          }
+          // ring slots [row, row + nr): one copy per page they touch (a run
+          // never wraps, so an unpaged ring takes one copy)
+          const int32_t sa = (int32_t)row, se = sa + nr;
+          for (int32_t s0 = sa; s0 < se;) {
+            const int32_t pe = a.c.page_table ? (s0 / a.c.page_rows + 1) * a.c.page_rows : se;
+            const int32_t cn = min(se, pe) - s0;
+            copy(ring_row(a.c, ring_page(a.c, s, s0), pt.g, s0), dst + (s0 - sa), cn);
+            s0 += cn;
+          }
         });
         if (with_new) {  // the appended token, straight from the caller's rows
           const size_t src = (size_t)pair * D;
@@ -554,8 +565,9 @@ __global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8)
       // decode step: this warp holds the appended token; store it in its ring
       // slot (the evicted row's, never visible to this step's queries)
       const int b = d.pair / Hkv, g = d.pair % Hkv, s = a.seq[b];
-      const int64_t slot = ((int64_t)a.head[b] + a.count[b] - 1) % a.c.W;
-      const size_t row = (((size_t)s * Hkv + g) * (size_t)a.c.slab_rows + a.c.P_max + slot) * D;
+      const int32_t slot = (int32_t)(((int64_t)a.head[b] + a.count[b] - 1) % a.c.W);
+      const int phys = ring_page(a.c, s, slot);
+      const size_t row = (size_t)ring_row(a.c, phys, g, slot) * D;
       const size_t so = ((size_t)stg * TR + d.nrows - 1) * D;
       constexpr int V16 = D * (int)sizeof(T) / 16;  // 16-byte pieces per row
       for (int x = lane; x < 2 * V16; x += 32) {
@@ -564,7 +576,7 @@ __global__ void __maxnreg__(65536 / (kThreadsDec * PS_DEC_CTAS_PER_SM) / 8 * 8)
         const uint4 val = ((const uint4*)((isv ? vtile : ktile) + so))[xi];
         ((uint4*)((T*)(isv ? a.c.V : a.c.K) + row))[xi] = val;
       }
-      if (lane == 0 && g == 0) a.c.pos[(size_t)s * a.c.W + slot] = a.t[b];
+      if (lane == 0 && g == 0) a.c.pos[pos_index(a.c, phys, slot)] = a.t[b];
     }
     __syncwarp();
     if (lane == 0) ptx::mbar_arrive(&empty[stg]);

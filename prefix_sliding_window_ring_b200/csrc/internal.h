@@ -19,6 +19,10 @@ struct BatchIds {
 };
 
 // ring.cu
+constexpr int kMaxPageSets = 256;  // page-table entries per update launch
+// page_table[idx[i]] = phys[i] for i < n (paged caches), in launches of kMaxPageSets.
+cudaError_t launch_page_set(const CacheDev& c, const int32_t* idx, const int32_t* phys, int n,
+                            cudaStream_t st);
 cudaError_t launch_meta_set(const CacheDev& c, int seq, const DevMeta& m, cudaStream_t st);
 cudaError_t launch_prefix_store(const CacheDev& c, int esize, int seq, const void* k,
                                 const void* v, int P_s, cudaStream_t st);
@@ -52,7 +56,7 @@ cudaError_t launch_decode(const CacheDev& c, int dtype, int G, const BatchIds& i
                           float scale, const DecodeWs& ws, int sm_count, cudaStream_t st);
 
 // chunk_tc.cu (tcgen05 chunk kernel: bf16, head_dim 128)
-bool chunk_tc_supported(int dtype, int d, int G);
+bool chunk_tc_supported(const CacheDev& c, int dtype, int d, int G);
 // prompt != 0: queries t0..t0+n-1 inside the prefix attend causally to the
 // prefix rows [0, t] (k_blk / v_blk unused); otherwise a chunk at t0 == next_pos.
 cudaError_t launch_chunk_tc(const CacheDev& c, int G, int seq, int64_t t0, int n, int Hq,

@@ -19,9 +19,14 @@ constexpr int kThreads = 256;
 
 __global__ void k_meta_set(DevMeta* meta, int seq, DevMeta m) { meta[seq] = m; }
 
-__device__ __forceinline__ size_t slab_row_off(const CacheDev& c, int s, int g, int64_t row,
-                                               int vpr) {
-  return (((size_t)s * c.Hkv + g) * (size_t)c.slab_rows + (size_t)row) * vpr;
+// Page-table updates of a paged cache: page_table[idx[i]] = phys[i].
+struct PageSets {
+  int32_t n;
+  int32_t idx[kMaxPageSets];
+  int32_t phys[kMaxPageSets];
+};
+__global__ void k_page_set(int32_t* page_table, PageSets u) {
+  for (int i = threadIdx.x; i < u.n; i += blockDim.x) page_table[u.idx[i]] = u.phys[i];
 }
 
 // Prefix rows: input [P_s][Hkv][d] -> slab rows [0, P_s) of every head.
@@ -36,7 +41,7 @@ __global__ void k_prefix_store(CacheDev c, int vpr, int seq, const uint4* __rest
     int64_t r = x / vpr;
     int g = (int)(r % c.Hkv);
     int64_t j = r / c.Hkv;
-    size_t dst = slab_row_off(c, seq, g, j, vpr) + vi;
+    size_t dst = (size_t)prefix_row(c, seq, g, j) * vpr + vi;
     K[dst] = k[x];
     V[dst] = v[x];
   }
@@ -64,12 +69,13 @@ __global__ void k_ring_append(CacheDev c, int vpr, BatchIds ids, const uint4* __
     int g = (int)(r % c.Hkv);
     int64_t i = i0 + r / c.Hkv;
     int64_t p = m.next_pos + i;
-    int64_t slot = ((int64_t)m.head + (p - base)) % W;
+    const int32_t slot = (int32_t)(((int64_t)m.head + (p - base)) % W);
+    const int phys = ring_page(c, s, slot);
     size_t src = (((size_t)b * n + i) * c.Hkv + g) * vpr + vi;
-    size_t dst = slab_row_off(c, s, g, c.P_max + slot, vpr) + vi;
+    size_t dst = (size_t)ring_row(c, phys, g, slot) * vpr + vi;
     K[dst] = k[src];
     V[dst] = v[src];
-    if (g == 0 && vi == 0) c.pos[(size_t)s * W + slot] = p;
+    if (g == 0 && vi == 0) c.pos[pos_index(c, phys, slot)] = p;
   }
   __threadfence();
   __syncthreads();
@@ -101,11 +107,12 @@ __global__ void k_ring_import(CacheDev c, int vpr, int seq, DevMeta mn,
     int64_t r = x / vpr;
     int g = (int)(r % c.Hkv);
     int64_t i = r / c.Hkv;
-    int64_t slot = ((int64_t)mn.head + i) % W;
-    size_t dst = slab_row_off(c, seq, g, c.P_max + slot, vpr) + vi;
+    const int32_t slot = (int32_t)(((int64_t)mn.head + i) % W);
+    const int phys = ring_page(c, seq, slot);
+    size_t dst = (size_t)ring_row(c, phys, g, slot) * vpr + vi;
     K[dst] = k[x];
     V[dst] = v[x];
-    if (g == 0 && vi == 0) c.pos[(size_t)seq * W + slot] = mn.next_pos - n + i;
+    if (g == 0 && vi == 0) c.pos[pos_index(c, phys, slot)] = mn.next_pos - n + i;
   }
   __threadfence();
   __syncthreads();
@@ -132,11 +139,12 @@ __global__ void k_ring_export(CacheDev c, int vpr, int seq, uint4* __restrict__ 
     int64_t r = x / vpr;
     int g = (int)(r % c.Hkv);
     int64_t i = r / c.Hkv;
-    int64_t slot = ((int64_t)m.head + i) % c.W;
-    size_t src = slab_row_off(c, seq, g, c.P_max + slot, vpr) + vi;
+    const int32_t slot = (int32_t)(((int64_t)m.head + i) % c.W);
+    const int phys = ring_page(c, seq, slot);
+    size_t src = (size_t)ring_row(c, phys, g, slot) * vpr + vi;
     k[x] = K[src];
     v[x] = V[src];
-    if (g == 0 && vi == 0) pos[i] = c.pos[(size_t)seq * c.W + slot];
+    if (g == 0 && vi == 0) pos[i] = c.pos[pos_index(c, phys, slot)];
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) *count_out = m.count;
 }
@@ -145,7 +153,7 @@ __global__ void k_ring_export(CacheDev c, int vpr, int seq, uint4* __restrict__ 
 __global__ void k_debug_visible(CacheDev c, int seq, int64_t t, int64_t* __restrict__ pos_out,
                                 int32_t* __restrict__ n_out) {
   const DevMeta m = c.meta[seq];
-  const SegSet s = build_segments(m, c.W, c.P_max, t);
+  const SegSet s = build_segments(m, c.W, t);
   if (!s.ring_ok && threadIdx.x == 0) atomicOr(c.err, ERR_RING);
   int32_t j0 = 0;
   for (int i = 0; i < s.n; ++i) {
@@ -154,8 +162,8 @@ __global__ void k_debug_visible(CacheDev c, int seq, int64_t t, int64_t* __restr
       if (s.src[i] == 0) {
         p = s.row0[i] + r;  // prefix row j holds position j
       } else if (s.src[i] == 1) {
-        int64_t slot = s.row0[i] - c.P_max + r;
-        p = c.pos[(size_t)seq * c.W + slot];
+        const int32_t slot = (int32_t)(s.row0[i] + r);
+        p = c.pos[pos_index(c, ring_page(c, seq, slot), slot)];
       } else {
         p = m.next_pos + s.row0[i] + r;
       }
@@ -188,6 +196,22 @@ int grid_for(int64_t work, int cap) {
 }
 
 }  // namespace
+
+cudaError_t launch_page_set(const CacheDev& c, const int32_t* idx, const int32_t* phys, int n,
+                            cudaStream_t st) {
+  for (int i0 = 0; i0 < n; i0 += kMaxPageSets) {
+    PageSets u;
+    u.n = n - i0 < kMaxPageSets ? n - i0 : kMaxPageSets;
+    for (int i = 0; i < u.n; ++i) {
+      u.idx[i] = idx[i0 + i];
+      u.phys[i] = phys[i0 + i];
+    }
+    k_page_set<<<1, 256, 0, st>>>(c.page_table, u);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
 
 cudaError_t launch_meta_set(const CacheDev& c, int seq, const DevMeta& m, cudaStream_t st) {
   k_meta_set<<<1, 1, 0, st>>>(c.meta, seq, m);

@@ -62,3 +62,23 @@ def test_create_rejects_bad_arguments_before_touching_cuda():
     assert e.value.code == abi.PS_ENOMEM
     assert "needs" in abi.ps_last_error()
     assert abi.ps_decode_workspace_bytes(None, 1, 1) == 0
+
+
+def test_paged_cache_bytes_and_argument_checks():
+    from prefix_sliding_window_ring_b200 import abi
+    unpaged = abi.ps_cache_bytes(512, 64, 2, 128, abi.PS_BF16, 4)
+    # one page per sequence holds the same rows as the unpaged layout plus a small page table
+    same = abi.ps_cache_bytes_paged(512, 64, 2, 128, abi.PS_BF16, 4, 512, 4)
+    assert unpaged <= same <= unpaged + 4096
+    half = abi.ps_cache_bytes_paged(512, 64, 2, 128, abi.PS_BF16, 4, 128, 8)   # 8 of 16 pages
+    assert half < same
+    assert abi.ps_cache_bytes_paged(512, 64, 2, 128, abi.PS_BF16, 4, 100, 8) == 0  # 512 % 100
+    assert abi.ps_cache_bytes_paged(512, 64, 2, 128, abi.PS_BF16, 4, 1024, 8) == 0  # page > W
+    assert abi.ps_cache_bytes_paged(512, 64, 2, 128, abi.PS_BF16, 4, 128, 0) == 0  # no pages
+    assert abi.ps_cache_bytes_paged(512, 64, 2, 128, abi.PS_BF16, 4, 0, 8) == 0
+    with pytest.raises(abi.PSError) as e:
+        abi.ps_cache_create_paged(512, 64, 2, 128, abi.PS_BF16, 4, 0, 8, 256, 1 << 20)
+    assert e.value.code == abi.PS_EINVAL
+    with pytest.raises(abi.PSError) as e:
+        abi.ps_ring_pages_free(None)
+    assert e.value.code == abi.PS_EINVAL
