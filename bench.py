@@ -467,7 +467,8 @@ def load_bf16_peak():
 def prefill_measure(steps: int):
     """Chunked prefill/extend on the tensor-core kernel: 4 sequences, each a
     2048-query block at t0=100000 (window full), P=256, W in {4096, 16384}.
-    One step = the 4 calls.  Throughput counts only visible (query, key) pairs:
+    One step = one ps_attend_chunk_batch call over the 4 blocks (packed).
+    Throughput counts only visible (query, key) pairs:
     4 * d * Hq * sum over queries of (P + W) flops."""
     import torch
 
@@ -482,9 +483,10 @@ def prefill_measure(steps: int):
                        f"Hq={HQ} Hkv={HKV} d={D} P={PF_P}, bf16",
            "kernel": "ps::k_chunk_tc (tcgen05)", "peak": peak, "peak_source": peak_src,
            "unit": "TFLOP/s"}
+    ids = list(range(PF_SEQS))
     for Wp in (4096, 16384):
         c = Cache(Wp, PF_P, HKV, D, PS_BF16, PF_SEQS)
-        blocks = []
+        qs, kbs, vbs = [], [], []
         for s in range(PF_SEQS):
             c.seq_reset(s, 0)
             c.prefill_prefix(s, dev(synth.rows(SEED, synth.TID_K, s, HKV, 0, PF_P, D, "bf16")),
@@ -493,24 +495,19 @@ def prefill_measure(steps: int):
                             dev(synth.rows(SEED, synth.TID_K, s, HKV, PF_T0 - Wp, Wp, D, "bf16")),
                             dev(synth.rows(SEED, synth.TID_V, s, HKV, PF_T0 - Wp, Wp, D, "bf16")),
                             Wp, (977 * s) % Wp)
-            q = dev(synth.rows(SEED, synth.TID_Q, s, HQ, PF_T0, PF_N, D, "bf16"))
-            kb = dev(synth.rows(SEED, synth.TID_K, s, HKV, PF_T0, PF_N, D, "bf16"))
-            vb = dev(synth.rows(SEED, synth.TID_V, s, HKV, PF_T0, PF_N, D, "bf16"))
-            blocks.append((q, kb, vb, torch.empty_like(q)))
+            qs.append(dev(synth.rows(SEED, synth.TID_Q, s, HQ, PF_T0, PF_N, D, "bf16")))
+            kbs.append(dev(synth.rows(SEED, synth.TID_K, s, HKV, PF_T0, PF_N, D, "bf16")))
+            vbs.append(dev(synth.rows(SEED, synth.TID_V, s, HKV, PF_T0, PF_N, D, "bf16")))
+        # the blocks packed end to end, as the batched call takes them
+        q, kb, vb = torch.cat(qs), torch.cat(kbs), torch.cat(vbs)
+        o = torch.empty_like(q)
+        del qs, kbs, vbs
         scale = 1.0 / math.sqrt(D)
 
-        side = [torch.cuda.Stream() for _ in blocks]
-
         def step(i, st=None):
-            # The sequences are independent: one stream each, joined at the end,
-            # so their CTAs fill the GPU together (one sequence is 1.7 waves).
-            st = st or torch.cuda.current_stream()
-            for ss in side:
-                ss.wait_stream(st)
-            for s, (q, kb, vb, o) in enumerate(blocks):
-                c.attend_chunk(s, q, kb, vb, PF_T0, PF_N, HQ, scale, o, 0, side[s])
-            for ss in side:
-                st.wait_stream(ss)
+            # one persistent launch over the four sequences' query tiles
+            c.attend_chunk_batch(ids, [PF_T0] * PF_SEQS, [PF_N] * PF_SEQS, q, kb, vb, HQ, scale,
+                                 o, 0, st)
 
         for i in range(3):
             step(i)
@@ -523,7 +520,7 @@ def prefill_measure(steps: int):
         res[f"W{Wp}"] = {"ms_per_step": round(ms, 4), "gflop_per_step": round(flops / 1e9, 1),
                          "achieved": round(tf, 1), "frac": round(tf / peak, 4)}
         c.close()
-        del blocks
+        del q, kb, vb, o
         torch.cuda.empty_cache()
     res["prompt"] = prompt_measure(steps, peak)
     return res
@@ -535,7 +532,7 @@ PR_P = 4096  # prompt length of the prompt-prefill measurement
 def prompt_measure(steps: int, peak: float):
     """Prompt prefill (queries inside the pinned prefix, causal over it) on the
     tensor-core kernel: 4 sequences with a 4096-token prompt each, one
-    ps_attend_prompt call per sequence.  Visible pairs only:
+    ps_attend_prompt_batch call over the 4 prompts (packed).  Visible pairs only:
     4 * d * Hq * sum over t < P of (t + 1) flops per sequence."""
     import torch
 
@@ -550,19 +547,15 @@ def prompt_measure(steps: int, peak: float):
     for s in range(PF_SEQS):
         c.prefill_prefix(s, dev(synth.rows(SEED, synth.TID_K, s, HKV, 0, PR_P, D, "bf16")),
                          dev(synth.rows(SEED, synth.TID_V, s, HKV, 0, PR_P, D, "bf16")), PR_P)
-        q = dev(synth.rows(SEED, synth.TID_Q, s, HQ, 0, PR_P, D, "bf16"))
-        qs.append((q, torch.empty_like(q)))
+        qs.append(dev(synth.rows(SEED, synth.TID_Q, s, HQ, 0, PR_P, D, "bf16")))
+    q = torch.cat(qs)  # the prompts packed end to end
+    o = torch.empty_like(q)
+    del qs
     scale = 1.0 / math.sqrt(D)
-    side = [torch.cuda.Stream() for _ in qs]
+    ids = list(range(PF_SEQS))
 
     def step(i, st=None):
-        st = st or torch.cuda.current_stream()
-        for ss in side:
-            ss.wait_stream(st)
-        for s, (q, o) in enumerate(qs):
-            c.attend_prompt(s, q, 0, PR_P, HQ, scale, o, side[s])
-        for ss in side:
-            st.wait_stream(ss)
+        c.attend_prompt_batch(ids, [0] * PF_SEQS, [PR_P] * PF_SEQS, q, HQ, scale, o, st)
 
     for i in range(3):
         step(i)
@@ -573,7 +566,7 @@ def prompt_measure(steps: int, peak: float):
     flops = 4.0 * D * HQ * (PR_P * (PR_P + 1) / 2) * PF_SEQS
     tf = flops / (ms / 1e3) / 1e12
     c.close()
-    del qs
+    del q, o
     torch.cuda.empty_cache()
     return {"workload": f"{PF_SEQS} sequences x {PR_P}-token prompt (causal over the pinned prefix), "
                         f"Hq={HQ} Hkv={HKV} d={D}, bf16",

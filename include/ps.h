@@ -153,6 +153,18 @@ PS_API int ps_share_prefix(ps_cache* c, int seq, int src, void* stream);
 PS_API int ps_attend_prompt(ps_cache* c, int seq, const void* q, int64_t t0, int n, int Hq,
                             float scale, void* out, void* stream);
 
+/* Prompt attention of B sequences in one launch: entry b is as the call above
+ * for sequence seq_ids[b] (host array of distinct active ids) with queries
+ * t0[b]..t0[b]+n[b]-1 (host arrays; n[b] >= 0, 0 <= t0[b], t0[b]+n[b] <= P_s).
+ * The entries' rows are packed end to end in entry order: q, out
+ * [sum n][Hq][d] (device), entry b from row n[0]+...+n[b-1].  On the
+ * tensor-core kernel the whole batch is one persistent launch, so one
+ * sequence's tail of work does not leave the GPU partly idle.
+ * Errors: as ps_attend_prompt, checked for every entry before anything runs. */
+PS_API int ps_attend_prompt_batch(ps_cache* c, const int* seq_ids, const int64_t* t0,
+                                  const int* n, int B, const void* q, int Hq, float scale,
+                                  void* out, void* stream);
+
 /* ---------------------------------------------------- a2 ring append ----- */
 
 /* Append n tokens to each of B active sequences seq_ids[0..B) (host array of
@@ -242,6 +254,21 @@ PS_API int ps_attend_decode_static(ps_cache* c, const void* q, const int* seq_id
 PS_API int ps_attend_chunk(ps_cache* c, int seq, const void* q, const void* k_blk,
                     const void* v_blk, int64_t t0, int n, int Hq, float scale, void* out,
                     int append_after, void* stream);
+
+/* Chunked prefill/extend of B sequences in one launch (batched serving):
+ * entry b is as ps_attend_chunk for sequence seq_ids[b] (host array of
+ * distinct active ids) with a block of n[b] >= 0 queries at t0[b] == its
+ * next_pos (host arrays).  The entries' rows are packed end to end in entry
+ * order: q, out [sum n][Hq][d]; k_blk, v_blk [sum n][Hkv][d] (device), entry
+ * b from row n[0]+...+n[b-1].  With append_after != 0 every entry's block is
+ * then appended to its ring.  On the tensor-core kernel the whole batch is one
+ * persistent launch (one CTA per SM working through all entries' query tiles).
+ * Errors: as ps_attend_chunk, checked for every entry (and, for a paged cache,
+ * the pages of all appends planned) before anything runs; PS_ENOMEM if the
+ * page pool cannot take all the appends. */
+PS_API int ps_attend_chunk_batch(ps_cache* c, const int* seq_ids, const int64_t* t0, const int* n,
+                                 int B, const void* q, const void* k_blk, const void* v_blk,
+                                 int Hq, float scale, void* out, int append_after, void* stream);
 
 /* ------------------------------------------- checkpoint / debug export --- */
 

@@ -47,6 +47,8 @@ SIGNATURES = {
     "ps_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _f, _vp, _vp, _sz, _vp]),
     "ps_attend_chunk": (_i, [_vp, _i, _vp, _vp, _vp, _i64, _i, _i, _f, _vp, _i, _vp]),
     "ps_attend_prompt": (_i, [_vp, _i, _vp, _i64, _i, _i, _f, _vp, _vp]),
+    "ps_attend_chunk_batch": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _i, _f, _vp, _i, _vp]),
+    "ps_attend_prompt_batch": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _i, _f, _vp, _vp]),
     "ps_share_prefix": (_i, [_vp, _i, _i, _vp]),
     "ps_debug_wait_timeout": (_i, [_vp, ctypes.c_longlong, _vp]),
     "ps_export_window": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp]),
@@ -212,6 +214,31 @@ def ps_attend_chunk(cache, seq, q, k_blk, v_blk, t0, n, Hq, scale, out, append_a
     _check("ps_attend_chunk", _lib.ps_attend_chunk(cache, seq, _ptr(q), _ptr(k_blk), _ptr(v_blk),
                                                    t0, n, Hq, scale, _ptr(out), int(append_after),
                                                    _stream(stream)))
+
+
+def _entries(seq_ids, t0, n):
+    ids, B = _ints(seq_ids, ctypes.c_int)
+    ts, Bt = _ints(t0, ctypes.c_int64)
+    ns, Bn = _ints(n, ctypes.c_int)
+    if not B == Bt == Bn:
+        raise ValueError("seq_ids, t0 and n differ in length")
+    return ids, ts, ns, B
+
+
+def ps_attend_chunk_batch(cache, seq_ids, t0, n, q, k_blk, v_blk, Hq, scale, out, append_after=0,
+                          stream=None) -> None:
+    """Chunks of several sequences in one launch; rows packed end to end in entry order."""
+    ids, ts, ns, B = _entries(seq_ids, t0, n)
+    _check("ps_attend_chunk_batch", _lib.ps_attend_chunk_batch(
+        cache, ids, ts, ns, B, _ptr(q), _ptr(k_blk), _ptr(v_blk), Hq, scale, _ptr(out),
+        int(append_after), _stream(stream)))
+
+
+def ps_attend_prompt_batch(cache, seq_ids, t0, n, q, Hq, scale, out, stream=None) -> None:
+    """Prompt attention of several sequences in one launch; rows packed in entry order."""
+    ids, ts, ns, B = _entries(seq_ids, t0, n)
+    _check("ps_attend_prompt_batch", _lib.ps_attend_prompt_batch(
+        cache, ids, ts, ns, B, _ptr(q), Hq, scale, _ptr(out), _stream(stream)))
 
 
 def ps_share_prefix(cache, seq, src, stream=None) -> None:

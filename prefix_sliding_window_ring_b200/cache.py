@@ -84,6 +84,14 @@ class Cache:
         abi.ps_attend_chunk(self.handle, seq, q, k_blk, v_blk, t0, n, Hq, scale, out, append_after,
                             stream)
 
+    def attend_chunk_batch(self, seq_ids, t0, n, q, k_blk, v_blk, Hq, scale, out, append_after=0,
+                           stream=None):
+        abi.ps_attend_chunk_batch(self.handle, seq_ids, t0, n, q, k_blk, v_blk, Hq, scale, out,
+                                  append_after, stream)
+
+    def attend_prompt_batch(self, seq_ids, t0, n, q, Hq, scale, out, stream=None):
+        abi.ps_attend_prompt_batch(self.handle, seq_ids, t0, n, q, Hq, scale, out, stream)
+
     def share_prefix(self, seq, src, stream=None):
         abi.ps_share_prefix(self.handle, seq, src, stream)
 

@@ -189,6 +189,123 @@ ps::DevMeta to_dev(const SeqHost& s) {
 
 }  // namespace
 
+// Chunk (prompt == false) or prompt attention of B sequences' blocks, rows
+// packed end to end in entry order; then, for chunks with append_after, the
+// blocks are appended to the rings.  Everything is validated (and paged ring
+// pages planned) before anything is enqueued.
+static int attend_blocks(ps_cache* c, const int* seq_ids, const int64_t* t0, const int* n, int B,
+                  const void* q, const void* k_blk, const void* v_blk, int Hq, float scale,
+                  void* out, int append_after, bool prompt, void* stream) {
+  if (!c) return fail(PS_EINVAL, "cache is NULL");
+  if (B < 0) return fail(PS_EINVAL, "negative B=%d", B);
+  if (B == 0) return ok();
+  if (!t0 || !n) return fail(PS_EINVAL, "t0 / n is NULL");
+  int r = check_batch(c, seq_ids, B);
+  if (r) return r;
+  int G = 0;
+  if ((r = check_group(c, Hq, &G))) return r;
+  int64_t N = 0;
+  for (int b = 0; b < B; ++b) {
+    const SeqHost& s = c->seqs[seq_ids[b]];
+    if (n[b] < 0) return fail(PS_EINVAL, "entry %d: negative n=%d", b, n[b]);
+    if (prompt) {
+      if (t0[b] < 0 || t0[b] + n[b] > s.P)
+        return fail(PS_EPOS, "sequence %d: prompt queries [%lld, %lld) are not inside the prefix (P=%d)",
+                    seq_ids[b], (long long)t0[b], (long long)(t0[b] + n[b]), s.P);
+    } else {
+      if (t0[b] != s.next_pos)
+        return fail(PS_EPOS, "sequence %d: t0=%lld does not follow the history (next position %lld)",
+                    seq_ids[b], (long long)t0[b], (long long)s.next_pos);
+      if (t0[b] < s.P)
+        return fail(PS_EPOS, "sequence %d: t0=%lld lies inside the prefix (P=%d)", seq_ids[b],
+                    (long long)t0[b], s.P);
+    }
+    N += n[b];
+  }
+  if (N > INT32_MAX) return fail(PS_EINVAL, "%lld packed rows exceed 2^31 - 1", (long long)N);
+  if (N == 0) return ok();
+  if (!q || !out || !aligned16(q) || !aligned16(out))
+    return fail(PS_EINVAL, "q/out must be non-NULL 16-byte aligned device pointers");
+  if (!prompt && (!k_blk || !v_blk || !aligned16(k_blk) || !aligned16(v_blk)))
+    return fail(PS_EINVAL, "k_blk/v_blk must be non-NULL 16-byte aligned device pointers");
+  if ((r = check_device(c))) return r;
+  // paged: ring pages for the blocks' appended slots, planned before anything runs
+  std::vector<int32_t> avail = c->free_pages, idx, phys;
+  std::vector<std::vector<int32_t>> pages;
+  if (append_after && !prompt) {
+    pages.resize(B);
+    for (int b = 0; b < B; ++b) {
+      const SeqHost& s = c->seqs[seq_ids[b]];
+      pages[b] = s.pages;
+      const int64_t n_eff = n[b] < c->W ? n[b] : c->W;
+      if (n[b] > 0 && !plan_pages(c, seq_ids[b], pages[b],
+                                  (int64_t)s.head + s.count + (n[b] - n_eff), n_eff, avail, idx,
+                                  phys))
+        return fail(PS_ENOMEM, "the ring page pool has no free page left");
+    }
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t qrow = (size_t)Hq * c->d * c->esize, krow = (size_t)c->Hkv * c->d * c->esize;
+  if (ps::chunk_tc_supported(c->dev, c->dtype, c->d, G)) {
+    // entries with queries, in launches of at most kMaxChunkBatch
+    std::vector<ps::ChunkEntry> es;
+    int64_t tok = 0, tok_first = 0;
+    auto flush = [&]() -> cudaError_t {
+      if (es.empty()) return cudaSuccess;
+      cudaError_t e = ps::launch_chunk_tc(
+          c->dev, G, es.data(), (int)es.size(), Hq, (const char*)q + tok_first * qrow,
+          prompt ? nullptr : (const char*)k_blk + tok_first * krow,
+          prompt ? nullptr : (const char*)v_blk + tok_first * krow, (char*)out + tok_first * qrow,
+          scale, prompt ? 1 : 0, c->sm_count, st);
+      es.clear();
+      return e;
+    };
+    for (int b = 0; b < B; ++b) {
+      if (n[b] > 0) {
+        if (es.empty()) tok_first = tok;
+        const SeqHost& sh = c->seqs[seq_ids[b]];
+        es.push_back(ps::ChunkEntry{seq_ids[b], n[b], t0[b], sh.next_pos, sh.P, sh.head, sh.count,
+                                    sh.owner});
+        if ((int)es.size() == ps::kMaxChunkBatch) PS_CUDA(flush());
+      }
+      tok += n[b];
+    }
+    PS_CUDA(flush());
+  } else {
+    int64_t tok = 0;
+    for (int b = 0; b < B; ++b) {
+      if (n[b] > 0)
+        PS_CUDA(ps::launch_chunk_cc(
+            c->dev, c->dtype, G, seq_ids[b], t0[b], n[b], Hq, (const char*)q + tok * qrow,
+            prompt ? nullptr : (const char*)k_blk + tok * krow,
+            prompt ? nullptr : (const char*)v_blk + tok * krow, (char*)out + tok * qrow, scale,
+            prompt ? 1 : 0, st));
+      tok += n[b];
+    }
+  }
+  if (append_after && !prompt) {
+    if (!idx.empty())
+      PS_CUDA(ps::launch_page_set(c->dev, idx.data(), phys.data(), (int)idx.size(), st));
+    int64_t tok = 0;
+    for (int b = 0; b < B; ++b) {
+      if (n[b] > 0) {
+        ps::BatchIds ids;
+        memset(&ids, 0, sizeof(ids));
+        ids.seq[0] = seq_ids[b];
+        PS_CUDA(ps::launch_ring_append(c->dev, c->esize, ids, 1, (const char*)k_blk + tok * krow,
+                                       (const char*)v_blk + tok * krow, n[b], st));
+      }
+      tok += n[b];
+    }
+    c->free_pages = avail;
+    for (int b = 0; b < B; ++b) {
+      c->seqs[seq_ids[b]].pages = pages[b];
+      advance(c->seqs[seq_ids[b]], c->W, n[b]);
+    }
+  }
+  return ok();
+}
+
 extern "C" {
 
 const char* ps_last_error(void) { return g_err.c_str(); }
@@ -539,74 +656,26 @@ int ps_decode_step(ps_cache* c, const void* q, const void* k_new, const void* v_
 int ps_attend_chunk(ps_cache* c, int seq, const void* q, const void* k_blk, const void* v_blk,
                     int64_t t0, int n, int Hq, float scale, void* out, int append_after,
                     void* stream) {
-  if (!c) return fail(PS_EINVAL, "cache is NULL");
-  int r = check_seq(c, seq, true);
-  if (r) return r;
-  int G = 0;
-  if ((r = check_group(c, Hq, &G))) return r;
-  if (n < 0) return fail(PS_EINVAL, "negative n=%d", n);
-  const SeqHost& s = c->seqs[seq];
-  if (t0 != s.next_pos)
-    return fail(PS_EPOS, "t0=%lld does not follow the history (next position %lld)",
-                (long long)t0, (long long)s.next_pos);
-  if (t0 < s.P)
-    return fail(PS_EPOS, "t0=%lld lies inside the prefix (P=%d)", (long long)t0, s.P);
-  if (n == 0) return ok();
-  if (!q || !out || !k_blk || !v_blk || !aligned16(q) || !aligned16(out) || !aligned16(k_blk) ||
-      !aligned16(v_blk))
-    return fail(PS_EINVAL, "q/k_blk/v_blk/out must be non-NULL 16-byte aligned device pointers");
-  if ((r = check_device(c))) return r;
-  // paged: ring pages for the block's appended slots, planned before anything runs
-  std::vector<int32_t> avail = c->free_pages, idx, phys, pages = s.pages;
-  if (append_after) {
-    const int64_t n_eff = n < c->W ? n : c->W;
-    if (!plan_pages(c, seq, pages, (int64_t)s.head + s.count + (n - n_eff), n_eff, avail, idx,
-                    phys))
-      return fail(PS_ENOMEM, "the ring page pool has no free page left");
-  }
-  cudaStream_t st = (cudaStream_t)stream;
-  if (ps::chunk_tc_supported(c->dev, c->dtype, c->d, G))
-    PS_CUDA(ps::launch_chunk_tc(c->dev, G, seq, t0, n, Hq, q, k_blk, v_blk, out, scale, 0, st));
-  else
-    PS_CUDA(ps::launch_chunk_cc(c->dev, c->dtype, G, seq, t0, n, Hq, q, k_blk, v_blk, out, scale,
-                                0, st));
-  if (append_after) {
-    if (!idx.empty())
-      PS_CUDA(ps::launch_page_set(c->dev, idx.data(), phys.data(), (int)idx.size(), st));
-    ps::BatchIds ids;
-    memset(&ids, 0, sizeof(ids));
-    ids.seq[0] = seq;
-    PS_CUDA(ps::launch_ring_append(c->dev, c->esize, ids, 1, k_blk, v_blk, n, st));
-    c->free_pages = avail;
-    c->seqs[seq].pages = pages;
-    advance(c->seqs[seq], c->W, n);
-  }
-  return ok();
+  return attend_blocks(c, &seq, &t0, &n, 1, q, k_blk, v_blk, Hq, scale, out, append_after, false,
+                       stream);
+}
+
+int ps_attend_chunk_batch(ps_cache* c, const int* seq_ids, const int64_t* t0, const int* n, int B,
+                          const void* q, const void* k_blk, const void* v_blk, int Hq,
+                          float scale, void* out, int append_after, void* stream) {
+  return attend_blocks(c, seq_ids, t0, n, B, q, k_blk, v_blk, Hq, scale, out, append_after, false,
+                       stream);
 }
 
 int ps_attend_prompt(ps_cache* c, int seq, const void* q, int64_t t0, int n, int Hq, float scale,
                      void* out, void* stream) {
-  if (!c) return fail(PS_EINVAL, "cache is NULL");
-  int r = check_seq(c, seq, true);
-  if (r) return r;
-  int G = 0;
-  if ((r = check_group(c, Hq, &G))) return r;
-  if (n < 0) return fail(PS_EINVAL, "negative n=%d", n);
-  const SeqHost& s = c->seqs[seq];
-  if (t0 < 0 || t0 + n > s.P)
-    return fail(PS_EPOS, "prompt queries [%lld, %lld) are not inside the prefix (P=%d)",
-                (long long)t0, (long long)(t0 + n), s.P);
-  if (n == 0) return ok();
-  if (!q || !out || !aligned16(q) || !aligned16(out))
-    return fail(PS_EINVAL, "q/out must be non-NULL 16-byte aligned device pointers");
-  if ((r = check_device(c))) return r;
-  cudaStream_t st = (cudaStream_t)stream;
-  if (ps::chunk_tc_supported(c->dev, c->dtype, c->d, G))
-    PS_CUDA(ps::launch_chunk_tc(c->dev, G, seq, t0, n, Hq, q, nullptr, nullptr, out, scale, 1, st));
-  else
-    PS_CUDA(ps::launch_chunk_cc(c->dev, c->dtype, G, seq, t0, n, Hq, q, nullptr, nullptr, out,
-                                scale, 1, st));
-  return ok();
+  return attend_blocks(c, &seq, &t0, &n, 1, q, nullptr, nullptr, Hq, scale, out, 0, true, stream);
+}
+
+int ps_attend_prompt_batch(ps_cache* c, const int* seq_ids, const int64_t* t0, const int* n, int B,
+                           const void* q, int Hq, float scale, void* out, void* stream) {
+  return attend_blocks(c, seq_ids, t0, n, B, q, nullptr, nullptr, Hq, scale, out, 0, true,
+                       stream);
 }
 
 int ps_export_window(ps_cache* c, int seq, void* k, void* v, int64_t* pos, int32_t* count_out,

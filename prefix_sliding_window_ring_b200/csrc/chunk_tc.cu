@@ -6,9 +6,11 @@
 // ("Prefix Sliding" digest, sections 03 and 06); prompt queries (t < P)
 // attend to the prefix rows [0, t].  Prefix rows are read from the slab of the
 // sequence that owns them (itself, or the sequence whose prefix it shares).
-// One CTA takes a 128-row
-// query tile: 128/G consecutive positions of each of the G query heads that
-// share one key/value head, so every key tile feeds all G heads at once.
+// One launch serves a batch of sequences, each with its own block, packed end
+// to end.  One CTA takes a 128-row query tile of one entry: 128/G consecutive
+// positions of each of the G query heads that share one key/value head, so
+// every key tile feeds all G heads at once.  The grid covers the query tiles
+// of all entries, so the GPU fills up across sequences.
 //
 // Key tiles (128 rows) are walked range by range -- prefix rows, the ring
 // window as at most two contiguous slot runs split at the physical wrap, then
@@ -58,20 +60,34 @@ constexpr uint32_t kTileBytes = kBN * kHD * 2;  // one K or V tile: 32 KiB
 __host__ __device__ __forceinline__ uint32_t col_s(int st) { return st ? 128u : 0u; }
 
 struct ChunkArgs {
-  CUtensorMap qmap;   // q [n][Hq][128]: box (64, 1, PT)
+  CUtensorMap qmap;   // q [N][Hq][128] (entries packed): box (64, 1, PT)
   CUtensorMap kpre;   // cache K prefix rows [S*Hkv][pstride][128]: box (64, 128, 1)
   CUtensorMap vpre;
   CUtensorMap kring;  // cache K ring pages [nphys*Hkv][page_rows][128]: box (64, 128, 1)
   CUtensorMap vring;
-  CUtensorMap kblk;   // k_blk [n][Hkv][128]: box (64, 1, 128)
+  CUtensorMap kblk;   // k_blk [N][Hkv][128] (entries packed): box (64, 1, 128)
   CUtensorMap vblk;
   CacheDev c;
-  void* out;
-  int seq, n, Hq, G, PT;
+  void* out;   // [N][Hq][128]
+  int Hq, G, PT;
   int prompt;  // queries inside the prefix: causal over the prefix rows only
-  int64_t t0;
-  float sc;  // softmax scale * log2(e)
+  int nb;      // entries
+  float sc;    // softmax scale * log2(e)
+  int32_t seq[kMaxChunkBatch];
+  int32_t n[kMaxChunkBatch];
+  int64_t t0[kMaxChunkBatch];
+  int64_t tok0[kMaxChunkBatch];     // first packed row of the entry
+  int32_t qtc[kMaxChunkBatch + 1];  // query tiles of the entries before b
+  // each entry's ring state from the host's bookkeeping (no dependent load
+  // before the first copy; the device record is checked against it)
+  int64_t next_pos[kMaxChunkBatch];
+  int32_t P[kMaxChunkBatch];
+  int32_t head[kMaxChunkBatch];
+  int32_t count[kMaxChunkBatch];
+  int32_t owner[kMaxChunkBatch];
 };
+// Kernel parameters above 4 KB need CUDA 12.1 and sm_70 or later (limit 32764 bytes).
+static_assert(sizeof(ChunkArgs) <= 32764, "chunk arguments fit the kernel parameter space");
 
 struct __align__(1024) TcSmem {
   uint8_t q[2][kBM * 128];       // two 64-column blocks of 128-byte rows
@@ -209,11 +225,27 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = blockIdx.y;
   const int PT = a.PT;
-  const int i0 = blockIdx.x * PT;
-  const DevMeta m = a.c.meta[a.seq];
-  const int64_t plo = a.t0 + i0;
-  const int64_t phi = a.t0 + min(i0 + PT, a.n) - 1;
-  const KSched ks = make_sched(m, a.c.W, a.c.page_table ? a.c.page_rows : 0, a.t0, plo, phi,
+  // this CTA's entry and query tile
+  int eb = 0;
+  {
+    int hi = a.nb - 1;
+    while (eb < hi) {  // last entry with qtc[b] <= blockIdx.x
+      const int mid = (eb + hi + 1) >> 1;
+      if (a.qtc[mid] <= (int)blockIdx.x) eb = mid; else hi = mid - 1;
+    }
+  }
+  const int seq = a.seq[eb], n = a.n[eb];
+  const int64_t t0 = a.t0[eb], tok0 = a.tok0[eb];
+  const int i0 = ((int)blockIdx.x - a.qtc[eb]) * PT;
+  DevMeta m;
+  m.next_pos = a.next_pos[eb];
+  m.P = a.P[eb];
+  m.head = a.head[eb];
+  m.count = a.count[eb];
+  m.owner = a.owner[eb];
+  const int64_t plo = t0 + i0;
+  const int64_t phi = t0 + min(i0 + PT, n) - 1;
+  const KSched ks = make_sched(m, a.c.W, a.c.page_table ? a.c.page_rows : 0, t0, plo, phi,
                                a.prompt != 0);
   const int T = ks.ntiles;
 
@@ -231,8 +263,6 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
     ptx::mbar_init(&mma_done, 1);
     abort_flag = 0;
     ptx::fence_mbar_init();
-    const bool bad = a.prompt ? a.t0 + a.n > m.P : m.next_pos != a.t0;
-    if (bad && blockIdx.x == 0 && g == 0) atomicOr(a.c.err, ERR_BATCH);
   }
   if (warp == 2) {
     ptx::tmem_alloc(&tmem_slot, kTmemCols);
@@ -251,15 +281,24 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
       ptx::mbar_arrive_expect_tx(&q_full, 2 * kBM * 128);
       for (int hh = 0; hh < a.G; ++hh)
         for (int b = 0; b < 2; ++b)
-          ptx::tma_load_3d(&sm.q[b][hh * PT * 128], &a.qmap, b * 64, g * a.G + hh, i0, &q_full);
+          ptx::tma_load_3d(&sm.q[b][hh * PT * 128], &a.qmap, b * 64, g * a.G + hh,
+                           (int32_t)(tok0 + i0), &q_full);
+      if (i0 == 0 && g == 0) {  // once per entry: the device record must agree
+        const DevMeta md = a.c.meta[seq];
+        const bool bad = md.next_pos != m.next_pos || md.P != m.P || md.head != m.head ||
+                         md.count != m.count || md.owner != m.owner ||
+                         (a.prompt ? t0 + n > m.P : m.next_pos != t0);
+        if (bad) atomicOr(a.c.err, ERR_BATCH);
+      }
       for (int j = 0; j < T && !abort_flag; ++j) {
         const int st = j & 1;
         const KTile kt = tile_of(ks, j);
         if (j >= 2 && !wait_bar(&k_empty[st], ((j >> 1) - 1) & 1, &abort_flag)) break;
         // a ring tile lies within one page: (slot within the page, page's slab)
         const int32_t kslot = (int32_t)kt.row;  // ring slot (ring tiles)
-        const int ring_z = kt.src == 0 ? ring_page(a.c, a.seq, kslot) * a.c.Hkv + g : 0;
+        const int ring_z = kt.src == 0 ? ring_page(a.c, seq, kslot) * a.c.Hkv + g : 0;
         const int32_t ring_y = kt.src == 0 ? kslot % a.c.page_rows : 0;
+        const int32_t blk_row = (int32_t)(tok0 + kt.row);  // block tiles: packed row
         ptx::mbar_arrive_expect_tx(&k_full[st], kTileBytes);
         for (int b = 0; b < 2; ++b) {
           if (kt.src == 2)
@@ -267,7 +306,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
           else if (kt.src == 0)
             ptx::tma_load_3d(sm.k[st][b], &a.kring, b * 64, ring_y, ring_z, &k_full[st]);
           else
-            ptx::tma_load_3d(sm.k[st][b], &a.kblk, b * 64, g, (int32_t)kt.row, &k_full[st]);
+            ptx::tma_load_3d(sm.k[st][b], &a.kblk, b * 64, g, blk_row, &k_full[st]);
         }
         issued_k = j + 1;
         if (j >= 2 && !wait_bar(&v_empty[st], ((j >> 1) - 1) & 1, &abort_flag)) break;
@@ -278,7 +317,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
           else if (kt.src == 0)
             ptx::tma_load_3d(sm.v[st][b], &a.vring, b * 64, ring_y, ring_z, &v_full[st]);
           else
-            ptx::tma_load_3d(sm.v[st][b], &a.vblk, b * 64, g, (int32_t)kt.row, &v_full[st]);
+            ptx::tma_load_3d(sm.v[st][b], &a.vblk, b * 64, g, blk_row, &v_full[st]);
         }
         issued_v = j + 1;
       }
@@ -341,7 +380,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
     const int half = (warp - 4) >> 2;     // which 64 columns of S / O it owns
     const int r = quad * 32 + lane;       // query row of this thread
     const int hh = r / PT, i = i0 + r % PT;
-    const int64_t tq = a.t0 + i;
+    const int64_t tq = t0 + i;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     const int cbase = half * 64;          // first S/O column of this thread
     // A prompt query t sees [0, t]: the mask below with the prefix taken as [0, t].
@@ -457,13 +496,13 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
     if (ok && T > 0) {
       ptx::tc_fence_after();
       const float inv = 1.f / l_row;
-      uint16_t* orow = (uint16_t*)a.out + ((size_t)i * a.Hq + (size_t)g * a.G + hh) * kHD;
+      uint16_t* orow = (uint16_t*)a.out + ((size_t)(tok0 + i) * a.Hq + (size_t)g * a.G + hh) * kHD;
 #pragma unroll
       for (int c2 = 0; c2 < 2; ++c2) {
         uint32_t o[32];
         ptx::tmem_ld32(tmem + lane_base + kColO + cbase + c2 * 32, o);
         ptx::tmem_wait_ld();
-        if (i < a.n) {
+        if (i < n) {
           uint32_t w[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c)
@@ -522,14 +561,33 @@ bool chunk_tc_supported(const CacheDev& c, int dtype, int d, int G) {
   return pages_ok && dtype == 1 && d == kHD && (G == 1 || G == 2 || G == 4 || G == 8);
 }
 
-cudaError_t launch_chunk_tc(const CacheDev& c, int G, int seq, int64_t t0, int n, int Hq,
+cudaError_t launch_chunk_tc(const CacheDev& c, int G, const ChunkEntry* e, int nb, int Hq,
                             const void* q, const void* k_blk, const void* v_blk, void* out,
-                            float scale, int prompt, cudaStream_t st) {
+                            float scale, int prompt, int sm_count, cudaStream_t st) {
+  (void)sm_count;
+  if (nb < 1 || nb > kMaxChunkBatch) return cudaErrorInvalidValue;
   ChunkArgs a;
   memset(&a, 0, sizeof(a));
   const uint64_t row = kHD * 2;  // bytes per head row
   const int PT = kBM / G;
-  bool ok = map3d(&a.qmap, q, kHD, Hq, n, row, (uint64_t)Hq * row, 64, 1, PT);
+  int64_t N = 0;  // packed rows of all entries
+  a.qtc[0] = 0;
+  for (int b = 0; b < nb; ++b) {
+    if (e[b].n < 1) return cudaErrorInvalidValue;
+    a.seq[b] = e[b].seq;
+    a.n[b] = e[b].n;
+    a.t0[b] = e[b].t0;
+    a.tok0[b] = N;
+    a.qtc[b + 1] = a.qtc[b] + (e[b].n + PT - 1) / PT;
+    a.next_pos[b] = e[b].next_pos;
+    a.P[b] = e[b].P;
+    a.head[b] = e[b].head;
+    a.count[b] = e[b].count;
+    a.owner[b] = e[b].owner;
+    N += e[b].n;
+  }
+  if (N > INT32_MAX) return cudaErrorInvalidValue;
+  bool ok = map3d(&a.qmap, q, kHD, Hq, N, row, (uint64_t)Hq * row, 64, 1, PT);
   // prefix rows: [S*Hkv][pstride] rows from the buffer start; ring pages:
   // [nphys*Hkv][page_rows] slabs rstride rows apart from row rbase
   const uint64_t prows = c.pstride > 0 ? (uint64_t)c.pstride : 1;
@@ -543,32 +601,31 @@ cudaError_t launch_chunk_tc(const CacheDev& c, int G, int seq, int64_t t0, int n
                    (uint64_t)c.rstride * row, 64, kBN, 1);
   // a prompt launch loads no block rows; its block maps describe the cache
   // K/V (never used) so that every map is well formed
-  ok = ok && map3d(&a.kblk, prompt ? c.K : k_blk, kHD, c.Hkv, n, row, (uint64_t)c.Hkv * row, 64,
+  const uint64_t nblk = prompt ? prows : (uint64_t)N;
+  ok = ok && map3d(&a.kblk, prompt ? c.K : k_blk, kHD, c.Hkv, nblk, row, (uint64_t)c.Hkv * row, 64,
                    1, kBN);
-  ok = ok && map3d(&a.vblk, prompt ? c.V : v_blk, kHD, c.Hkv, n, row, (uint64_t)c.Hkv * row, 64,
+  ok = ok && map3d(&a.vblk, prompt ? c.V : v_blk, kHD, c.Hkv, nblk, row, (uint64_t)c.Hkv * row, 64,
                    1, kBN);
   if (!ok) return cudaErrorInvalidValue;
   a.c = c;
   a.out = out;
-  a.seq = seq;
-  a.n = n;
   a.Hq = Hq;
   a.G = G;
   a.PT = PT;
   a.prompt = prompt;
-  a.t0 = t0;
+  a.nb = nb;
   a.sc = scale * 1.4426950408889634f;
   const size_t dyn = sizeof(TcSmem) + 1024;
   static std::atomic<uint64_t> configured{0};
   int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
   if (!(configured.load() & (1ull << (dev & 63)))) {
-    e = cudaFuncSetAttribute(k_chunk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
-    if (e != cudaSuccess) return e;
+    err = cudaFuncSetAttribute(k_chunk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
+    if (err != cudaSuccess) return err;
     configured.fetch_or(1ull << (dev & 63));
   }
-  dim3 grid((n + PT - 1) / PT, c.Hkv);
+  dim3 grid(a.qtc[nb], c.Hkv);
   k_chunk_tc<<<grid, kThreadsTC, dyn, st>>>(a);
   return cudaGetLastError();
 }

@@ -34,10 +34,16 @@
 // transpose-reduction leaves every lane with one complete score, the lane
 // exponentiates only that score, and the 8 weights are gathered back for the
 // weighted sum of the value rows.  Pairs of float32 values use the packed
-// sm_100 FMA (each half is an ordinary IEEE fma).
+// sm_100 FMA (each half is an ordinary IEEE fma).  A lane holds VEC elements
+// of a row (16 bytes, or 8 for bfloat16 at G >= 8 so that q and the G
+// accumulators stay in registers).  The running max of a head moves only when
+// a score passes it by more than 2^8, so the accumulators are rescaled on few
+// updates; the exact max is not needed, only one shared by the sum and the
+// accumulator (the weights stay below 2^8).
 //
 // Every wait is bounded; a time-out stops the CTA, sets ERR_TIMEOUT and lets
 // the copies already issued land before the CTA exits.
+#include <type_traits>
 #include <math.h>
 #include <string.h>
 
@@ -79,6 +85,7 @@ constexpr int kStages = PS_DEC_STAGES;
 constexpr long long kWaitLimitCycles = 1ll << 30;  // about half a second
 constexpr int kPieceBatch = 8;  // partials read together by the pair merge
 constexpr int kMergeThreads = 128;
+constexpr float kRaiseLog2 = 8.0f;  // running-max hysteresis, log2 units
 
 template <typename T, int D> struct DecTile {
   static constexpr int RW = PS_DEC_WARP_BYTES / (D * (int)sizeof(T));  // rows per warp per tile
@@ -107,7 +114,16 @@ struct DecodeArgs {
 // Kernel parameters above 4 KB need CUDA 12.1 and sm_70 or later (limit 32764 bytes).
 static_assert(sizeof(DecodeArgs) <= 32764, "decode arguments fit the kernel parameter space");
 
-// bfloat16 pairs of a 16-byte vector as float2 (exact widening).
+// Elements of one row a lane holds: a 16-byte vector, or for bfloat16 with
+// G >= 8 an 8-byte one -- q and the accumulator of all G heads live in
+// registers, G * VEC * 2 floats, which must stay well inside the 128-register
+// budget of a thread.
+template <typename T, int G> struct LaneVec {
+  static constexpr int N = (sizeof(T) == 2 && G >= 8) ? 4 : Vec<T>::N;
+  using Raw = typename std::conditional<N * sizeof(T) == 16, uint4, uint2>::type;
+};
+
+// Pairs of a lane's vector as float2 (exact widening for bfloat16).
 template <typename T> struct Vec2;
 template <> struct Vec2<uint16_t> {
   __device__ __forceinline__ static void unpack(const uint4& x, float2* f) {
@@ -115,6 +131,10 @@ template <> struct Vec2<uint16_t> {
     f[1] = make_float2(bf16lo(x.y), bf16hi(x.y));
     f[2] = make_float2(bf16lo(x.z), bf16hi(x.z));
     f[3] = make_float2(bf16lo(x.w), bf16hi(x.w));
+  }
+  __device__ __forceinline__ static void unpack(const uint2& x, float2* f) {
+    f[0] = make_float2(bf16lo(x.x), bf16hi(x.x));
+    f[1] = make_float2(bf16lo(x.y), bf16hi(x.y));
   }
 };
 template <> struct Vec2<float> {
@@ -129,7 +149,8 @@ template <> struct Vec2<float> {
 // operations each) apply directly.
 template <typename T, int D, int G>
 struct DecState {
-  static constexpr int VEC = Vec<T>::N;
+  static constexpr int VEC = LaneVec<T, G>::N;
+  using Raw = typename LaneVec<T, G>::Raw;
   static constexpr int V2 = VEC / 2;
   static constexpr int LPR = D / VEC;   // lanes per row
   static constexpr int RPI = 32 / LPR;  // rows per warp load instruction
@@ -157,7 +178,7 @@ struct DecState {
     const float2 s2 = make_float2(qscale, qscale);
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      uint4 raw = *(const uint4*)(qrow + (size_t)h * D + c * VEC);
+      const Raw raw = *(const Raw*)(qrow + (size_t)h * D + c * VEC);
       Vec2<T>::unpack(raw, q[h]);
 #pragma unroll
       for (int e = 0; e < V2; ++e) {
@@ -170,7 +191,7 @@ struct DecState {
     lpart = 0.f;
   }
 
-  __device__ __forceinline__ void update(const uint4 (&kr)[U], const uint4 (&vr)[U],
+  __device__ __forceinline__ void update(const Raw (&kr)[U], const Raw (&vr)[U],
                                          const bool (&ok)[U]) {
     const unsigned FULL = 0xffffffffu;
     const int lane = threadIdx.x & 31;
@@ -223,28 +244,34 @@ struct DecState {
     if (G <= 4) tm = fmaxf(tm, __shfl_xor_sync(FULL, tm, S1));
     if (G <= 2) tm = fmaxf(tm, __shfl_xor_sync(FULL, tm, S2));
     if (G == 1) tm = fmaxf(tm, __shfl_xor_sync(FULL, tm, S3));
-    const float mo_new = fmaxf(mo, tm);
+    // The running max moves only when a score passes it by more than 2^8
+    // (weights stay below 2^8, far from float overflow), so the rescale of
+    // the accumulators is skipped for nearly every row group.
+    const float mo_new = tm > mo + kRaiseLog2 ? tm : mo;
     const float p = okown ? exp2f(sc - mo_new) : 0.f;
-    const float ao = (mo_new == -INFINITY) ? 1.f : exp2f(mo - mo_new);
-    lpart = lpart * ao + p;
+    if (mo_new != mo) lpart *= exp2f(mo - mo_new);
+    lpart += p;
     mo = mo_new;
-    // every head's new max and rescale factor, in every lane
-    float alpha[G];
+    // every head's new max, in every lane (the same rule as mo)
+    float mold[G];
+    bool raise = false;
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       const float th = __shfl_sync(FULL, tm, base | lane_of(h));
-      const float mn = fmaxf(m[h], th);
-      alpha[h] = (mn == -INFINITY) ? 1.f : exp2f(m[h] - mn);
-      m[h] = mn;
+      mold[h] = m[h];
+      if (th > m[h] + kRaiseLog2) { m[h] = th; raise = true; }
     }
     float pk[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) pk[k] = __shfl_sync(FULL, p, base | lane_of(k));
+    if (raise) {
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float2 a2 = make_float2(alpha[h], alpha[h]);
+      for (int h = 0; h < G; ++h) {
+        const float alpha = exp2f(mold[h] - m[h]);  // 0 when mold is -inf, 1 when unchanged
+        const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
-      for (int e = 0; e < V2; ++e) o[h][e] = __fmul2_rn(o[h][e], a2);
+        for (int e = 0; e < V2; ++e) o[h][e] = __fmul2_rn(o[h][e], a2);
+      }
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -262,17 +289,17 @@ struct DecState {
   // Rows [0, nrows) of a contiguous tile in shared memory (row stride D).
   __device__ __forceinline__ void tile(const T* ks, const T* vs, int nrows) {
     for (int r0 = 0; r0 < nrows; r0 += STEP) {
-      uint4 kr[U], vr[U];
+      Raw kr[U], vr[U];
       bool ok[U];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int r = r0 + u * RPI + rs;
         ok[u] = r < nrows;
-        kr[u] = make_uint4(0, 0, 0, 0);
+        kr[u] = Raw{};
         vr[u] = kr[u];
         if (ok[u]) {
-          kr[u] = *(const uint4*)(ks + (size_t)r * D + c * VEC);
-          vr[u] = *(const uint4*)(vs + (size_t)r * D + c * VEC);
+          kr[u] = *(const Raw*)(ks + (size_t)r * D + c * VEC);
+          vr[u] = *(const Raw*)(vs + (size_t)r * D + c * VEC);
         }
       }
       update(kr, vr, ok);

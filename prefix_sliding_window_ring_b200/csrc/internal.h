@@ -57,11 +57,21 @@ cudaError_t launch_decode(const CacheDev& c, int dtype, int G, const BatchIds& i
 
 // chunk_tc.cu (tcgen05 chunk kernel: bf16, head_dim 128)
 bool chunk_tc_supported(const CacheDev& c, int dtype, int d, int G);
-// prompt != 0: queries t0..t0+n-1 inside the prefix attend causally to the
-// prefix rows [0, t] (k_blk / v_blk unused); otherwise a chunk at t0 == next_pos.
-cudaError_t launch_chunk_tc(const CacheDev& c, int G, int seq, int64_t t0, int n, int Hq,
+// One sequence's block in a batched chunk or prompt launch: n >= 1 queries at
+// t0..t0+n-1, rows packed end to end in q / k_blk / v_blk / out in entry order.
+struct ChunkEntry {
+  int seq;
+  int n;
+  int64_t t0;
+  int64_t next_pos;  // the sequence's ring state from the host's bookkeeping
+  int P, head, count, owner;
+};
+constexpr int kMaxChunkBatch = 64;  // entries per launch
+// prompt != 0: queries inside the prefix attend causally to the prefix rows
+// [0, t] (k_blk / v_blk unused); otherwise chunks at t0 == next_pos.
+cudaError_t launch_chunk_tc(const CacheDev& c, int G, const ChunkEntry* e, int nb, int Hq,
                             const void* q, const void* k_blk, const void* v_blk, void* out,
-                            float scale, int prompt, cudaStream_t st);
+                            float scale, int prompt, int sm_count, cudaStream_t st);
 
 // attend.cu (CUDA-core chunk kernel)
 cudaError_t launch_chunk_cc(const CacheDev& c, int dtype, int G, int seq, int64_t t0, int n,
