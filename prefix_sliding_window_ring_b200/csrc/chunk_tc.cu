@@ -236,7 +236,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
   }
   const int seq = a.seq[eb], n = a.n[eb];
   const int64_t t0 = a.t0[eb], tok0 = a.tok0[eb];
-  const int i0 = ((int)blockIdx.x - a.qtc[eb]) * PT;
+  // an entry's query tiles run last first: later queries see more keys (causal
+  // prompts, windows not yet full), so the longest CTAs start first and the
+  // launch ends on short ones
+  const int i0 = (a.qtc[eb + 1] - 1 - (int)blockIdx.x) * PT;
   DevMeta m;
   m.next_pos = a.next_pos[eb];
   m.P = a.P[eb];
