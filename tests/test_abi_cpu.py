@@ -82,3 +82,39 @@ def test_paged_cache_bytes_and_argument_checks():
     with pytest.raises(abi.PSError) as e:
         abi.ps_ring_pages_free(None)
     assert e.value.code == abi.PS_EINVAL
+
+
+def test_every_call_rejects_a_null_cache_before_touching_cuda():
+    from prefix_sliding_window_ring_b200 import abi
+    lib = ctypes.CDLL(abi.LIB_PATH)
+    for name, (res, args) in abi.SIGNATURES.items():
+        getattr(lib, name).restype, getattr(lib, name).argtypes = res, args
+    ids = (ctypes.c_int * 2)(0, 1)
+    ts = (ctypes.c_int64 * 2)(5, 6)
+    ns = (ctypes.c_int * 2)(1, 1)
+    info = abi.SeqInfo()
+    calls = {
+        "ps_seq_info_get": (None, 0, ctypes.byref(info)),
+        "ps_seq_reset": (None, 0, 0, None),
+        "ps_prefill_prefix": (None, 0, None, None, 1, None),
+        "ps_share_prefix": (None, 1, 0, None),
+        "ps_append_kv": (None, ids, 2, None, None, 1, None),
+        "ps_attend_decode": (None, None, ids, ts, 2, 2, 1.0, None, None, 0, None),
+        "ps_attend_decode_static": (None, None, ids, ts, 2, 2, 1.0, None, None),
+        "ps_decode_step": (None, None, None, None, ids, ts, 2, 2, 1.0, None, None, 0, None),
+        "ps_attend_chunk": (None, 0, None, None, None, 5, 1, 2, 1.0, None, 0, None),
+        "ps_attend_chunk_batch": (None, ids, ts, ns, 2, None, None, None, 2, 1.0, None, 0, None),
+        "ps_attend_prompt": (None, 0, None, 0, 1, 2, 1.0, None, None),
+        "ps_attend_prompt_batch": (None, ids, ts, ns, 2, None, 2, 1.0, None, None),
+        "ps_export_window": (None, 0, None, None, None, None, None),
+        "ps_import_window": (None, 0, 5, None, None, 1, 0, None),
+        "ps_debug_visible": (None, 0, 5, None, None, None),
+        "ps_debug_wait_timeout": (None, 1000, None),
+        "ps_device_error": (None, None, None),
+        "ps_ring_pages_free": (None,),
+    }
+    for name, a in calls.items():
+        assert getattr(lib, name)(*a) == abi.PS_EINVAL, name
+        assert abi.ps_last_error(), name
+    assert lib.ps_decode_workspace_bytes(None, 1, 1) == 0
+    lib.ps_cache_destroy(None)  # deleting NULL is a no-op
