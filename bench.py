@@ -409,11 +409,15 @@ def run_ours(args, rank, world, local_rank):
     prefill = None
     if rank == 0 and not args.no_prefill:
         prefill = prefill_measure(max(3, min(args.steps, 10)))
-    ragged = shared = paged = None
+    ragged = shared = paged = t_sweep = None
     if rank == 0 and not args.no_prefill:
         ragged = ragged_measure(max(3, min(args.steps, 10)))
         shared = shared_prefix_measure(max(3, min(args.steps, 10)))
         paged = paged_measure(max(3, min(args.steps, 10)))
+        try:  # an extra section: a failure here is reported, not fatal to the line
+            t_sweep = t_sweep_measure(max(args.steps, 16))
+        except Exception as e:  # noqa: BLE001
+            t_sweep = {"error": f"{type(e).__name__}: {e}"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -448,6 +452,7 @@ def run_ours(args, rank, world, local_rank):
         "ragged": ragged,
         "shared_prefix": shared,
         "paged": paged,
+        "t_sweep": t_sweep,
     }
     print(json.dumps(line), flush=True)
 
@@ -766,6 +771,63 @@ def paged_measure(steps: int):
         res[key] = {"us_per_step": round(ms * 1e3, 2),
                     "GBps": round(kv_bytes_per_step() / (ms / 1e3) / 1e9, 1)}
         c.close()
+        torch.cuda.empty_cache()
+    return res
+
+
+def t_sweep_measure(steps: int):
+    """The decode call (ps_attend_decode, B=8, Hq=16, Hkv=8, d=128, bf16) at the
+    positions the workload is quoted at, t in {2048, 4224, 16384, 65536} with
+    P=128, W=4096: n = P + min(W, t - P + 1) visible rows (2049 at t=2048, 4224
+    from t=4223 on).  Beside them the same 4224 rows as plain causal attention
+    over the whole history (P=0, W=8192 >= t+1 at t=4223), the full-history
+    case of the same kernel.  Inputs are seeded N(0,1) rows drawn on the device
+    (only timing is taken here); 4 disjoint batches of 8 sequences rotate, so
+    every call streams from HBM (at least 268 MB resident)."""
+    import torch
+
+    from prefix_sliding_window_ring_b200 import PS_BF16, Cache
+    peak, _ = load_peaks()
+    g = torch.Generator(device="cuda").manual_seed(SEED + 7)
+    scale = 1.0 / math.sqrt(D)
+    res = {"note": "ps_attend_decode, B=8 Hq=16 Hkv=8 d=128 bf16; 4 rotating batches (HBM-resident)"}
+    cases = [("t2048", P, W, 2048), ("t4224", P, W, 4224), ("t16384", P, W, 16384),
+             ("t65536", P, W, 65536), ("causal_P0_W8192_t4223", 0, 8192, 4223)]
+    for name, Pc, Wc, t in cases:
+        S = B * ROT
+        c = Cache(Wc, max(Pc, 1), HKV, D, PS_BF16, S)
+        nwin = min(Wc, t - Pc + 1)  # window rows held once position t is stored
+        for s in range(S):
+            h0 = (s * 613) % Wc
+            c.seq_reset(s, h0)
+            kp = torch.randn((Pc, HKV, D), generator=g, device="cuda").to(torch.bfloat16)
+            vp = torch.randn((Pc, HKV, D), generator=g, device="cuda").to(torch.bfloat16)
+            c.prefill_prefix(s, kp, vp, Pc)
+            kw = torch.randn((nwin, HKV, D), generator=g, device="cuda").to(torch.bfloat16)
+            vw = torch.randn((nwin, HKV, D), generator=g, device="cuda").to(torch.bfloat16)
+            c.import_window(s, t + 1, kw, vw, nwin, h0)
+            del kp, vp, kw, vw
+        q = torch.randn((B, HQ, D), generator=g, device="cuda").to(torch.bfloat16)
+        out = torch.empty_like(q)
+        ws = c.decode_workspace(B, HQ)
+
+        def dec(i, st=None):
+            r = i % ROT
+            c.attend_decode(q, list(range(r * B, (r + 1) * B)), [t] * B, HQ, scale, out, ws, st)
+
+        for i in range(2 * ROT):
+            dec(i)
+        torch.cuda.synchronize()
+        ms = time_graph(torch, dec, max(steps, 4 * ROT))
+        if c.device_error():
+            raise RuntimeError(f"device error word set by the decode at {name}")
+        nvis = Pc + nwin
+        gbs = B * HKV * nvis * D * 2 * 2 / (ms / 1e3) / 1e9
+        res[name] = {"t": t, "P": Pc, "W": Wc, "visible_rows": nvis,
+                     "us_per_call": round(ms * 1e3, 2), "GBps": round(gbs, 1),
+                     "frac": round(gbs / peak, 4), "tokens_per_s": round(B / (ms / 1e3), 1)}
+        c.close()
+        del q, out, ws
         torch.cuda.empty_cache()
     return res
 
