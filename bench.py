@@ -78,6 +78,18 @@ def kv_bytes_per_step():
     return B * kv_bytes_per_seq()
 
 
+def prefill_flops(Wp: int) -> float:
+    """Visible (query, key) pairs of the chunk-prefill step, 4 d flops per pair per
+    query head (Q K^T and P V): every query of a block at t0 = 100000 sees its
+    P + W keys (the window is full)."""
+    return 4.0 * D * HQ * PF_N * (PF_P + Wp) * PF_SEQS
+
+
+def prompt_flops() -> float:
+    """Visible pairs of the prompt-prefill step: prompt query t sees t + 1 keys."""
+    return 4.0 * D * HQ * (PR_P * (PR_P + 1) / 2) * PF_SEQS
+
+
 def decode_traffic():
     """DRAM bytes per decode launch from the committed ncu record, or None when
     the decode kernel's sources have changed since that capture."""
@@ -520,7 +532,7 @@ def prefill_measure(steps: int):
         if c.device_error():
             raise RuntimeError("device error word set by the chunk kernel")
         ms = min(time_graph(torch, step, steps) for _ in range(2))
-        flops = 4.0 * D * HQ * PF_N * (PF_P + Wp) * PF_SEQS
+        flops = prefill_flops(Wp)
         tf = flops / (ms / 1e3) / 1e12
         res[f"W{Wp}"] = {"ms_per_step": round(ms, 4), "gflop_per_step": round(flops / 1e9, 1),
                          "achieved": round(tf, 1), "frac": round(tf / peak, 4)}
@@ -568,7 +580,7 @@ def prompt_measure(steps: int, peak: float):
     if c.device_error():
         raise RuntimeError("device error word set by the prompt kernel")
     ms = min(time_graph(torch, step, steps) for _ in range(2))
-    flops = 4.0 * D * HQ * (PR_P * (PR_P + 1) / 2) * PF_SEQS
+    flops = prompt_flops()
     tf = flops / (ms / 1e3) / 1e12
     c.close()
     del q, o
