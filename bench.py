@@ -522,7 +522,7 @@ def prefill_measure(steps: int):
         scale = 1.0 / math.sqrt(D)
 
         def step(i, st=None):
-            # one persistent launch over the four sequences' query tiles
+            # one launch over the four sequences' query tiles
             c.attend_chunk_batch(ids, [PF_T0] * PF_SEQS, [PF_N] * PF_SEQS, q, kb, vb, HQ, scale,
                                  o, 0, st)
 

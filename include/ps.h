@@ -158,8 +158,9 @@ PS_API int ps_attend_prompt(ps_cache* c, int seq, const void* q, int64_t t0, int
  * t0[b]..t0[b]+n[b]-1 (host arrays; n[b] >= 0, 0 <= t0[b], t0[b]+n[b] <= P_s).
  * The entries' rows are packed end to end in entry order: q, out
  * [sum n][Hq][d] (device), entry b from row n[0]+...+n[b-1].  On the
- * tensor-core kernel the whole batch is one persistent launch, so one
- * sequence's tail of work does not leave the GPU partly idle.
+ * tensor-core kernel the whole batch is one launch whose grid covers every
+ * entry's query tiles, so one sequence's tail of work does not leave the GPU
+ * partly idle.
  * Errors: as ps_attend_prompt, checked for every entry before anything runs. */
 PS_API int ps_attend_prompt_batch(ps_cache* c, const int* seq_ids, const int64_t* t0,
                                   const int* n, int B, const void* q, int Hq, float scale,
@@ -262,7 +263,7 @@ PS_API int ps_attend_chunk(ps_cache* c, int seq, const void* q, const void* k_bl
  * order: q, out [sum n][Hq][d]; k_blk, v_blk [sum n][Hkv][d] (device), entry
  * b from row n[0]+...+n[b-1].  With append_after != 0 every entry's block is
  * then appended to its ring.  On the tensor-core kernel the whole batch is one
- * persistent launch (one CTA per SM working through all entries' query tiles).
+ * launch with one CTA per (query tile, kv head) of every entry.
  * Errors: as ps_attend_chunk, checked for every entry (and, for a paged cache,
  * the pages of all appends planned) before anything runs; PS_ENOMEM if the
  * page pool cannot take all the appends. */

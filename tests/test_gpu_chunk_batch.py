@@ -1,8 +1,8 @@
 """GPU parity of the batched chunk and prompt calls (ps_attend_chunk_batch,
 ps_attend_prompt_batch): one launch over several sequences, rows packed end
 to end, gives bit for bit the outputs of one call per sequence -- on the
-persistent tensor-core kernel (with more query tiles than SMs, so CTAs take
-several units across sequences) and on the CUDA-core kernel -- appends the
+tensor-core kernel (with more query-tile CTAs than SMs, so the launch runs in
+several waves across sequences) and on the CUDA-core kernel -- appends the
 same rows to the rings, matches the oracle on sampled rows, and rejects a bad
 batch before anything runs."""
 import numpy as np
@@ -40,7 +40,7 @@ def _setup(dtype, d, Hq, Hkv, W, P, starts, heads, page=0, seed=41):
 
 
 # dtype, d, Hq, Hkv, W, P, page_rows, block lengths.  The tensor-core cases have
-# 182 query-tile units (more than the 148 SMs: CTAs take several, across
+# 182 query-tile CTAs (more than the 148 SMs: the launch runs in waves that mix
 # sequences), while each sequence alone has fewer.
 CASES = [
     ("bf16", 128, 4, 2, 512, 96, 0, [3000, 0, 129, 2500, 63]),
