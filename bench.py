@@ -884,9 +884,20 @@ def cpu_baseline(seed, kscale, budget_s=15.0, nthreads=None):
         if el >= budget_s or reps >= 1000:
             break
     tok = reps * B
+    # the same sample on one core, for a per-core figure (a short bounded run)
+    reps1 = 0
+    t1 = time.perf_counter()
+    while True:
+        batch.run(1)
+        reps1 += 1
+        el1 = time.perf_counter() - t1
+        if el1 >= min(budget_s / 4, 5.0) or reps1 >= 250:
+            break
     return {"value": round(tok / el, 2), "unit": UNIT, "cores": nthreads, "kind": "oracle",
             "sample": f"{reps} repetitions of one {B}-sequence decode step at t={T_START} "
-                      f"(float64 masked attention, {reps * B} sequence-decodes, {el:.1f} s)"}
+                      f"(float64 masked attention, {reps * B} sequence-decodes, {el:.1f} s)",
+            "one_core": {"value": round(reps1 * B / el1, 2), "unit": UNIT,
+                         "sample": f"{reps1} repetitions on 1 thread, {el1:.1f} s"}}
 
 
 def run_reference(args, rank, world):
