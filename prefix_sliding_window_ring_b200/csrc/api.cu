@@ -14,6 +14,7 @@
 
 #include "ps.h"
 #include "internal.h"
+#include "page_plan.h"
 
 namespace {
 
@@ -141,31 +142,14 @@ int check_group(const ps_cache* c, int Hq, int* G) {
   return PS_OK;
 }
 
-// Paged cache: ring slots [slot0, slot0 + n) (mod W) of sequence `seq` are
-// about to be written.  Assigns a physical page to every ring page they touch
-// that has none yet, taking pages from `avail` and recording the page-table
-// entries to set; `pages` is the sequence's page list to update.  Returns
-// false if the pool runs out (the caller then changes nothing).
+// Paged cache: page planning for a write to ring slots [slot0, slot0 + n) of
+// sequence `seq` (page_plan.h); nothing to do for an unpaged cache.
 bool plan_pages(const ps_cache* c, int seq, std::vector<int32_t>& pages, int64_t slot0, int64_t n,
                 std::vector<int32_t>& avail, std::vector<int32_t>& idx,
                 std::vector<int32_t>& phys) {
-  if (!c->paged || n <= 0) return true;
-  const int64_t W = c->W, pr = c->dev.page_rows;
-  int64_t s = ((slot0 % W) + W) % W;
-  for (int64_t left = n < W ? n : W; left > 0;) {
-    const int64_t page = s / pr;
-    const int64_t chunk = pr - s % pr < left ? pr - s % pr : left;
-    if (pages[page] < 0) {
-      if (avail.empty()) return false;
-      pages[page] = avail.back();
-      avail.pop_back();
-      idx.push_back((int32_t)(seq * (int64_t)c->dev.npg + page));
-      phys.push_back(pages[page]);
-    }
-    left -= chunk;
-    s = (s + chunk) % W;
-  }
-  return true;
+  if (!c->paged) return true;
+  const ps::PageShape sh{c->W, c->dev.page_rows, c->dev.npg};
+  return ps::plan_pages(sh, seq, pages, slot0, n, avail, idx, phys);
 }
 
 void advance(SeqHost& s, int W, int64_t n) {
