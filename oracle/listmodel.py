@@ -8,11 +8,12 @@ Cells are ``(pos, payload)`` tuples; the payload is opaque to the model.
 
 - ``last_window`` / ``valid``: blog section 2.3.  The legal cache for history
   ``hs`` is ``hs`` with its first ``len(hs) - min(w, len(hs))`` cells dropped.
-- ``step`` / ``run``: blog sections 3.3 and 4.2.  Append the new cell, then drop
-  the oldest one when the length exceeds ``w``; ``run`` folds ``step`` over a
-  token stream from the empty cache.  The branch condition is garbled on the
-  page; it is read as "w < length after the append", the only reading under
-  which the key equation of section 2.4 holds at the just-full boundary.
+- ``step`` / ``run``: blog sections 3.3 and 4.2.  A token joins the end of the
+  cache and only the newest ``w`` cells are kept; ``run`` folds ``step`` over a
+  token stream from the empty cache.  The page's eviction condition is garbled;
+  it is read as "evict when the grown cache holds more than w cells", the only
+  reading under which the key equation of section 2.4 holds at the just-full
+  boundary.
 - ``position_invariant``: blog section 3.2 (some base with pos_i = base + i).
 - ``RingBuffer`` / ``ring_to_list``: blog section 3.4 (fixed array plus head;
   logical cell i lives in slot (head + i) mod w).  The page maps all w slots;
@@ -29,19 +30,20 @@ Cell = Tuple[int, Any]
 
 
 def last_window(w: int, hs: Sequence[Cell]) -> List[Cell]:
-    n = len(hs)
-    return list(hs[n - min(w, n):])
+    """The newest ``w`` cells of the history (all of it while it is shorter)."""
+    return list(hs[max(0, len(hs) - w):])
 
 
 def valid(w: int, hs: Sequence[Cell], c: Sequence[Cell]) -> bool:
+    """The cache is exactly the last window of the history: same cells, same order."""
     return list(c) == last_window(w, hs)
 
 
 def step(w: int, c: Sequence[Cell], kv: Cell) -> List[Cell]:
-    c2 = list(c) + [kv]
-    if w < len(c2):
-        c2 = c2[1:]
-    return c2
+    """One token: the cache with the new cell at its end, cut back to its
+    newest ``w`` cells.  For a cache of at most ``w`` cells that evicts exactly
+    the oldest cell when the grown cache would hold ``w + 1``."""
+    return [*c, kv][-w:]
 
 
 def run(w: int, tokens: Iterable[Cell]) -> List[Cell]:
@@ -52,6 +54,8 @@ def run(w: int, tokens: Iterable[Cell]) -> List[Cell]:
 
 
 def position_invariant(c: Sequence[Cell]) -> bool:
+    """Some base position makes cell i hold position base + i (consecutive,
+    increasing by one); the empty cache satisfies it."""
     if not c:
         return True
     base = c[0][0]

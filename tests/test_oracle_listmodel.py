@@ -186,3 +186,100 @@ def test_exhaustive_small_streams():
     for w, n in itertools.product(range(1, 5), range(0, 9)):
         xs = cells(range(10, 10 + n))
         assert lm.run(w, xs) == lm.last_window(w, xs)
+
+
+# ---- negative pins: the obligations must reject caches that break them ----
+# (blog section 2.3 Valid: the cache IS the last window, cells and order;
+#  section 3.2 PositionInvariant: cell i holds base + i for one base)
+
+def _bad_caches(w, n):
+    """Caches that are NOT the last window of history cells(range(n)), n >= w + 2,
+    each with the rule it breaks."""
+    hs = cells(range(n))
+    good = hs[n - w:]
+    bad = {
+        "reordered": good[::-1] if w > 1 else None,
+        "oldest_stale": [hs[n - w - 1]] + good[1:],          # an evicted cell kept
+        "one_too_many": hs[n - w - 1:],                       # w + 1 cells
+        "newest_missing": good[:-1],                          # truncated at the end
+        "oldest_missing": good[1:],                           # truncated at the start
+        "shifted_back": hs[n - w - 1:n - 1],                  # the window one step late
+        "gap": good[:1] + good[2:] + [hs[0]] if w > 2 else None,
+        "payload_changed": good[:-1] + [(n - 1, "other")],
+        "empty": [],
+    }
+    return hs, {k: v for k, v in bad.items() if v is not None}
+
+
+@pytest.mark.parametrize("w", [1, 2, 3, 5, 8])
+def test_valid_rejects_every_other_cache(w):
+    n = 3 * w + 2
+    hs, bad = _bad_caches(w, n)
+    assert lm.valid(w, hs, hs[n - w:])
+    for name, c in bad.items():
+        assert not lm.valid(w, hs, c), name
+    # while the history is shorter than w the whole history is the only valid cache
+    short = cells(range(w - 1)) if w > 1 else []
+    assert lm.valid(w, short, short)
+    if short:
+        assert not lm.valid(w, short, short[1:])
+        assert not lm.valid(w, short, short + [(99, "x")])
+
+
+def test_position_invariant_rejects_non_consecutive():
+    assert lm.position_invariant(cells([7]))
+    assert lm.position_invariant(cells([3, 4, 5, 6]))
+    for name, ps in {"gap": [3, 4, 6], "descending": [6, 5, 4], "repeat": [4, 4, 5],
+                     "late_gap": [0, 1, 2, 3, 5], "step_two": [0, 2, 4],
+                     "first_off": [2, 4, 5, 6], "swapped_middle": [3, 5, 4, 6]}.items():
+        assert not lm.position_invariant(cells(ps)), name
+
+
+# mutants of the two predicates that accept too much; each must fail a pin above
+
+def _valid_any_order(w, hs, c):
+    return sorted(c) == sorted(lm.last_window(w, hs))
+
+
+def _valid_subset(w, hs, c):
+    lw = lm.last_window(w, hs)
+    return all(cell in lw for cell in c)
+
+
+def _valid_positions_only(w, hs, c):
+    return [x[0] for x in c] == [x[0] for x in lm.last_window(w, hs)]
+
+
+def _valid_length_only(w, hs, c):
+    return len(c) == min(w, len(hs))
+
+
+def _pi_nondecreasing(c):
+    return all(c[i][0] >= c[0][0] + i for i in range(len(c)))
+
+
+def _pi_endpoints(c):
+    return not c or c[-1][0] - c[0][0] == len(c) - 1
+
+
+def _pi_increasing(c):
+    return all(c[i][0] < c[i + 1][0] for i in range(len(c) - 1))
+
+
+def test_predicate_mutants_are_caught(monkeypatch):
+    caught = []
+    mutants = [("valid", _valid_any_order), ("valid", _valid_subset),
+               ("valid", _valid_positions_only), ("valid", _valid_length_only),
+               ("position_invariant", _pi_nondecreasing),
+               ("position_invariant", _pi_endpoints),
+               ("position_invariant", _pi_increasing)]
+    for name, mutant in mutants:
+        with monkeypatch.context() as m:
+            m.setattr(lm, name, mutant)
+            try:
+                for w in [1, 2, 3, 5, 8]:
+                    test_valid_rejects_every_other_cache(w)
+                test_position_invariant_rejects_non_consecutive()
+            except AssertionError:
+                caught.append(mutant.__name__)
+    assert caught == [f.__name__ for _, f in mutants]
