@@ -309,7 +309,7 @@ def run_ours(args, rank, world, local_rank):
         dist = td
 
     K, Wm = args.steps, args.warmup
-    total_steps = Wm + K + Wm + K + 4
+    total_steps = Wm + K + K + K + 6
     wl = Workload(rank, total_steps)
     # warm-up (eager), also loads every kernel
     for i in range(Wm):
@@ -380,8 +380,10 @@ def run_ours(args, rank, world, local_rank):
     # Each step's inputs sit in one pinned host record [q | k | v] and cross
     # to the device in one copy; the call gets views of the device copy, and
     # its output is read back into pinned host memory, all on one stream.
-    # (Moving the copies to a second stream, double-buffered, measured slower:
-    # the extra event calls per step make the host loop the bottleneck.)
+    # The K steps -- upload, ps_decode_step, read-back, each step -- are
+    # captured into one CUDA graph and replayed, as a serving loop would run
+    # them; the same steps issued eagerly from Python are reported beside it
+    # (there the host's issue path, not the device, sets the pace).
     nq, nk = B * HQ * D, B * HKV * D
     hin = [torch.cat([wl.q_pool[r].reshape(wl.visits, -1), wl.k_pool[r].reshape(wl.visits, -1),
                       wl.v_pool[r].reshape(wl.visits, -1)], dim=1).cpu().pin_memory()
@@ -392,29 +394,51 @@ def run_ours(args, rank, world, local_rank):
     dk = din[nq:nq + nk].view(B, HKV, D)
     dv = din[nq + nk:].view(B, HKV, D)
 
-    def e2e_step(i):
+    def e2e_step(i, stream=None):
         r = i % ROT
         v = wl.visit[r]
         din.copy_(hin[r][v], non_blocking=True)
-        out = wl.step(i, host=lambda r_, v_: (dk, dv, dq))
+        out = wl.step(i, stream, host=lambda r_, v_: (dk, dv, dq))
         hout.copy_(out, non_blocking=True)
 
     base = Wm + K
     for i in range(2):
         e2e_step(base + i)
     torch.cuda.synchronize()
+    base += 2
+    s2 = torch.cuda.Stream()
+    s2.wait_stream(torch.cuda.current_stream())
+    g2 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g2, stream=s2):
+        for i in range(K):
+            e2e_step(base + i, s2)
+    torch.cuda.synchronize()
+    upload_graph(torch, g2, s2)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s2):
+        e0.record(s2)
+        g2.replay()
+        e1.record(s2)
+    torch.cuda.synchronize()
+    del g2
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1), dist, "cuda")
+    _check_device(wl)
+    e2e_value = job_tokens_per_s(world, K, ms_e2e)
+    base += K
+    # the same steps issued eagerly, one Python call after another
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     e0.record()
     for i in range(K):
-        e2e_step(base + 2 + i)
+        e2e_step(base + i)
     e1.record()
     torch.cuda.synchronize()
-    ms_e2e = e0.elapsed_time(e1)
-    ms_e2e = max_over_ranks(ms_e2e, dist, "cuda")
+    ms_eager = max_over_ranks(e0.elapsed_time(e1), dist, "cuda")
     _check_device(wl)
-    e2e_value = job_tokens_per_s(world, K, ms_e2e)
+    e2e_eager = job_tokens_per_s(world, K, ms_eager)
     h2d = (B * HKV * D * 2) * 2 + B * HQ * D * 2
     d2h = B * HQ * D * 2
 
@@ -455,7 +479,11 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "copies": "one upload of a pinned [q | k | v] record and one read-back of the "
-                          "output per step, on the decode stream"},
+                          "output per step, on the decode stream",
+                "issue": "the K steps (upload, ps_decode_step, read-back) captured into one "
+                         "CUDA graph and replayed",
+                "eager": {"value": round(e2e_eager, 1), "unit": UNIT,
+                          "issue": "the same steps issued one by one from Python"}},
         "gpu_launches": 2 * K,  # per step: the decode-step stream launch and the pair merge
         "clocks": clk,
         "cpu_baseline": cpu,
@@ -936,13 +964,25 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--only", choices=["prefill", "prompt", "ragged", "shared", "paged", "t_sweep"],
+                    help="run one side measurement alone and print its record (for profiling "
+                         "one kernel under ncu); not a benchmark line")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.impl == "reference":
+    if args.only:
+        import torch
+        torch.cuda.set_device(local_rank)
+        k = max(3, min(args.steps, 10))
+        fn = {"prefill": prefill_measure, "ragged": ragged_measure,
+              "shared": shared_prefix_measure, "paged": paged_measure,
+              "t_sweep": lambda n: t_sweep_measure(max(n, 16)),
+              "prompt": lambda n: prompt_measure(n, load_bf16_peak()[0])}[args.only]
+        print(json.dumps({"only": args.only, "result": fn(k)}), flush=True)
+    elif args.impl == "reference":
         run_reference(args, rank, world)
     else:
         run_ours(args, rank, world, local_rank)

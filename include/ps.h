@@ -76,7 +76,12 @@ typedef struct {
 
 /* Bytes of device memory a cache with these parameters needs (0 if invalid).
  * W >= 1 window slots, P_max >= 0 prefix rows, Hkv >= 1 key/value heads,
- * d in {64, 128}, dtype a ps_dtype, max_seqs >= 1 sequences. */
+ * d in {64, 128}, dtype a ps_dtype, max_seqs >= 1 sequences.  The K/V part is
+ * the blog's section 1.1 size formula for one layer with the sequence length
+ * bounded by the pinned prefix plus the window:
+ * 2 * Hkv * d * (P_max + W) * max_seqs * sizeof(dtype), plus the per-slot
+ * positions (8 bytes per ring slot) and 32 bytes of bookkeeping per sequence,
+ * each region rounded up to 256 bytes. */
 PS_API size_t ps_cache_bytes(int W, int P_max, int Hkv, int d, int dtype, int max_seqs);
 
 /* Bind a cache to the caller's device buffer `dev_buf` (dev_bytes >=
@@ -231,10 +236,15 @@ PS_API int ps_decode_step(ps_cache* c, const void* q, const void* k_new, const v
  * split-K scratch lives in a fixed 4 MiB array inside the library's device
  * image (held by every GPU that loads the library until the process exits).
  * It allocates nothing.  A batch whose scratch would exceed 4 MiB is rejected
- * with PS_ENOMEM.  The first call on each device looks up the array's address
- * and zero-fills it, which synchronises that device: make that first call
- * before any stream capture.  All calls on a device share the array, so calls
- * that overlap on the GPU (other streams, other threads) race; order them. */
+ * with PS_ENOMEM.  Arguments and sequence states are checked first, as by
+ * ps_attend_decode; B = 0 returns PS_OK with nothing set up or enqueued.  The
+ * first call on each device (and the first after that device's context was
+ * reset) looks up the array's device address; the look-up does not
+ * synchronise, but it may make the runtime load the library's device code, so
+ * make that first call before any stream capture.  Nothing in the array has
+ * to start at zero: every call writes the scratch it reads.  All calls on a
+ * device share the array, so calls that overlap on the GPU (other streams,
+ * other threads) race; order them. */
 PS_API int ps_attend_decode_static(ps_cache* c, const void* q, const int* seq_ids,
                                    const int64_t* t, int B, int Hq, float scale, void* out,
                                    void* stream);
@@ -246,7 +256,11 @@ PS_API int ps_attend_decode_static(ps_cache* c, const void* q, const int* seq_id
  * and t0 >= P_s.  q: [n][Hq][d]; k_blk, v_blk: [n][Hkv][d], the block's own
  * keys/values; out: [n][Hq][d] (all device).  Query t0+i sees the prefix, the
  * ring entries in its window and block tokens t0..t0+i (causal inside the
- * block).  The ring must still hold [max(P_s, t0-W+1), t0-1], which is always
+ * block): the digest's section 03 visibility rule applied to every query of
+ * the block, evaluated as in its section 06 kernel -- key tiles walked over
+ * the prefix range and the window range separately (the evicted middle is
+ * never loaded) with an element mask only on tiles that straddle a window or
+ * causal edge.  The ring must still hold [max(P_s, t0-W+1), t0-1], which is always
  * true before the block is appended.  If append_after != 0 the block is then
  * appended as by ps_append_kv (only its last W tokens survive in the ring).
  * bf16 with d = 128 and Hq/Hkv in {1, 2, 4, 8} runs on the tcgen05 tensor-core

@@ -42,6 +42,8 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
     if not force and not _stale():
         return LIB
     nvcc = os.environ.get("NVCC", "nvcc")
+    # PS_NVCC_EXTRA: extra nvcc flags, e.g. tile-shape macros (-DPS_DMMA_STAGES=4)
+    extra = list(extra or []) + os.environ.get("PS_NVCC_EXTRA", "").split()
     objs = []
     os.makedirs(os.path.join(HERE, "_build"), exist_ok=True)
     for src in sources():

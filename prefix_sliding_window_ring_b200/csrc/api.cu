@@ -102,6 +102,7 @@ struct ps_cache {
   int device;
   int sm_count;
   ps::CacheDev dev;
+  ps::DecodeMaps dmaps;  // bf16 caches: tensor maps of K/V for the decode kernel
   std::vector<SeqHost> seqs;
 };
 
@@ -346,6 +347,10 @@ int create_cache(int W, int P_max, int Hkv, int d, int dtype, int max_seqs, int 
   c->dev.pstride = paged ? P_max : (int64_t)P_max + W;
   c->dev.rstride = paged ? page_rows : (int64_t)P_max + W;
   c->dev.rbase = paged ? (int64_t)max_seqs * Hkv * P_max : P_max;
+  if (dtype == PS_BF16 && !ps::make_decode_maps(c->dev, &c->dmaps)) {
+    delete c;
+    return fail(PS_ECUDA, "tensor-map encoding of the cache's K/V failed");
+  }
   SeqHost empty{0, 0, 0, 0, 0};
   if (paged) {
     empty.pages.assign(c->dev.npg, -1);
@@ -519,32 +524,16 @@ size_t ps_decode_workspace_bytes(const ps_cache* c, int B, int Hq) {
 int ps_attend_decode(ps_cache* c, const void* q, const int* seq_ids, const int64_t* t, int B,
                      int Hq, float scale, void* out, void* workspace, size_t workspace_bytes,
                      void* stream) {
-  if (!c) return fail(PS_EINVAL, "cache is NULL");
-  if (B < 0) return fail(PS_EINVAL, "negative B=%d", B);
   int G = 0;
-  int r = check_group(c, Hq, &G);
+  int r = ps::check_decode_call(c, q, seq_ids, t, B, Hq, out, &G);
   if (r) return r;
   if (B == 0) return ok();
-  if ((r = check_batch(c, seq_ids, B))) return r;
-  if (!t) return fail(PS_EINVAL, "t is NULL");
-  for (int b = 0; b < B; ++b) {
-    const SeqHost& s = c->seqs[seq_ids[b]];
-    if (t[b] != s.next_pos - 1)
-      return fail(PS_EPOS, "sequence %d: t=%lld is not the last appended position %lld",
-                  seq_ids[b], (long long)t[b], (long long)(s.next_pos - 1));
-    if (t[b] < s.P)
-      return fail(PS_EPOS, "sequence %d: t=%lld lies inside the prefix (P=%d); append first",
-                  seq_ids[b], (long long)t[b], s.P);
-  }
-  if (!q || !out || !aligned16(q) || !aligned16(out))
-    return fail(PS_EINVAL, "q/out must be non-NULL 16-byte aligned device pointers");
   if (!workspace || ((uintptr_t)workspace & 255))
     return fail(PS_EINVAL, "workspace must be a non-NULL 256-byte aligned device pointer");
   size_t need = 0;
   ps::DecodeWs ws = ps::decode_ws_layout(workspace, B, c->Hkv, G, c->d, c->sm_count, &need);
   if (need > workspace_bytes)
     return fail(PS_ENOMEM, "workspace holds %zu bytes, this call needs %zu", workspace_bytes, need);
-  if ((r = check_device(c))) return r;
   cudaStream_t st = (cudaStream_t)stream;
   size_t per_entry = (size_t)Hq * c->d * c->esize;
   for (int b0 = 0; b0 < B; b0 += ps::kMaxBatchPerLaunch) {
@@ -562,7 +551,7 @@ int ps_attend_decode(ps_cache* c, const void* q, const int* seq_ids, const int64
     }
     PS_CUDA(ps::launch_decode(c->dev, c->dtype, G, ids, nb, Hq, (const char*)q + b0 * per_entry,
                               nullptr, nullptr, (char*)out + b0 * per_entry, scale, ws,
-                              c->sm_count, st));
+                              c->sm_count, c->dtype == PS_BF16 ? &c->dmaps : nullptr, st));
   }
   return ok();
 }
@@ -627,7 +616,8 @@ int ps_decode_step(ps_cache* c, const void* q, const void* k_new, const void* v_
     }
     PS_CUDA(ps::launch_decode(c->dev, c->dtype, G, ids, nb, Hq, (const char*)q + b0 * per_entry,
                               (const char*)k_new + b0 * per_row, (const char*)v_new + b0 * per_row,
-                              (char*)out + b0 * per_entry, scale, ws, c->sm_count, st));
+                              (char*)out + b0 * per_entry, scale, ws, c->sm_count,
+                              c->dtype == PS_BF16 ? &c->dmaps : nullptr, st));
   }
   c->free_pages = avail;
   for (int b = 0; b < B; ++b) {
@@ -763,6 +753,29 @@ int set_error(int code, const char* fmt, ...) {
   va_end(ap);
   g_err = buf;
   return code;
+}
+
+int check_decode_call(ps_cache* c, const void* q, const int* seq_ids, const int64_t* t, int B,
+                      int Hq, const void* out, int* G) {
+  if (!c) return fail(PS_EINVAL, "cache is NULL");
+  if (B < 0) return fail(PS_EINVAL, "negative B=%d", B);
+  int r = check_group(c, Hq, G);
+  if (r) return r;
+  if (B == 0) return PS_OK;
+  if ((r = check_batch(c, seq_ids, B))) return r;
+  if (!t) return fail(PS_EINVAL, "t is NULL");
+  for (int b = 0; b < B; ++b) {
+    const SeqHost& s = c->seqs[seq_ids[b]];
+    if (t[b] != s.next_pos - 1)
+      return fail(PS_EPOS, "sequence %d: t=%lld is not the last appended position %lld",
+                  seq_ids[b], (long long)t[b], (long long)(s.next_pos - 1));
+    if (t[b] < s.P)
+      return fail(PS_EPOS, "sequence %d: t=%lld lies inside the prefix (P=%d); append first",
+                  seq_ids[b], (long long)t[b], s.P);
+  }
+  if (!q || !out || !aligned16(q) || !aligned16(out))
+    return fail(PS_EINVAL, "q/out must be non-NULL 16-byte aligned device pointers");
+  return check_device(c);
 }
 
 int cache_hkv(const ps_cache* c) { return c->Hkv; }

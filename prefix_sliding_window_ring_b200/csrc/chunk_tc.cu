@@ -31,13 +31,10 @@
 //            finally normalise O into the output.
 // Every wait is bounded: a time-out sets ERR_TIMEOUT, every role stops, the
 // MMA issuer waits for its issued work and the TMEM is freed.
-#include <cuda.h>
-#include <cudaTypedefs.h>
 #include <math.h>
 #include <string.h>
 
 #include <atomic>
-#include <mutex>
 
 #include "chunk_sched.cuh"
 #include "internal.h"
@@ -426,35 +423,6 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
   }
 }
 
-// ------------------------------------------------------------ tensor maps --
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
-  });
-  return fn;
-}
-
-// 3-D bf16 map, dims innermost first, byte strides of dims 1 and 2, 128B swizzle.
-bool map3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
-           uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[3] = {d0, d1, d2};
-  cuuint64_t strides[2] = {s1, s2};
-  cuuint32_t box[3] = {b0, b1, b2};
-  cuuint32_t es[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
-            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 bool chunk_tc_supported(const CacheDev& c, int dtype, int d, int G) {
@@ -489,24 +457,24 @@ cudaError_t launch_chunk_tc(const CacheDev& c, int G, const ChunkEntry* e, int n
     N += e[b].n;
   }
   if (N > INT32_MAX) return cudaErrorInvalidValue;
-  bool ok = map3d(&a.qmap, q, kHD, Hq, N, row, (uint64_t)Hq * row, 64, 1, PT);
+  bool ok = encode_map3d_bf16(&a.qmap, q, kHD, Hq, N, row, (uint64_t)Hq * row, 64, 1, PT);
   // prefix rows: [S*Hkv][pstride] rows from the buffer start; ring pages:
   // [nphys*Hkv][page_rows] slabs rstride rows apart from row rbase
   const uint64_t prows = c.pstride > 0 ? (uint64_t)c.pstride : 1;
   const char* kring = (const char*)c.K + (size_t)c.rbase * row;
   const char* vring = (const char*)c.V + (size_t)c.rbase * row;
-  ok = ok && map3d(&a.kpre, c.K, kHD, prows, (uint64_t)c.S * c.Hkv, row, prows * row, 64, kBN, 1);
-  ok = ok && map3d(&a.vpre, c.V, kHD, prows, (uint64_t)c.S * c.Hkv, row, prows * row, 64, kBN, 1);
-  ok = ok && map3d(&a.kring, kring, kHD, (uint64_t)c.page_rows, (uint64_t)c.nphys * c.Hkv, row,
+  ok = ok && encode_map3d_bf16(&a.kpre, c.K, kHD, prows, (uint64_t)c.S * c.Hkv, row, prows * row, 64, kBN, 1);
+  ok = ok && encode_map3d_bf16(&a.vpre, c.V, kHD, prows, (uint64_t)c.S * c.Hkv, row, prows * row, 64, kBN, 1);
+  ok = ok && encode_map3d_bf16(&a.kring, kring, kHD, (uint64_t)c.page_rows, (uint64_t)c.nphys * c.Hkv, row,
                    (uint64_t)c.rstride * row, 64, kBN, 1);
-  ok = ok && map3d(&a.vring, vring, kHD, (uint64_t)c.page_rows, (uint64_t)c.nphys * c.Hkv, row,
+  ok = ok && encode_map3d_bf16(&a.vring, vring, kHD, (uint64_t)c.page_rows, (uint64_t)c.nphys * c.Hkv, row,
                    (uint64_t)c.rstride * row, 64, kBN, 1);
   // a prompt launch loads no block rows; its block maps describe the cache
   // K/V (never used) so that every map is well formed
   const uint64_t nblk = prompt ? prows : (uint64_t)N;
-  ok = ok && map3d(&a.kblk, prompt ? c.K : k_blk, kHD, c.Hkv, nblk, row, (uint64_t)c.Hkv * row, 64,
+  ok = ok && encode_map3d_bf16(&a.kblk, prompt ? c.K : k_blk, kHD, c.Hkv, nblk, row, (uint64_t)c.Hkv * row, 64,
                    1, kBN);
-  ok = ok && map3d(&a.vblk, prompt ? c.V : v_blk, kHD, c.Hkv, nblk, row, (uint64_t)c.Hkv * row, 64,
+  ok = ok && encode_map3d_bf16(&a.vblk, prompt ? c.V : v_blk, kHD, c.Hkv, nblk, row, (uint64_t)c.Hkv * row, 64,
                    1, kBN);
   if (!ok) return cudaErrorInvalidValue;
   a.c = c;

@@ -1,0 +1,886 @@
+// Decode attention for bfloat16 caches (head_dim 64 or 128) with the per-row
+// products on the tensor cores, and the decode step that appends the token in
+// the same pass.
+//
+// Why tensor cores for a bandwidth-bound kernel.  Per visible K/V row a
+// decode query does 2 G d multiply-adds for its G query heads.  Done on the
+// CUDA cores (one lane per 16 bytes of a row, shuffle reductions for the
+// scores) that costs about 50 warp instructions per row, which caps an SM at
+// about the copy bandwidth and leaves no slack to absorb the pipeline's start
+// and end.  As warp-level MMAs the same work is about 4 warp instructions per
+// row, so HBM is the only bound.  The products themselves are negligible
+// (G <= 8 heads padded to the MMA's 8 columns).
+//
+// Work division (as in the CUDA-core kernel): each (batch entry, kv head)
+// pair's visible rows are cut into tiles of kTR rows, the tiles of all pairs
+// are laid end to end and CTA c streams the tiles [T c / NC, T (c + 1) / NC);
+// every (CTA range, pair) piece emits one partial, merged by k_decode_merge.
+// The tile layout (decode_pack.cuh) places every row at the offset within its
+// 8-row atom that its row or slot has modulo 8, so that whole atoms can be
+// loaded by tensor-map copies; no atom holds rows of two pieces.
+//
+// Streaming.  One lane of warp kMW is the producer: per tile it issues
+// tensor-map copies (cp.async.bulk.tensor, 128-byte swizzle, no multicast) of
+// the atoms holding each piece's K and V rows -- 64-row boxes, then 8-row
+// boxes for the rest -- into a kStages-deep ring of shared-memory stages; the
+// pair's q rows come with the first tile of a piece and the appended token of
+// a decode step by plain bulk copies.  Rows a box reads before or after its
+// piece are masked.
+// No evicted row is a valid row of any tile ("Prefix Sliding" digest, section
+// 06: the prefix and the window are walked separately).
+//
+// Consumers (kMW warps).  Warp w takes the 16-row groups w, w + kMW, ... of
+// every tile and keeps its own online-softmax state for its rows:
+//   S^T (16 rows x 8 heads) = K (16 x d) Q^T (d x 8)   m16n8k16 bf16 MMAs,
+//       K fragments by ldmatrix from the swizzled tile, Q^T (heads beyond G
+//       zero) in registers;
+//   per head a running max raised lazily (only when a score passes it by more
+//       than 2^8, so the accumulators are rescaled on few groups; a warp vote
+//       decides, the rare raise takes a shuffle maximum over the 16 rows);
+//   weights p = 2^(s - max) rounded to bfloat16 and transposed in registers
+//       (movmatrix) into the B fragment of
+//   O^T (d x 8) += V^T (d x 16 rows) P^T (16 rows x 8)   with V^T fragments
+//       by transposing ldmatrix.
+// Rows of a group that are not valid get score -inf and their V rows in
+// shared memory are zeroed first, so nothing outside the visible set reaches
+// the accumulators.  At the end of a piece the warps' states are merged
+// through shared memory into the piece's partial.
+//
+// Every wait is bounded; a time-out stops the CTA, sets ERR_TIMEOUT and lets
+// the copies already issued land before the CTA exits.
+#include <math.h>
+#include <string.h>
+
+#include <atomic>
+
+#include "decode_common.cuh"
+#include "decode_pack.cuh"
+#include "internal.h"
+#include "sm100_ptx.cuh"
+
+#ifndef PS_DMMA_TR
+#define PS_DMMA_TR 64
+#endif
+#ifndef PS_DMMA_STAGES
+#define PS_DMMA_STAGES 3
+#endif
+#ifndef PS_DMMA_CTAS_PER_SM
+#define PS_DMMA_CTAS_PER_SM 2
+#endif
+#ifndef PS_DMMA_L2_PROMOTION
+#define PS_DMMA_L2_PROMOTION 2
+#endif
+#ifndef PS_DMMA_PREFETCH_TILES
+#define PS_DMMA_PREFETCH_TILES 4
+#endif
+
+namespace ps {
+
+namespace {
+
+using namespace dec;
+
+constexpr int kMW = 4;                      // consumer warps
+constexpr int kThreadsM = (kMW + 1) * 32;   // plus one producer warp
+constexpr int kTR = PS_DMMA_TR;             // rows per tile
+constexpr int kStagesM = PS_DMMA_STAGES;
+constexpr int kGroups = kTR / 16;           // 16-row MMA groups per tile
+constexpr int kBox = 64;                    // rows of the large tensor-map box
+constexpr int kMaxCluster = 8;              // CTAs per pair in cluster mode, at most
+static_assert(kTR == 64, "tile rows: 64 (the valid-row mask is one 64-bit word)");
+static_assert(PS_DMMA_CTAS_PER_SM <= kDecMaxCtasPerSm, "workspace slots cover every CTA");
+
+struct MmaDecodeArgs {
+  DecodeMaps maps;  // first: tensor maps must be 64-byte aligned
+  DecodeArgs a;
+};
+static_assert(sizeof(MmaDecodeArgs) <= 32764, "decode arguments fit the kernel parameter space");
+
+struct TileDescM {
+  uint32_t mask[kTR / 32];  // valid rows: bit r % 32 of word r / 32
+  int32_t pair, flags;
+  int32_t slot;             // partial-result slot of the piece: CTA range + pair
+  int32_t new_row;          // TD_NEW: tile row of the appended token
+};
+
+// ------------------------------------------------------------- warp MMA --
+__device__ __forceinline__ void ldsm4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+__device__ __forceinline__ void ldsm4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+// d += a b, m16n8k16, bf16 inputs, f32 accumulators (row-major A, column-major B)
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t movm_t(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Online-softmax state of one consumer lane: lane (g, t) holds, for the
+// query heads 2t and 2t+1, the running max m (log2 units; +inf for a padding
+// head, which then gets weight 0), its partial sum l over the rows it has
+// seen, and O^T rows d = 16 mt + g and 16 mt + g + 8 of both heads.
+template <int D, int G>
+struct MmaState {
+  static constexpr int KS = D / 16;  // k-steps of S^T, m-tiles of O^T
+  uint32_t qf[KS][2];                // Q^T fragments
+  float o[KS][4];
+  float m[2], l[2];
+
+  __device__ __forceinline__ void init(const uint8_t* qs) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      // heads g >= G are padding: zero columns of Q^T (their q rows are not loaded)
+      const uint8_t* row = qs + (size_t)(g < G ? g : 0) * D * 2 + (size_t)(16 * ks + 2 * t) * 2;
+      const uint32_t lo = *(const uint32_t*)row, hi = *(const uint32_t*)(row + 16);
+      qf[ks][0] = g < G ? lo : 0u;
+      qf[ks][1] = g < G ? hi : 0u;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[ks][e] = 0.f;
+    }
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      m[hh] = 2 * t + hh < G ? -INFINITY : INFINITY;
+      l[hh] = 0.f;
+    }
+  }
+};
+
+// CL: cluster mode.  Pair p is streamed by the csize CTAs of cluster p, CTA
+// rank r taking an equal share of its padded rows (dec_cluster_share); each CTA
+// publishes its merged state in its own shared memory, and rank 0 reads its
+// peers' states through distributed shared memory, writes the pair's output
+// and (decode step) commits the sequence's bookkeeping -- no partials in global
+// memory, no second grid.  Otherwise the flattened split with k_decode_merge.
+template <int D, int G, bool CL>
+__global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
+    k_decode_mma(const __grid_constant__ MmaDecodeArgs ma) {
+  constexpr int HALVES = D / 64;                       // 128-byte column blocks of a row
+  constexpr uint32_t kHalfBytes = kTR * 128;           // one column block of a tile
+  constexpr uint32_t kTileBytes = HALVES * kHalfBytes; // K (or V) of one tile
+  constexpr int KS = D / 16;
+  const DecodeArgs& a = ma.a;
+  extern __shared__ uint8_t dsm_raw[];
+  uint8_t* const kbuf = (uint8_t*)(((uintptr_t)dsm_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* const vbuf = kbuf + kStagesM * kTileBytes;
+  uint8_t* const qbuf = vbuf + kStagesM * kTileBytes;  // [kStagesM][G][D] bf16
+  __shared__ __align__(8) uint64_t full[kStagesM], empty[kStagesM];
+  __shared__ __align__(8) uint64_t sync_a, sync_b, sync_c;
+  __shared__ __align__(8) uint64_t pub_bar, done_bar;  // cluster: peers published / rank 0 done
+  __shared__ TileDescM desc[kStagesM];
+  __shared__ int abort_flag;
+  __shared__ MergeSmem<G, D, kMW> sm;
+  __shared__ float pub_ml[G][2];  // cluster: this CTA's merged (max, sum) per head
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int Hkv = a.c.Hkv;
+  const int64_t R = a.total, NC = a.nctas;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStagesM; ++i) {
+      ptx::mbar_init(&full[i], 1);
+      ptx::mbar_init(&empty[i], kMW);
+    }
+    ptx::mbar_init(&sync_a, kMW);
+    ptx::mbar_init(&sync_b, kMW);
+    ptx::mbar_init(&sync_c, kMW);
+    ptx::mbar_init(&pub_bar, CL ? a.csize - 1 : 1);
+    ptx::mbar_init(&done_bar, 1);
+    abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == kMW && lane == 0) {
+    // fetch the tensor maps' descriptors while the previous grid drains
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      ptx::prefetch_tmap(&ma.maps.kpre[k]);
+      ptx::prefetch_tmap(&ma.maps.vpre[k]);
+      ptx::prefetch_tmap(&ma.maps.kring[k]);
+      ptx::prefetch_tmap(&ma.maps.vring[k]);
+    }
+  }
+  __syncthreads();
+  // every CTA of the cluster has initialised its barriers before any remote arrive
+  if (CL) ptx::cluster_sync_all();
+  // Programmatic dependent launch: the next grid may be scheduled.  Only the
+  // producer waits for the previous grid (griddepcontrol.wait), just before its
+  // first copy: everything the consumers read or write in global memory comes
+  // after a tile that the producer issued after that wait, and the setup of
+  // the first piece overlaps the previous grid's tail.
+  ptx::pdl_launch_dependents();
+
+  if (warp == kMW) {
+    if (lane != 0) return;
+    // ------------------------------------------------------------ producer --
+    const bool step = a.knew != nullptr;
+    const int32_t page = a.c.page_table ? a.c.page_rows : 0;
+    int i = 0;  // tiles handed out so far
+    bool alive = true;
+    bool waited = false;  // griddepcontrol.wait done
+    auto wait_primary = [&]() {
+      if (!waited) {
+        ptx::pdl_wait_primary();
+        waited = true;
+      }
+    };
+    // One piece of pair (b, g): its tiles [j0, j1) (flattened split, tph
+    // tiles in all), or with rank >= 0 the cluster share of CTA `rank`.
+    // check: compare the device record with the launch's state (flattened
+    // split; in cluster mode rank 0 of kv head 0 does it at the end).
+    auto piece = [&](int b, int g, int32_t tph, int32_t j0, int32_t j1, int rank, bool check) {
+      const int s = a.seq[b];
+      DevMeta m;
+      m.next_pos = a.t[b] + 1;
+      m.P = a.P[b];
+      m.head = a.head[b];
+      m.count = a.count[b];
+      m.owner = a.owner[b];
+      const DecRuns runs = dec_runs(m, a.c.W, a.t[b], page, step);
+      bool bad = runs.rows != m.P + m.count || (rank < 0 && dec_tiles(runs, kTR) != tph);
+      const int pair = b * Hkv + g;
+      const int zpre = m.owner * Hkv + g;
+      // padded rows [xs, xe) of this piece, in tiles of kTR rows (the last may be short)
+      int32_t xs, xe;
+      if (rank >= 0) {
+        dec_cluster_share(runs, rank, a.csize, &xs, &xe);
+      } else {
+        xs = j0 * kTR;
+        xe = min(j1 * kTR, runs.padded);
+      }
+      const int32_t nt = xe > xs ? (xe - xs + kTR - 1) / kTR : 0;
+      // Before the previous grid has completed: bring this CTA's first whole
+      // tiles into L2, so that DRAM works during the previous grid's tail and
+      // the copies after the wait hit L2.  (Only the cache is touched; the
+      // copies themselves still come after griddepcontrol.wait.)
+      if (!waited) {
+        for (int32_t k = 0; k < nt && k < PS_DMMA_PREFETCH_TILES; ++k) {
+          const int32_t x0 = xs + k * kTR, x1 = min(x0 + kTR, xe);
+          int32_t wsrc, wrow;
+          if (!dec_range_whole(runs, kTR, x0, x1, &wsrc, &wrow)) continue;
+          const bool pre = wsrc == RUN_PREFIX;
+          if (!pre && page) continue;  // a page-table read would have to wait
+          const int32_t z = pre ? zpre : s * Hkv + g;
+          if (HALVES == 2 && ma.maps.whole) {
+            ptx::tma_prefetch_l2_4d(pre ? &ma.maps.kpre_w : &ma.maps.kring_w, 0, wrow, 0, z);
+            ptx::tma_prefetch_l2_4d(pre ? &ma.maps.vpre_w : &ma.maps.vring_w, 0, wrow, 0, z);
+          } else {
+            ptx::tma_prefetch_l2_3d(pre ? &ma.maps.kpre[0] : &ma.maps.kring[0], 0, wrow, z);
+            ptx::tma_prefetch_l2_3d(pre ? &ma.maps.vpre[0] : &ma.maps.vring[0], 0, wrow, z);
+          }
+        }
+      }
+      for (int32_t k = 0; k < nt && alive; ++k) {
+        const int32_t x0 = xs + k * kTR, x1 = min(x0 + kTR, xe);
+        const int st = i % kStagesM;
+        if (i >= kStagesM && !ptx::mbar_wait_bounded(&empty[st], ((i / kStagesM) - 1) & 1,
+                                                      &abort_flag, kWaitLimitCycles)) {
+          alive = false;
+          break;
+        }
+        wait_primary();
+        uint8_t* const kd = kbuf + (size_t)st * kTileBytes;
+        uint8_t* const vd = vbuf + (size_t)st * kTileBytes;
+        const int32_t flags0 = (k == 0 ? TD_FIRST : 0) | (k == nt - 1 ? TD_LAST : 0);
+        int32_t wsrc, wrow;
+        if (dec_range_whole(runs, kTR, x0, x1, &wsrc, &wrow)) {
+          // the common case: the tile is kTR rows of one run, copied whole
+          desc[st].mask[0] = 0xffffffffu;
+          desc[st].mask[1] = 0xffffffffu;
+          desc[st].pair = pair;
+          desc[st].flags = flags0;
+          desc[st].slot = (int32_t)blockIdx.x + pair;
+          desc[st].new_row = -1;
+          ptx::mbar_arrive_expect_tx(
+              &full[st], 2u * kTR * D * 2u + ((flags0 & TD_FIRST) ? (uint32_t)(G * D * 2) : 0u));
+          if (flags0 & TD_FIRST)
+            ptx::bulk_g2s(qbuf + (size_t)st * G * D * 2,
+                          (const uint16_t*)a.q + ((size_t)b * a.Hq + (size_t)g * G) * D,
+                          (uint32_t)(G * D * 2), &full[st]);
+          const bool pre = wsrc == RUN_PREFIX;
+          const int32_t y = pre ? wrow : (page ? wrow % page : wrow);
+          const int32_t z = pre ? zpre : ring_page(a.c, s, wrow) * Hkv + g;
+          if (HALVES == 2 && ma.maps.whole) {
+            ptx::tma_load_4d(kd, pre ? &ma.maps.kpre_w : &ma.maps.kring_w, 0, y, 0, z, &full[st]);
+            ptx::tma_load_4d(vd, pre ? &ma.maps.vpre_w : &ma.maps.vring_w, 0, y, 0, z, &full[st]);
+          } else {
+#pragma unroll
+            for (int h = 0; h < HALVES; ++h) {
+              ptx::tma_load_3d(kd + h * kHalfBytes, pre ? &ma.maps.kpre[0] : &ma.maps.kring[0],
+                               h * 64, y, z, &full[st]);
+              ptx::tma_load_3d(vd + h * kHalfBytes, pre ? &ma.maps.vpre[0] : &ma.maps.vring[0],
+                               h * 64, y, z, &full[st]);
+            }
+          }
+          ++i;
+          continue;
+        }
+        uint64_t mask = 0;  // valid tile rows
+        int32_t flags = flags0;
+        int32_t new_row = -1;
+        uint32_t bytes = (flags & TD_FIRST) ? (uint32_t)(G * D * 2) : 0u;
+        dec_range_pieces(runs, x0, x1, [&](int32_t src, int32_t, int32_t sr, int32_t n) {
+          mask |= (n >= 64 ? ~0ull : ((1ull << n) - 1ull)) << sr;
+          if (src == RUN_NEW) {
+            flags |= TD_NEW;
+            new_row = sr;
+            bytes += 2u * D * 2u;
+          } else {  // whole atoms from the one holding the piece's first row
+            const int32_t nb = (sr & (kPadRows - 1)) + n;
+            const int32_t boxed = (nb / kBox) * kBox + pad8(nb % kBox);
+            bytes += 2u * (uint32_t)boxed * D * 2u;
+          }
+        });
+        desc[st].mask[0] = (uint32_t)mask;
+        desc[st].mask[1] = (uint32_t)(mask >> 32);
+        desc[st].pair = pair;
+        desc[st].flags = flags;
+        desc[st].slot = (int32_t)blockIdx.x + pair;
+        desc[st].new_row = new_row;
+        ptx::mbar_arrive_expect_tx(&full[st], bytes);
+        if (flags & TD_FIRST)
+          ptx::bulk_g2s(qbuf + (size_t)st * G * D * 2,
+                        (const uint16_t*)a.q + ((size_t)b * a.Hq + (size_t)g * G) * D,
+                        (uint32_t)(G * D * 2), &full[st]);
+        dec_range_pieces(runs, x0, x1, [&](int32_t src, int32_t row, int32_t sr, int32_t n) {
+          if (src == RUN_NEW) {  // the appended token, straight from the caller's rows
+            const uint16_t* kn = (const uint16_t*)a.knew + (size_t)pair * D;
+            const uint16_t* vn = (const uint16_t*)a.vnew + (size_t)pair * D;
+#pragma unroll
+            for (int h = 0; h < HALVES; ++h) {  // row sr % 8 == 0: the swizzle is the identity
+              ptx::bulk_g2s(kd + h * kHalfBytes + sr * 128, kn + h * 64, 128u, &full[st]);
+              ptx::bulk_g2s(vd + h * kHalfBytes + sr * 128, vn + h * 64, 128u, &full[st]);
+            }
+            return;
+          }
+          const CUtensorMap* km = src == RUN_PREFIX ? ma.maps.kpre : ma.maps.kring;
+          const CUtensorMap* vm = src == RUN_PREFIX ? ma.maps.vpre : ma.maps.vring;
+          int32_t y, z;
+          if (src == RUN_PREFIX) {
+            y = row;
+            z = zpre;
+          } else {  // a ring piece lies within one page
+            y = page ? row % page : row;
+            z = ring_page(a.c, s, row) * Hkv + g;
+          }
+          // copy whole atoms, from the one that holds the piece's first row
+          // (its row or slot minus the offset within the atom: same page)
+          const int32_t lead = sr & (kPadRows - 1);
+          sr -= lead;
+          y -= lead;
+          n += lead;
+          while (n > 0) {
+            const bool big = n >= kBox;
+            const int32_t rows = big ? kBox : kPadRows;
+#pragma unroll
+            for (int h = 0; h < HALVES; ++h) {
+              ptx::tma_load_3d(kd + h * kHalfBytes + sr * 128, big ? &km[0] : &km[1], h * 64, y, z,
+                               &full[st]);
+              ptx::tma_load_3d(vd + h * kHalfBytes + sr * 128, big ? &vm[0] : &vm[1], h * 64, y, z,
+                               &full[st]);
+            }
+            sr += rows;
+            y += rows;
+            n -= rows;
+          }
+        });
+        ++i;
+      }
+      if (check) {
+        const DevMeta md = a.c.meta[s];
+        DevMeta me = md;  // the device record before this launch (a step advances it by one)
+        if (step) {
+          const int64_t W = a.c.W, cn = (int64_t)md.count + 1;
+          me.next_pos = md.next_pos + 1;
+          me.count = (int32_t)(cn < W ? cn : W);
+          me.head = (int32_t)((md.head + (cn > W ? 1 : 0)) % W);
+        }
+        if (me.next_pos != m.next_pos || me.P != m.P || me.head != m.head ||
+            me.count != m.count || me.owner != m.owner)
+          bad = true;
+      }
+      if (bad) atomicOr(a.c.err, ERR_BATCH);
+      if (!runs.ring_ok) atomicOr(a.c.err, ERR_RING);
+    };
+    if (CL) {
+      const int pair = blockIdx.x / a.csize, rank = (int)ptx::cluster_ctarank();
+      const int b = pair / Hkv, g = pair % Hkv;
+      piece(b, g, 0, 0, 0, rank, false);
+    } else {
+      const int32_t x1 = range_start(blockIdx.x + 1, R, NC);
+      for (int32_t x = range_start(blockIdx.x, R, NC); x < x1 && alive;) {
+        const PairTiles pt = pair_of_tile(a, x);
+        const int32_t j0 = x - pt.first, j1 = min(pt.tph, x1 - pt.first);
+        x = pt.first + j1;
+        piece(pt.b, pt.g, pt.tph, j0, j1, -1, true);
+      }
+    }
+    if (alive) {  // end marker: a descriptor with no bytes
+      wait_primary();
+      const int st = i % kStagesM;
+      if (i < kStagesM || ptx::mbar_wait_bounded(&empty[st], ((i / kStagesM) - 1) & 1,
+                                                  &abort_flag, kWaitLimitCycles)) {
+        TileDescM end;
+        for (int w = 0; w < kTR / 32; ++w) end.mask[w] = 0u;
+        end.pair = 0; end.flags = TD_END; end.slot = 0; end.new_row = -1;
+        desc[st] = end;
+        ptx::mbar_arrive(&full[st]);
+        ++i;
+      }
+    }
+    if (abort_flag) {  // let the copies already issued land before the CTA exits
+      int quiet = 0;
+      for (int k = max(0, i - kStagesM); k < i; ++k)
+        ptx::mbar_wait_bounded(&full[k % kStagesM], (k / kStagesM) & 1, &quiet, kWaitLimitCycles);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers --
+  auto csync = [&](uint64_t* bar, int phase) -> bool {
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(bar);
+    return __all_sync(0xffffffffu,
+                      ptx::mbar_wait_bounded(bar, phase & 1, &abort_flag, kWaitLimitCycles));
+  };
+  const unsigned FULL = 0xffffffffu;
+  const int g = lane >> 2, tq = lane & 3;
+  const int sw = lane & 7;  // 128-byte swizzle: 16-byte chunk c of row r sits at c ^ (r & 7)
+  // ldmatrix source rows of this lane: K as the A operand (matrices: rows 0-7 /
+  // 8-15 of k 0-7, then of k 8-15), V transposed (rows 0-7 of d 0-7 / 8-15,
+  // then rows 8-15)
+  const int krow = (lane & 7) + ((lane >> 3) & 1) * 8, kchk = lane >> 4;
+  const int vrow = (lane & 7) + ((lane >> 4) & 1) * 8, vchk = (lane >> 3) & 1;
+  const float qs = a.qscale;
+  MmaState<D, G> st;
+  int np = 0;
+  bool stopped = false;
+  for (int i = 0;; ++i) {
+    const int stg = i % kStagesM;
+    const bool ok = ptx::mbar_wait_bounded(&full[stg], (i / kStagesM) & 1, &abort_flag,
+                                           kWaitLimitCycles);
+    if (!__all_sync(FULL, ok)) { stopped = true; break; }
+    const TileDescM d = desc[stg];
+    if (d.flags & TD_END) break;
+    if (d.flags & TD_FIRST) st.init(qbuf + (size_t)stg * G * D * 2);
+    uint8_t* const kt = kbuf + (size_t)stg * kTileBytes;
+    uint8_t* const vt = vbuf + (size_t)stg * kTileBytes;
+    const uint32_t kt_s = ptx::smem_u32(kt), vt_s = ptx::smem_u32(vt);
+    bool wrote = false;
+#pragma unroll 1
+    for (int grp = warp; grp < kGroups; grp += kMW) {
+      // (the mask word is read from shared memory: indexing a local copy by
+      // the loop variable would put the copy in local memory)
+      const uint32_t vm = (desc[stg].mask[grp >> 1] >> ((grp & 1) * 16)) & 0xffffu;
+      if (vm == 0) continue;
+      const int R0 = grp * 16;
+      if (vm != 0xffffu) {
+        // rows outside the visible set: their V rows must not reach O
+        for (int idx = lane; idx < 16 * HALVES * 8; idx += 32) {
+          const int r = idx / (HALVES * 8), h = (idx / 8) % HALVES, ch = idx % 8;
+          if (!((vm >> r) & 1u))
+            *(uint4*)(vt + h * kHalfBytes + (R0 + r) * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
+        }
+        __syncwarp();
+        wrote = true;
+      }
+      // S^T = K Q^T
+      float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        const int h = ks >> 2, chunk = (ks & 3) * 2 + kchk;
+        uint32_t af[4];
+        ldsm4(kt_s + h * kHalfBytes + (R0 + krow) * 128 + ((chunk ^ sw) << 4), af);
+        mma16816(c, af, st.qf[ks][0], st.qf[ks][1]);
+      }
+      const bool r0 = (vm >> g) & 1u, r1 = (vm >> (g + 8)) & 1u;
+      const float s0 = r0 ? c[0] * qs : -INFINITY, s1 = r0 ? c[1] * qs : -INFINITY;
+      const float s2 = r1 ? c[2] * qs : -INFINITY, s3 = r1 ? c[3] * qs : -INFINITY;
+      const bool need = s0 > st.m[0] + kRaiseLog2 || s2 > st.m[0] + kRaiseLog2 ||
+                        s1 > st.m[1] + kRaiseLog2 || s3 > st.m[1] + kRaiseLog2;
+      if (__any_sync(FULL, need)) {
+        // rare: raise the running max of a head to the group's max
+        float gm[2] = {fmaxf(s0, s2), fmaxf(s1, s3)};
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          gm[hh] = fmaxf(gm[hh], __shfl_xor_sync(FULL, gm[hh], 4));
+          gm[hh] = fmaxf(gm[hh], __shfl_xor_sync(FULL, gm[hh], 8));
+          gm[hh] = fmaxf(gm[hh], __shfl_xor_sync(FULL, gm[hh], 16));
+          if (gm[hh] > st.m[hh] + kRaiseLog2) {
+            const float alpha = ex2(st.m[hh] - gm[hh]);  // 0 when the max was -inf
+#pragma unroll
+            for (int mt = 0; mt < KS; ++mt) {
+              st.o[mt][hh] *= alpha;
+              st.o[mt][hh + 2] *= alpha;
+            }
+            st.l[hh] *= alpha;
+            st.m[hh] = gm[hh];
+          }
+        }
+      }
+      // every valid head's max is finite here; a padding head's is +inf
+      const float p0 = ex2(s0 - st.m[0]), p1 = ex2(s1 - st.m[1]);
+      const float p2 = ex2(s2 - st.m[0]), p3 = ex2(s3 - st.m[1]);
+      st.l[0] += p0 + p2;
+      st.l[1] += p1 + p3;
+      const uint32_t b0 = movm_t(pack_bf16(p0, p1)), b1 = movm_t(pack_bf16(p2, p3));
+      // O^T += V^T P^T
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        const int h = mt >> 2, chunk = (mt & 3) * 2 + vchk;
+        uint32_t af[4];
+        ldsm4_t(vt_s + h * kHalfBytes + (R0 + vrow) * 128 + ((chunk ^ sw) << 4), af);
+        mma16816(st.o[mt], af, b0, b1);
+      }
+    }
+    if ((d.flags & TD_NEW) && warp == (d.new_row >> 4) % kMW) {
+      // decode step: store the appended token in its ring slot (the evicted
+      // row's, never visible to this step's queries); tile row new_row is a
+      // multiple of 8, where the swizzle is the identity
+      const int b = d.pair / Hkv, gg = d.pair % Hkv, s = a.seq[b];
+      const int32_t slot = (int32_t)(((int64_t)a.head[b] + a.count[b] - 1) % a.c.W);
+      const int phys = ring_page(a.c, s, slot);
+      const size_t row = (size_t)ring_row(a.c, phys, gg, slot) * D;
+      constexpr int V16 = D * 2 / 16;  // 16-byte pieces per row
+      for (int x = lane; x < 2 * V16; x += 32) {
+        const bool isv = x >= V16;
+        const int xi = isv ? x - V16 : x;
+        const uint4 val =
+            *(const uint4*)((isv ? vt : kt) + (xi / 8) * kHalfBytes + d.new_row * 128 + (xi % 8) * 16);
+        ((uint4*)((uint16_t*)(isv ? a.c.V : a.c.K) + row))[xi] = val;
+      }
+      if (lane == 0 && gg == 0) a.c.pos[pos_index(a.c, phys, slot)] = a.t[b];
+    }
+    if (wrote) fence_proxy_async_smem();  // generic writes before the stage's next copies
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(&empty[stg]);
+    if (!(d.flags & TD_LAST)) continue;
+
+    // ---- end of a (CTA range, pair) piece: merge the warps' states ----
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      st.l[hh] += __shfl_xor_sync(FULL, st.l[hh], 4);
+      st.l[hh] += __shfl_xor_sync(FULL, st.l[hh], 8);
+      st.l[hh] += __shfl_xor_sync(FULL, st.l[hh], 16);
+    }
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int h = 2 * tq + hh;
+      if (h < G) {
+        if (g == 0) {
+          sm.m[warp][h] = st.m[hh];
+          sm.l[warp][h] = st.l[hh];
+        }
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt) {
+          sm.o[warp][h][16 * mt + g] = st.o[mt][hh];
+          sm.o[warp][h][16 * mt + g + 8] = st.o[mt][hh + 2];
+        }
+      }
+    }
+    if (!csync(&sync_a, np)) { stopped = true; break; }
+    const int64_t slot = d.slot;
+    float* pml = a.part_ml + (size_t)slot * G * 2;
+    float* po = a.part_o + (size_t)slot * G * D;
+    for (int idx = threadIdx.x; idx < G * D; idx += kMW * 32) {
+      const int h = idx / D, e = idx % D;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kMW; ++w) mx = fmaxf(mx, sm.m[w][h]);
+      float l = 0.f, acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < kMW; ++w) {
+        const float wt = (mx == -INFINITY) ? 0.f : exp2f(sm.m[w][h] - mx);
+        l += sm.l[w][h] * wt;
+        acc += sm.o[w][h][e] * wt;
+      }
+      if (CL) {  // this CTA's state, in place (each thread rewrites only its own (h, e))
+        sm.o[0][h][e] = acc;
+        if (e == 0) { pub_ml[h][0] = mx; pub_ml[h][1] = l; }
+      } else {
+        po[idx] = acc;
+        if (e == 0) {
+          pml[h * 2] = mx;
+          pml[h * 2 + 1] = l;
+        }
+      }
+    }
+    if (!csync(&sync_b, np)) { stopped = true; break; }
+    ++np;
+  }
+
+  if (CL && !stopped && !abort_flag) {
+    // ---- cluster: combine the pair's csize states into its output ----
+    if (np == 0) {  // no tiles in this CTA's share: an empty state
+      for (int idx = threadIdx.x; idx < G * D; idx += kMW * 32) {
+        const int h = idx / D, e = idx % D;
+        sm.o[0][h][e] = 0.f;
+        if (e == 0) { pub_ml[h][0] = -INFINITY; pub_ml[h][1] = 0.f; }
+      }
+      if (!csync(&sync_c, 0)) stopped = true;
+    }
+    const int rank = (int)ptx::cluster_ctarank(), C = a.csize;
+    if (!stopped && rank != 0) {
+      // publish to rank 0, then keep this CTA's shared memory alive until it has read it
+      if (threadIdx.x == 0) {
+        ptx::fence_acq_rel_cluster();
+        ptx::mbar_arrive_cluster(ptx::map_to_rank(&pub_bar, 0));
+        ptx::mbar_wait_cluster_bounded(&done_bar, 0, &abort_flag, kWaitLimitCycles);
+      }
+    } else if (!stopped) {
+      const bool ok = ptx::mbar_wait_cluster_bounded(&pub_bar, 0, &abort_flag, kWaitLimitCycles);
+      if (__all_sync(FULL, ok)) {
+        const int pair = blockIdx.x / C, b = pair / Hkv, gg = pair % Hkv;
+        for (int idx = threadIdx.x; idx < G * D; idx += kMW * 32) {
+          const int h = idx / D, e = idx % D;
+          float mr[kMaxCluster], lr[kMaxCluster], orr[kMaxCluster];
+          float M = -INFINITY;
+#pragma unroll
+          for (int r = 0; r < kMaxCluster; ++r) {
+            if (r < C) {
+              mr[r] = r == 0 ? pub_ml[h][0] : ptx::ld_cluster_f32(ptx::map_to_rank(&pub_ml[h][0], r));
+              lr[r] = r == 0 ? pub_ml[h][1] : ptx::ld_cluster_f32(ptx::map_to_rank(&pub_ml[h][1], r));
+              orr[r] = r == 0 ? sm.o[0][h][e] : ptx::ld_cluster_f32(ptx::map_to_rank(&sm.o[0][h][e], r));
+              M = fmaxf(M, mr[r]);
+            }
+          }
+          float L = 0.f, A = 0.f;
+#pragma unroll
+          for (int r = 0; r < kMaxCluster; ++r) {
+            if (r < C) {
+              const float w = (mr[r] == -INFINITY) ? 0.f : exp2f(mr[r] - M);
+              L += lr[r] * w;
+              A += orr[r] * w;
+            }
+          }
+          store_out<uint16_t>((uint16_t*)a.out + ((size_t)b * a.Hq + (size_t)gg * G + h) * D + e,
+                              A / L);
+        }
+        // the peers' shared memory has been read: let them exit
+        if (csync(&sync_c, np == 0 ? 1 : 0) && threadIdx.x == 0) {
+          for (int r = 1; r < C; ++r) ptx::mbar_arrive_cluster(ptx::map_to_rank(&done_bar, r));
+          if (gg == 0) {
+            // the sequence's bookkeeping: check the device record, then (decode
+            // step) commit the state after the append
+            const int s = a.seq[b];
+            const DevMeta md = a.c.meta[s];
+            DevMeta m;
+            memset(&m, 0, sizeof(m));
+            m.next_pos = a.t[b] + 1;
+            m.P = a.P[b];
+            m.head = a.head[b];
+            m.count = a.count[b];
+            m.owner = a.owner[b];
+            DevMeta me = md;
+            if (a.knew != nullptr) {
+              const int64_t W = a.c.W, cn = (int64_t)md.count + 1;
+              me.next_pos = md.next_pos + 1;
+              me.count = (int32_t)(cn < W ? cn : W);
+              me.head = (int32_t)((md.head + (cn > W ? 1 : 0)) % W);
+            }
+            if (me.next_pos != m.next_pos || me.P != m.P || me.head != m.head ||
+                me.count != m.count || me.owner != m.owner)
+              atomicOr(a.c.err, ERR_BATCH);
+            if (a.knew != nullptr) a.c.meta[s] = m;
+          }
+        }
+      }
+    }
+  }
+  if (threadIdx.x == 0 && abort_flag) atomicOr(a.c.err, ERR_TIMEOUT);
+}
+
+// Resident CTAs per SM of one instantiation (at most PS_DMMA_CTAS_PER_SM).
+template <int D, int G, bool CL>
+int ctas_per_sm(size_t dyn) {
+  static std::atomic<int> cached{0};
+  int n = cached.load();
+  if (n == 0) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_decode_mma<D, G, CL>, kThreadsM,
+                                                      dyn) != cudaSuccess || n < 1)
+      n = 1;
+    if (n > PS_DMMA_CTAS_PER_SM) n = PS_DMMA_CTAS_PER_SM;
+    cached.store(n);
+  }
+  return n;
+}
+
+template <int D, int G, bool CL>
+cudaError_t configure(size_t dyn) {
+  static std::atomic<uint64_t> configured{0};  // one bit per device
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (!(configured.load() & bit)) {
+    e = cudaFuncSetAttribute(k_decode_mma<D, G, CL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)dyn);
+    if (e != cudaSuccess) return e;
+    // all of the unified L1/shared memory as shared, so that two CTAs fit per SM
+    e = cudaFuncSetAttribute(k_decode_mma<D, G, CL>,
+                             cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    configured.fetch_or(bit);
+  }
+  return cudaSuccess;
+}
+
+template <int D, int G>
+cudaError_t launch_mma(MmaDecodeArgs& ma, int sm_count, cudaStream_t st) {
+  DecodeArgs& a = ma.a;
+  const int32_t page = a.c.page_table ? a.c.page_rows : 0;
+  const bool step = a.knew != nullptr;
+  a.tcum[0] = 0;
+  int32_t tmin = INT32_MAX, tmax = 0;
+  for (int b = 0; b < a.B; ++b) {
+    DevMeta m;
+    memset(&m, 0, sizeof(m));
+    m.next_pos = a.t[b] + 1;
+    m.P = a.P[b];
+    m.head = a.head[b];
+    m.count = a.count[b];
+    m.owner = a.owner[b];
+    const DecRuns r = dec_runs(m, a.c.W, a.t[b], page, step);
+    const int32_t tph = dec_tiles(r, kTR);
+    a.tcum[b + 1] = a.tcum[b] + a.c.Hkv * tph;
+    tmin = tph < tmin ? tph : tmin;
+    tmax = tph > tmax ? tph : tmax;
+  }
+  a.total = a.tcum[a.B];
+  constexpr size_t dyn = 1024 + (size_t)kStagesM * (2 * (D / 64) * kTR * 128 + G * D * 2);
+  // Cluster mode when there are few pairs of about equal length: csize CTAs
+  // per pair with csize the largest of 8, 4, 2 that keeps every CTA resident
+  // at once, provided that fills at least half of the resident slots and gives
+  // each CTA a few tiles.  Otherwise the flattened split.
+  const int64_t pairs = (int64_t)a.B * a.c.Hkv;
+  cudaError_t e;
+  if ((e = configure<D, G, true>(dyn)) != cudaSuccess) return e;
+  if ((e = configure<D, G, false>(dyn)) != cudaSuccess) return e;
+  int csize = 0;
+#ifndef PS_DMMA_NO_CLUSTER
+  {
+    const int64_t slots = (int64_t)sm_count * ctas_per_sm<D, G, true>(dyn);
+    for (int c = kMaxCluster; c >= 2; c /= 2) {
+      if (pairs * c <= slots) {
+        if (2 * pairs * c >= slots && tmin >= 2 * c && 4 * tmax <= 5 * tmin) csize = c;
+        break;
+      }
+    }
+  }
+#endif
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t dcfg = {};
+  dcfg.blockDim = dim3(kThreadsM);
+  dcfg.dynamicSmemBytes = dyn;
+  dcfg.stream = st;
+  dcfg.attrs = attr;
+  if (csize > 0) {
+    a.csize = csize;
+    a.nctas = (int)(pairs * csize);
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)csize;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    dcfg.numAttrs = 2;
+    dcfg.gridDim = dim3((unsigned)a.nctas);
+    return cudaLaunchKernelEx(&dcfg, k_decode_mma<D, G, true>, ma);
+  }
+  a.csize = 0;
+  int64_t nc = ((int64_t)a.total + kMinTilesPerCta - 1) / kMinTilesPerCta;
+  const int64_t maxc = (int64_t)sm_count * ctas_per_sm<D, G, false>(dyn);
+  if (nc > maxc) nc = maxc;
+  if (nc < 1) nc = 1;
+  a.nctas = (int)nc;
+  dcfg.numAttrs = 1;
+  dcfg.gridDim = dim3((unsigned)a.nctas);
+  e = cudaLaunchKernelEx(&dcfg, k_decode_mma<D, G, false>, ma);
+  if (e != cudaSuccess) return e;
+  return launch_merge<uint16_t, D, G>(a, st);
+}
+
+}  // namespace
+
+bool make_decode_maps(const CacheDev& c, DecodeMaps* m) {
+  const uint64_t row = (uint64_t)c.d * 2;
+  const uint64_t prows = c.pstride > 0 ? (uint64_t)c.pstride : 1;
+  const char* kring = (const char*)c.K + (size_t)c.rbase * row;
+  const char* vring = (const char*)c.V + (size_t)c.rbase * row;
+  const uint64_t nslab = (uint64_t)c.S * c.Hkv, nring = (uint64_t)c.nphys * c.Hkv;
+  bool ok = true;
+  for (int k = 0; k < 2; ++k) {
+    const uint32_t box = k == 0 ? (uint32_t)kBox : (uint32_t)kPadRows;
+    const int pr = PS_DMMA_L2_PROMOTION;
+    ok = ok && encode_map3d_bf16(&m->kpre[k], c.K, c.d, prows, nslab, row, prows * row, 64, box, 1,
+                                 pr);
+    ok = ok && encode_map3d_bf16(&m->vpre[k], c.V, c.d, prows, nslab, row, prows * row, 64, box, 1,
+                                 pr);
+    ok = ok && encode_map3d_bf16(&m->kring[k], kring, c.d, (uint64_t)c.page_rows, nring, row,
+                                 (uint64_t)c.rstride * row, 64, box, 1, pr);
+    ok = ok && encode_map3d_bf16(&m->vring[k], vring, c.d, (uint64_t)c.page_rows, nring, row,
+                                 (uint64_t)c.rstride * row, 64, box, 1, pr);
+  }
+  // Whole-tile maps (head_dim 128): dimensions (64 columns, rows, column
+  // block, slab); the column block is the outer box dimension, so one copy
+  // writes the tile's two 64-column blocks one after the other, as the kernel
+  // lays them out.
+  m->whole = 0;
+  if (ok && c.d == 128) {
+    const uint32_t box[4] = {64, (uint32_t)kBox, 2, 1};
+    const uint64_t dp[4] = {64, prows, 2, nslab}, sp[3] = {row, 128, prows * row};
+    const uint64_t dr[4] = {64, (uint64_t)c.page_rows, 2, nring},
+                   sr[3] = {row, 128, (uint64_t)c.rstride * row};
+    const int pr = PS_DMMA_L2_PROMOTION;
+    m->whole = encode_map_bf16(&m->kpre_w, c.K, 4, dp, sp, box, pr) &&
+               encode_map_bf16(&m->vpre_w, c.V, 4, dp, sp, box, pr) &&
+               encode_map_bf16(&m->kring_w, kring, 4, dr, sr, box, pr) &&
+               encode_map_bf16(&m->vring_w, vring, 4, dr, sr, box, pr);
+  }
+  return ok;
+}
+
+cudaError_t launch_decode_mma(const DecodeArgs& a, int G, const DecodeMaps& maps, int sm_count,
+                              cudaStream_t st) {
+  MmaDecodeArgs ma;
+  memset(&ma, 0, sizeof(ma));
+  ma.maps = maps;
+  ma.a = a;
+  const int D = a.c.d;
+#define PS_DMMA_CASE(DD, GG) \
+  if (D == DD && G == GG) return launch_mma<DD, GG>(ma, sm_count, st);
+  PS_DMMA_CASE(128, 1) PS_DMMA_CASE(128, 2) PS_DMMA_CASE(128, 4) PS_DMMA_CASE(128, 8)
+  PS_DMMA_CASE(64, 1) PS_DMMA_CASE(64, 2) PS_DMMA_CASE(64, 4) PS_DMMA_CASE(64, 8)
+#undef PS_DMMA_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace ps

@@ -1,5 +1,6 @@
 // Host-side declarations shared by the library's translation units.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -17,6 +18,17 @@ struct BatchIds {
   int32_t owner[kMaxBatchPerLaunch];  // sequence whose slab holds the prefix rows
   int64_t t[kMaxBatchPerLaunch];
 };
+
+// tmap.cu: a 3-D bf16 tensor map with 128-byte swizzle; dims innermost first,
+// byte strides of dims 1 and 2, box sizes b0..b2, L2 promotion of its loads
+// (0 none, 1 128 bytes, 2 256 bytes).  False if encoding failed.
+bool encode_map3d_bf16(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                       uint64_t s1, uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2,
+                       int l2_promotion = 2);
+// The same for a map of `rank` dimensions (strides[i]: bytes between
+// consecutive indices of dimension i + 1).
+bool encode_map_bf16(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+                     const uint64_t* strides, const uint32_t* box, int l2_promotion = 2);
 
 // ring.cu
 constexpr int kMaxPageSets = 256;  // page-table entries per update launch
@@ -51,9 +63,22 @@ size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int sm_count);
 // [B][Hkv][d] at positions ids.t (ids then holds the state after the append),
 // which the launch reads for the attention, writes to their ring slots, and
 // after which it commits the new bookkeeping.
+// Tensor maps of a bf16 cache's K/V for the tensor-core decode kernel: prefix
+// slabs and ring pages, each with a box of 64 rows ([0]) and of 8 rows ([1])
+// of one 64-column block, and (whole, when encodable) a box of 64 rows of
+// both column blocks of a 128-column row, which fills a whole tile with one
+// copy.
+struct DecodeMaps {
+  CUtensorMap kpre[2], vpre[2], kring[2], vring[2];
+  CUtensorMap kpre_w, vpre_w, kring_w, vring_w;
+  int whole;  // 1 if the whole-tile maps exist (head_dim 128)
+};
+bool make_decode_maps(const CacheDev& c, DecodeMaps* m);
+// maps: the cache's decode maps (bf16 caches; NULL for float32).
 cudaError_t launch_decode(const CacheDev& c, int dtype, int G, const BatchIds& ids, int B, int Hq,
                           const void* q, const void* k_new, const void* v_new, void* out,
-                          float scale, const DecodeWs& ws, int sm_count, cudaStream_t st);
+                          float scale, const DecodeWs& ws, int sm_count, const DecodeMaps* maps,
+                          cudaStream_t st);
 
 // chunk_tc.cu (tcgen05 chunk kernel: bf16, head_dim 128)
 bool chunk_tc_supported(const CacheDev& c, int dtype, int d, int G);
@@ -85,6 +110,10 @@ int set_error(int code, const char* fmt, ...);
 
 struct ps_cache;
 namespace ps {
+// Every host-side check of ps_attend_decode except the workspace's (the
+// message is set on failure); *G receives Hq / Hkv.
+int check_decode_call(ps_cache* c, const void* q, const int* seq_ids, const int64_t* t, int B,
+                      int Hq, const void* out, int* G);
 int cache_hkv(const ps_cache* c);
 int cache_head_dim(const ps_cache* c);
 int cache_sm_count(const ps_cache* c);

@@ -5,16 +5,20 @@ device memory through its own pool, or a latency-critical loop that must not
 call cudaMalloc (it synchronises the device).  This entry point runs the same
 decode with its scratch in a fixed array inside the library.  These tests call
 it through the C ABI and compare it with ps_attend_decode (caller workspace) on
-two calls in a row, within the bf16 tolerances used by every parity test.
-The file is named to be collected last.
+two calls in a row: the same kernels with the same slot layout, so the outputs
+must be bit-identical (which is within the bf16 tolerances of every parity
+test); both are also checked against the float64 oracle.  The file is named to
+be collected last.
 """
 import math
 
+import numpy as np
 import pytest
 import torch
 
+import oracle
 from prefix_sliding_window_ring_b200 import Cache, PSError, abi
-from tests.helpers import SeqData, check_close, ps_dtype, to_f64, to_torch
+from tests.helpers import SeqData, check_close, oracle_decode, ps_dtype, to_f64, to_torch
 
 pytestmark = pytest.mark.gpu
 
@@ -46,7 +50,14 @@ def test_static_scratch_matches_workspace_decode_twice():
         abi.ps_attend_decode(c.handle, q, ids, [t] * B, Hq, scale, ref, ws, ws.numel())
         abi.ps_attend_decode_static(c.handle, q, ids, [t] * B, Hq, scale, got)
         torch.cuda.synchronize()
+        assert torch.equal(got, ref), f"static vs workspace differ, call {step + 1}"
         check_close(to_f64(got), to_f64(ref), "bf16", f"static vs workspace, call {step + 1}")
+        batch = oracle.Batch()
+        q64 = to_f64(q)
+        exp = [oracle_decode(batch, sd, P, W, t, scale, q64[b]) for b, sd in enumerate(sds)]
+        batch.run()
+        want = np.stack([np.concatenate(e, axis=0) for e in exp])
+        check_close(to_f64(got), want, "bf16", f"static vs oracle, call {step + 1}")
     assert c.device_error() == 0
 
 
@@ -66,3 +77,22 @@ def test_static_scratch_rejects_batches_over_its_size():
         abi.ps_attend_decode_static(c.handle, q, list(range(B)), [P + W - 1] * B, Hq, 0.1, out)
     assert e.value.code == abi.PS_ENOMEM
     assert "scratch" in str(e.value)
+
+
+def test_static_scratch_checks_arguments_first():
+    """Bad arguments are reported as by ps_attend_decode (not as a set-up
+    failure), and an empty batch is a no-op."""
+    c, sds = _setup(2, 4, 2, 128, 8, 64, 100)
+    q = torch.zeros((2, 4, 128), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty_like(q)
+    abi.ps_attend_decode_static(c.handle, q, [], [], 4, 0.1, out)          # B = 0
+    with pytest.raises(PSError) as e:
+        abi.ps_attend_decode_static(c.handle, q, [0, 1], [100, 100], 4, 0.1, out)
+    assert e.value.code == abi.PS_EPOS                                      # t is not next_pos-1
+    with pytest.raises(PSError) as e:
+        abi.ps_attend_decode_static(c.handle, q, [0, 0], [99, 99], 4, 0.1, out)
+    assert e.value.code == abi.PS_EINVAL                                    # duplicate id
+    with pytest.raises(PSError) as e:
+        abi.ps_attend_decode_static(c.handle, q, [0, 1], [99, 99], 3, 0.1, out)
+    assert e.value.code == abi.PS_EINVAL                                    # Hq % Hkv
+    assert c.device_error() == 0
