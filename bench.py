@@ -406,12 +406,40 @@ def run_ours(args, rank, world, local_rank):
         e2e_step(base + i)
     torch.cuda.synchronize()
     base += 2
+    # Graph of the K steps with the copies on a second stream: the upload of
+    # step i+1 (into the other of two input buffers) overlaps the decode of
+    # step i, and the read-back of step i overlaps the decode of step i+1.
+    # Every step still uploads its own inputs and reads back its own output.
+    din2 = [din, torch.empty_like(din)]
+    dviews = [(d[:nq].view(B, HQ, D), d[nq:nq + nk].view(B, HKV, D), d[nq + nk:].view(B, HKV, D))
+              for d in din2]
+    hout2 = [hout, torch.empty_like(hout).pin_memory()]
     s2 = torch.cuda.Stream()
+    sc = torch.cuda.Stream()
     s2.wait_stream(torch.cuda.current_stream())
+    sc.wait_stream(torch.cuda.current_stream())
     g2 = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g2, stream=s2):
+        sc.wait_stream(s2)
+        ev_in = [torch.cuda.Event() for _ in range(K)]
+        ev_dec = [torch.cuda.Event() for _ in range(K)]
         for i in range(K):
-            e2e_step(base + i, s2)
+            b = i % 2
+            r = (base + i) % ROT
+            v = wl.visit[r]
+            with torch.cuda.stream(sc):
+                if i >= 2:
+                    sc.wait_event(ev_dec[i - 2])  # input buffer b is free again
+                din2[b].copy_(hin[r][v], non_blocking=True)
+                ev_in[i].record(sc)
+            s2.wait_event(ev_in[i])
+            qv, kv_, vv = dviews[b]
+            out = wl.step(base + i, s2, host=lambda r_, v_: (kv_, vv, qv))
+            ev_dec[i].record(s2)
+            with torch.cuda.stream(sc):
+                sc.wait_event(ev_dec[i])
+                hout2[b].copy_(out, non_blocking=True)
+        s2.wait_stream(sc)
     torch.cuda.synchronize()
     upload_graph(torch, g2, s2)
     if dist:
@@ -445,9 +473,10 @@ def run_ours(args, rank, world, local_rank):
     prefill = None
     if rank == 0 and not args.no_prefill:
         prefill = prefill_measure(max(3, min(args.steps, 10)))
-    ragged = shared = paged = t_sweep = None
+    ragged = shared = paged = t_sweep = gqa = None
     if rank == 0 and not args.no_prefill:
         ragged = ragged_measure(max(3, min(args.steps, 10)))
+        gqa = gqa_measure(max(args.steps, 16))
         shared = shared_prefix_measure(max(3, min(args.steps, 10)))
         paged = paged_measure(max(3, min(args.steps, 10)))
         try:  # an extra section: a failure here is reported, not fatal to the line
@@ -481,7 +510,8 @@ def run_ours(args, rank, world, local_rank):
                 "copies": "one upload of a pinned [q | k | v] record and one read-back of the "
                           "output per step, on the decode stream",
                 "issue": "the K steps (upload, ps_decode_step, read-back) captured into one "
-                         "CUDA graph and replayed",
+                         "CUDA graph and replayed; uploads and read-backs on a second stream, "
+                         "double-buffered, overlapping the neighbouring steps' kernels",
                 "eager": {"value": round(e2e_eager, 1), "unit": UNIT,
                           "issue": "the same steps issued one by one from Python"}},
         "gpu_launches": 2 * K,  # per step: the decode-step stream launch and the pair merge
@@ -493,6 +523,7 @@ def run_ours(args, rank, world, local_rank):
         "shared_prefix": shared,
         "paged": paged,
         "t_sweep": t_sweep,
+        "gqa": gqa,
     }
     print(json.dumps(line), flush=True)
 
@@ -815,6 +846,53 @@ def paged_measure(steps: int):
     return res
 
 
+def gqa_measure(steps: int):
+    """The decode call (ps_attend_decode) at B=8, Hkv=8, d=128, P=128, W=4096,
+    t=65536, bf16, for GQA group sizes G = Hq / Hkv in {1, 2, 4, 8}: the same
+    K/V bytes per call (138.4 MB), G query heads per kv head.  4 disjoint
+    batches rotate (HBM-resident)."""
+    import torch
+
+    from prefix_sliding_window_ring_b200 import PS_BF16, Cache
+    peak, _ = load_peaks()
+    g = torch.Generator(device="cuda").manual_seed(SEED + 11)
+    scale = 1.0 / math.sqrt(D)
+    t = 65536
+    res = {"note": "ps_attend_decode, B=8 Hkv=8 d=128 P=128 W=4096 t=65536 bf16, Hq = G * 8"}
+    S = B * ROT
+    c = Cache(W, P, HKV, D, PS_BF16, S)
+    for s in range(S):
+        h0 = (s * 613) % W
+        c.seq_reset(s, h0)
+        c.prefill_prefix(s, torch.randn((P, HKV, D), generator=g, device="cuda").to(torch.bfloat16),
+                         torch.randn((P, HKV, D), generator=g, device="cuda").to(torch.bfloat16), P)
+        c.import_window(s, t + 1, torch.randn((W, HKV, D), generator=g, device="cuda").to(torch.bfloat16),
+                        torch.randn((W, HKV, D), generator=g, device="cuda").to(torch.bfloat16), W, h0)
+    for G in (1, 2, 4, 8):
+        hq = G * HKV
+        q = torch.randn((B, hq, D), generator=g, device="cuda").to(torch.bfloat16)
+        out = torch.empty_like(q)
+        ws = c.decode_workspace(B, hq)
+
+        def dec(i, st=None):
+            r = i % ROT
+            c.attend_decode(q, list(range(r * B, (r + 1) * B)), [t] * B, hq, scale, out, ws, st)
+
+        for i in range(2 * ROT):
+            dec(i)
+        torch.cuda.synchronize()
+        ms = time_graph(torch, dec, max(steps, 4 * ROT))
+        if c.device_error():
+            raise RuntimeError(f"device error word set by the decode at G={G}")
+        gbs = kv_bytes_per_step() / (ms / 1e3) / 1e9
+        res[f"G{G}"] = {"Hq": hq, "us_per_call": round(ms * 1e3, 2), "GBps": round(gbs, 1),
+                        "frac": round(gbs / peak, 4)}
+        del q, out, ws
+    c.close()
+    torch.cuda.empty_cache()
+    return res
+
+
 def t_sweep_measure(steps: int):
     """The decode call (ps_attend_decode, B=8, Hq=16, Hkv=8, d=128, bf16) at the
     positions the workload is quoted at, t in {2048, 4224, 16384, 65536} with
@@ -964,7 +1042,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-prefill", action="store_true")
-    ap.add_argument("--only", choices=["prefill", "prompt", "ragged", "shared", "paged", "t_sweep"],
+    ap.add_argument("--only", choices=["prefill", "prompt", "ragged", "shared", "paged", "t_sweep",
+                                       "gqa"],
                     help="run one side measurement alone and print its record (for profiling "
                          "one kernel under ncu); not a benchmark line")
     args = ap.parse_args()
@@ -980,6 +1059,7 @@ def main():
         fn = {"prefill": prefill_measure, "ragged": ragged_measure,
               "shared": shared_prefix_measure, "paged": paged_measure,
               "t_sweep": lambda n: t_sweep_measure(max(n, 16)),
+              "gqa": lambda n: gqa_measure(max(n, 16)),
               "prompt": lambda n: prompt_measure(n, load_bf16_peak()[0])}[args.only]
         print(json.dumps({"only": args.only, "result": fn(k)}), flush=True)
     elif args.impl == "reference":

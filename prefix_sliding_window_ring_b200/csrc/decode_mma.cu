@@ -70,9 +70,6 @@
 #ifndef PS_DMMA_L2_PROMOTION
 #define PS_DMMA_L2_PROMOTION 2
 #endif
-#ifndef PS_DMMA_PREFETCH_TILES
-#define PS_DMMA_PREFETCH_TILES 4
-#endif
 
 namespace ps {
 
@@ -228,8 +225,11 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
     }
   }
   __syncthreads();
-  // every CTA of the cluster has initialised its barriers before any remote arrive
-  if (CL) ptx::cluster_sync_all();
+  // Cluster mode: every CTA of the cluster must have initialised its barriers
+  // before any remote arrive (the consumers' epilogue).  All threads arrive
+  // here; the consumers wait at once, the producer only after setting up its
+  // first piece, which so overlaps the barrier.
+  if (CL) ptx::cluster_arrive();
   // Programmatic dependent launch: the next grid may be scheduled.  Only the
   // producer waits for the previous grid (griddepcontrol.wait), just before its
   // first copy: everything the consumers read or write in global memory comes
@@ -247,6 +247,7 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
     bool waited = false;  // griddepcontrol.wait done
     auto wait_primary = [&]() {
       if (!waited) {
+        if (CL) ptx::cluster_wait_one();
         ptx::pdl_wait_primary();
         waited = true;
       }
@@ -276,27 +277,6 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
         xe = min(j1 * kTR, runs.padded);
       }
       const int32_t nt = xe > xs ? (xe - xs + kTR - 1) / kTR : 0;
-      // Before the previous grid has completed: bring this CTA's first whole
-      // tiles into L2, so that DRAM works during the previous grid's tail and
-      // the copies after the wait hit L2.  (Only the cache is touched; the
-      // copies themselves still come after griddepcontrol.wait.)
-      if (!waited) {
-        for (int32_t k = 0; k < nt && k < PS_DMMA_PREFETCH_TILES; ++k) {
-          const int32_t x0 = xs + k * kTR, x1 = min(x0 + kTR, xe);
-          int32_t wsrc, wrow;
-          if (!dec_range_whole(runs, kTR, x0, x1, &wsrc, &wrow)) continue;
-          const bool pre = wsrc == RUN_PREFIX;
-          if (!pre && page) continue;  // a page-table read would have to wait
-          const int32_t z = pre ? zpre : s * Hkv + g;
-          if (HALVES == 2 && ma.maps.whole) {
-            ptx::tma_prefetch_l2_4d(pre ? &ma.maps.kpre_w : &ma.maps.kring_w, 0, wrow, 0, z);
-            ptx::tma_prefetch_l2_4d(pre ? &ma.maps.vpre_w : &ma.maps.vring_w, 0, wrow, 0, z);
-          } else {
-            ptx::tma_prefetch_l2_3d(pre ? &ma.maps.kpre[0] : &ma.maps.kring[0], 0, wrow, z);
-            ptx::tma_prefetch_l2_3d(pre ? &ma.maps.vpre[0] : &ma.maps.vring[0], 0, wrow, z);
-          }
-        }
-      }
       for (int32_t k = 0; k < nt && alive; ++k) {
         const int32_t x0 = xs + k * kTR, x1 = min(x0 + kTR, xe);
         const int st = i % kStagesM;
@@ -464,6 +444,7 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
   }
 
   // -------------------------------------------------------------- consumers --
+  if (CL) ptx::cluster_wait();
   auto csync = [&](uint64_t* bar, int phase) -> bool {
     __syncwarp();
     if (lane == 0) ptx::mbar_arrive(bar);

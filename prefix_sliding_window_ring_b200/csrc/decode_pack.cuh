@@ -96,7 +96,8 @@ __host__ __device__ __forceinline__ DecRuns dec_runs(const DevMeta& m, int32_t W
     }
     if (hi >= lo) {
       const int64_t nw = hi - lo + 1;
-      s0 = (int32_t)(((int64_t)m.head + (lo - base)) % W);
+      s0 = m.head + (int32_t)(lo - base);  // head < W and lo - base < W: one wrap at most
+      if (s0 >= W) s0 -= W;
       lenA = (int32_t)(nw < (int64_t)(W - s0) ? nw : (int64_t)(W - s0));
       lenB = (int32_t)(nw - lenA);
     }

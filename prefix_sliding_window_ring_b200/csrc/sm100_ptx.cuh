@@ -111,11 +111,17 @@ __device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_
 __device__ __forceinline__ void fence_acq_rel_cluster() {
   asm volatile("fence.acq_rel.cluster;" ::: "memory");
 }
-// All threads of all CTAs of the cluster (every CTA of a cluster is resident
-// together, so this completes once each has reached it).
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
-               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+// Cluster barrier in two halves (every CTA of a cluster is resident together,
+// so the wait completes once each non-exited thread has arrived).  The
+// aligned forms are executed by whole warps; cluster_wait_one by one thread.
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_one() {
+  asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
 }
 
 // ------------------------------------------- programmatic dependent launch --
@@ -169,22 +175,6 @@ __device__ __forceinline__ void tma_load_4d(void* smem_dst, const void* tmap, in
       "[%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(smem_dst)),
       "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
       : "memory");
-}
-
-// Prefetch of a tensor-map box into L2 (no shared memory, no completion):
-// only warms the cache, so it may run before the grid's dependencies are met.
-__device__ __forceinline__ void tma_prefetch_l2_3d(const void* tmap, int32_t x, int32_t y,
-                                                   int32_t z) {
-  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(tmap),
-               "r"(x), "r"(y), "r"(z)
-               : "memory");
-}
-__device__ __forceinline__ void tma_prefetch_l2_4d(const void* tmap, int32_t x, int32_t y,
-                                                   int32_t z, int32_t w) {
-  asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
-                   tmap),
-               "r"(x), "r"(y), "r"(z), "r"(w)
-               : "memory");
 }
 
 // ------------------------------------------------------------ tensor memory --
