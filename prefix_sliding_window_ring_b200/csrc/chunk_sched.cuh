@@ -37,18 +37,27 @@ __host__ __device__ __forceinline__ void add_range(KSched& s, int src, int64_t r
                                           int64_t len, int64_t page = 0) {
   if (len <= 0) return;
   int64_t first = len;
-  if (page > 0) {
-    const int64_t to_edge = page - row0 % page;
+  if (page > 0) {  // a ring range: row0 is a slot, below 2^28
+    const int64_t to_edge = page - (int32_t)row0 % (int32_t)page;
     first = to_edge < len ? to_edge : len;
   }
-  s.src[s.n] = src;
-  s.row0[s.n] = row0;
-  s.pos0[s.n] = pos0;
-  s.len[s.n] = (int32_t)len;
-  s.first[s.n] = (int32_t)first;
-  s.tfirst[s.n] = (int32_t)((first + kBN - 1) / kBN);
-  s.tbase[s.n] = s.ntiles;
-  s.ntiles += s.tfirst[s.n] + (int32_t)((len - first + kBN - 1) / kBN);
+  const int32_t tfirst = (int32_t)((first + kBN - 1) / kBN);
+  // stored through constant indices (a store at index s.n would put the
+  // schedule in local memory instead of registers)
+  auto put = [&](int k) {
+    s.src[k] = src;
+    s.row0[k] = row0;
+    s.pos0[k] = pos0;
+    s.len[k] = (int32_t)len;
+    s.first[k] = (int32_t)first;
+    s.tfirst[k] = tfirst;
+    s.tbase[k] = s.ntiles;
+  };
+  if (s.n == 0) put(0);
+  if (s.n == 1) put(1);
+  if (s.n == 2) put(2);
+  if (s.n == 3) put(3);
+  s.ntiles += tfirst + (int32_t)((len - first + kBN - 1) / kBN);
   s.n++;
 }
 
@@ -60,6 +69,7 @@ __host__ __device__ __forceinline__ KSched make_sched(const DevMeta& m, int W, i
   KSched s;
   s.n = 0;
   s.ntiles = 0;
+#pragma unroll
   for (int i = 0; i < 4; ++i) {
     s.src[i] = 0; s.row0[i] = 0; s.pos0[i] = 0; s.len[i] = 0;
     s.first[i] = 0; s.tfirst[i] = 0; s.tbase[i] = 0;
@@ -75,7 +85,8 @@ __host__ __device__ __forceinline__ KSched make_sched(const DevMeta& m, int W, i
   int64_t rlo = lo < base ? base : lo;  // never below what the ring holds
   if (t0 - 1 >= rlo) {
     const int64_t nw = t0 - rlo;
-    const int64_t s0 = ((int64_t)m.head + (rlo - base)) % W;
+    int64_t s0 = (int64_t)m.head + (rlo - base);  // head < W, rlo - base < W: one wrap at most
+    if (s0 >= W) s0 -= W;
     const int64_t lenA = nw < W - s0 ? nw : W - s0;
     add_range(s, 0, s0, rlo, lenA, page);
     add_range(s, 0, 0, rlo + lenA, nw - lenA, page);
