@@ -229,6 +229,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
           ptx::mbar_wait_bounded(&v_full[j & 1], (j >> 1) & 1, &quiet, kWaitLimit);
       }
     }
+    __syncwarp();  // the whole warp meets the final block barrier together
   } else if (warp == 1) {
     // --------------------------------------------------------- MMA issuer --
     if (lane == 0) {
@@ -273,6 +274,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
       int quiet = 0;
       ptx::mbar_wait_bounded(&mma_done, 0, &quiet, kWaitLimit);
     }
+    __syncwarp();  // the whole warp meets the final block barrier together
   } else if (warp >= 4) {
     // ------------------------------------------------------------- softmax --
     const int quad = warp & 3;            // TMEM lane quadrant this warp may access
