@@ -84,6 +84,7 @@ constexpr int kStagesM = PS_DMMA_STAGES;
 constexpr int kGroups = kTR / 16;           // 16-row MMA groups per tile
 constexpr int kBox = 64;                    // rows of the large tensor-map box
 constexpr int kMaxCluster = 8;              // CTAs per pair in cluster mode, at most
+constexpr int kTblMax = 256;                // page-table entries staged in shared memory
 static_assert(kTR == 64, "tile rows: 64 (the valid-row mask is one 64-bit word)");
 static_assert(PS_DMMA_CTAS_PER_SM <= kDecMaxCtasPerSm, "workspace slots cover every CTA");
 
@@ -197,6 +198,9 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
   __shared__ int abort_flag;
   __shared__ MergeSmem<G, D, kMW> sm;
   __shared__ float pub_ml[G][2];  // cluster: this CTA's merged (max, sum) per head
+  // paged cache: the page-table row of the piece's sequence (read by the producer only)
+  __shared__ __align__(16) int32_t tbl[kTblMax + 4];
+  __shared__ __align__(8) uint64_t tbl_bar;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Hkv = a.c.Hkv;
@@ -211,6 +215,7 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
     ptx::mbar_init(&sync_c, kMW);
     ptx::mbar_init(&pub_bar, CL ? a.csize - 1 : 1);
     ptx::mbar_init(&done_bar, 1);
+    ptx::mbar_init(&tbl_bar, 1);
     abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -222,6 +227,10 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
       ptx::prefetch_tmap(&ma.maps.vpre[k]);
       ptx::prefetch_tmap(&ma.maps.kring[k]);
       ptx::prefetch_tmap(&ma.maps.vring[k]);
+    }
+    if (ma.maps.page_box) {
+      ptx::prefetch_tmap(&ma.maps.kring_p);
+      ptx::prefetch_tmap(&ma.maps.vring_p);
     }
   }
   __syncthreads();
@@ -245,6 +254,7 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
     int i = 0;  // tiles handed out so far
     bool alive = true;
     bool waited = false;  // griddepcontrol.wait done
+    int tbl_n = 0;        // page-table rows staged so far (the barrier's phase)
     auto wait_primary = [&]() {
       if (!waited) {
         if (CL) ptx::cluster_wait_one();
@@ -277,6 +287,29 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
         xe = min(j1 * kTR, runs.padded);
       }
       const int32_t nt = xe > xs ? (xe - xs + kTR - 1) / kTR : 0;
+      // Paged cache: stage the sequence's page-table row in shared memory with
+      // one bulk copy, so that a page's physical number is a shared-memory read
+      // instead of a dependent global load on this thread.
+      const int32_t* tab = nullptr;  // shared copy, or NULL: read the global table
+      if (page && nt > 0 && a.c.npg <= kTblMax && alive) {
+        wait_primary();  // the table may just have been written by the previous grid
+        const uintptr_t src = (uintptr_t)(a.c.page_table + (int64_t)s * a.c.npg);
+        const uintptr_t src16 = src & ~(uintptr_t)15;
+        const int lead = (int)((src - src16) / 4);
+        const uint32_t bytes = (uint32_t)(((src - src16) + (size_t)a.c.npg * 4 + 15) & ~(size_t)15);
+        if (tbl_n > 0) fence_proxy_async_smem();  // earlier reads before the copy overwrites
+        ptx::mbar_arrive_expect_tx(&tbl_bar, bytes);
+        ptx::bulk_g2s(tbl, (const void*)src16, bytes, &tbl_bar);
+        if (ptx::mbar_wait_bounded(&tbl_bar, tbl_n & 1, &abort_flag, kWaitLimitCycles)) {
+          tab = tbl + lead;
+        } else {
+          alive = false;
+        }
+        ++tbl_n;
+      }
+      auto phys_of = [&](int32_t slot) -> int {
+        return tab ? tab[slot / page] : ring_page(a.c, s, slot);
+      };
       for (int32_t k = 0; k < nt && alive; ++k) {
         const int32_t x0 = xs + k * kTR, x1 = min(x0 + kTR, xe);
         const int st = i % kStagesM;
@@ -306,7 +339,7 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
                           (uint32_t)(G * D * 2), &full[st]);
           const bool pre = wsrc == RUN_PREFIX;
           const int32_t y = pre ? wrow : (page ? wrow % page : wrow);
-          const int32_t z = pre ? zpre : ring_page(a.c, s, wrow) * Hkv + g;
+          const int32_t z = pre ? zpre : phys_of(wrow) * Hkv + g;
           if (HALVES == 2 && ma.maps.whole) {
             ptx::tma_load_4d(kd, pre ? &ma.maps.kpre_w : &ma.maps.kring_w, 0, y, 0, z, &full[st]);
             ptx::tma_load_4d(vd, pre ? &ma.maps.vpre_w : &ma.maps.vring_w, 0, y, 0, z, &full[st]);
@@ -368,7 +401,7 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
             z = zpre;
           } else {  // a ring piece lies within one page
             y = page ? row % page : row;
-            z = ring_page(a.c, s, row) * Hkv + g;
+            z = phys_of(row) * Hkv + g;
           }
           // copy whole atoms, from the one that holds the piece's first row
           // (its row or slot minus the offset within the atom: same page)
@@ -376,6 +409,17 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
           sr -= lead;
           y -= lead;
           n += lead;
+          if (src == RUN_RING && ma.maps.page_box && lead == 0 && n == page) {
+            // a whole small page: one box per column block
+#pragma unroll
+            for (int h = 0; h < HALVES; ++h) {
+              ptx::tma_load_3d(kd + h * kHalfBytes + sr * 128, &ma.maps.kring_p, h * 64, y, z,
+                               &full[st]);
+              ptx::tma_load_3d(vd + h * kHalfBytes + sr * 128, &ma.maps.vring_p, h * 64, y, z,
+                               &full[st]);
+            }
+            return;
+          }
           while (n > 0) {
             const bool big = n >= kBox;
             const int32_t rows = big ? kBox : kPadRows;
@@ -834,6 +878,14 @@ bool make_decode_maps(const CacheDev& c, DecodeMaps* m) {
   // block, slab); the column block is the outer box dimension, so one copy
   // writes the tile's two 64-column blocks one after the other, as the kernel
   // lays them out.
+  m->page_box = 0;
+  if (ok && c.page_table && c.page_rows >= 16 && c.page_rows < kBox && c.page_rows % kPadRows == 0) {
+    const int pr = PS_DMMA_L2_PROMOTION;
+    m->page_box = encode_map3d_bf16(&m->kring_p, kring, c.d, (uint64_t)c.page_rows, nring, row,
+                                    (uint64_t)c.rstride * row, 64, (uint32_t)c.page_rows, 1, pr) &&
+                  encode_map3d_bf16(&m->vring_p, vring, c.d, (uint64_t)c.page_rows, nring, row,
+                                    (uint64_t)c.rstride * row, 64, (uint32_t)c.page_rows, 1, pr);
+  }
   m->whole = 0;
   if (ok && c.d == 128) {
     const uint32_t box[4] = {64, (uint32_t)kBox, 2, 1};

@@ -71,7 +71,11 @@ size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int sm_count);
 struct DecodeMaps {
   CUtensorMap kpre[2], vpre[2], kring[2], vring[2];
   CUtensorMap kpre_w, vpre_w, kring_w, vring_w;
-  int whole;  // 1 if the whole-tile maps exist (head_dim 128)
+  // paged caches with pages of 16..56 rows (a multiple of 8): a box of one
+  // page of one 64-column block
+  CUtensorMap kring_p, vring_p;
+  int whole;     // 1 if the whole-tile maps exist (head_dim 128)
+  int page_box;  // 1 if the one-page maps exist
 };
 bool make_decode_maps(const CacheDev& c, DecodeMaps* m);
 // maps: the cache's decode maps (bf16 caches; NULL for float32).
