@@ -415,31 +415,38 @@ def run_ours(args, rank, world, local_rank):
               for d in din2]
     hout2 = [hout, torch.empty_like(hout).pin_memory()]
     s2 = torch.cuda.Stream()
-    sc = torch.cuda.Stream()
-    s2.wait_stream(torch.cuda.current_stream())
-    sc.wait_stream(torch.cuda.current_stream())
+    s_in = torch.cuda.Stream()   # uploads
+    s_out = torch.cuda.Stream()  # read-backs (the other copy direction, concurrently)
+    for x_ in (s2, s_in, s_out):
+        x_.wait_stream(torch.cuda.current_stream())
     g2 = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g2, stream=s2):
-        sc.wait_stream(s2)
+        s_in.wait_stream(s2)
+        s_out.wait_stream(s2)
         ev_in = [torch.cuda.Event() for _ in range(K)]
         ev_dec = [torch.cuda.Event() for _ in range(K)]
+        ev_out = [torch.cuda.Event() for _ in range(K)]
         for i in range(K):
             b = i % 2
             r = (base + i) % ROT
             v = wl.visit[r]
-            with torch.cuda.stream(sc):
+            with torch.cuda.stream(s_in):
                 if i >= 2:
-                    sc.wait_event(ev_dec[i - 2])  # input buffer b is free again
+                    s_in.wait_event(ev_dec[i - 2])  # input buffer b is free again
                 din2[b].copy_(hin[r][v], non_blocking=True)
-                ev_in[i].record(sc)
+                ev_in[i].record(s_in)
             s2.wait_event(ev_in[i])
+            if i >= 2:
+                s2.wait_event(ev_out[i - 2])  # output buffer b has been read back
             qv, kv_, vv = dviews[b]
             out = wl.step(base + i, s2, host=lambda r_, v_: (kv_, vv, qv))
             ev_dec[i].record(s2)
-            with torch.cuda.stream(sc):
-                sc.wait_event(ev_dec[i])
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_dec[i])
                 hout2[b].copy_(out, non_blocking=True)
-        s2.wait_stream(sc)
+                ev_out[i].record(s_out)
+        s2.wait_stream(s_in)
+        s2.wait_stream(s_out)
     torch.cuda.synchronize()
     upload_graph(torch, g2, s2)
     if dist:
@@ -510,7 +517,7 @@ def run_ours(args, rank, world, local_rank):
                 "copies": "one upload of a pinned [q | k | v] record and one read-back of the "
                           "output per step, on the decode stream",
                 "issue": "the K steps (upload, ps_decode_step, read-back) captured into one "
-                         "CUDA graph and replayed; uploads and read-backs on a second stream, "
+                         "CUDA graph and replayed; uploads and read-backs on two more streams, "
                          "double-buffered, overlapping the neighbouring steps' kernels",
                 "eager": {"value": round(e2e_eager, 1), "unit": UNIT,
                           "issue": "the same steps issued one by one from Python"}},
