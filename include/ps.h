@@ -23,9 +23,18 @@
  *    stream) and is asynchronous unless stated otherwise.  Calls that touch
  *    the same cache must be ordered on one stream (or by the caller's events).
  *  - Every argument, sequence state and position is validated on the host
- *    BEFORE anything is enqueued.  A call that returns an error has changed
- *    neither the device memory nor the host-side state; the message is
- *    available from ps_last_error() in the calling thread.
+ *    BEFORE anything is enqueued.  A call that returns an error other than
+ *    PS_ECUDA has changed neither the device memory nor the host-side state;
+ *    the message is available from ps_last_error() in the calling thread.
+ *  - PS_ECUDA is the one partial outcome.  Some calls enqueue more than one
+ *    launch: a paged ring's page-table update before an append, and one
+ *    launch per 128 batch entries in ps_append_kv, ps_decode_step and
+ *    ps_attend_decode (one append per entry in ps_attend_chunk_batch with
+ *    append_after).  If a launch fails, the launches before it stay enqueued
+ *    and the host-side state records exactly them: mapped pages stay mapped,
+ *    the entries whose append was enqueued are advanced, the others are
+ *    unchanged, and outputs of entries not yet launched are not written.  A
+ *    failed launch usually leaves the CUDA context unusable in any case.
  *  - The library owns only the opaque host object.  All device storage lives
  *    in the caller's buffer passed to ps_cache_create; decode scratch lives in
  *    the caller's workspace passed to ps_attend_decode / ps_decode_step (or in

@@ -161,6 +161,18 @@ void advance(SeqHost& s, int W, int64_t n) {
   s.next_pos += n;
 }
 
+// Records a planned page-table update once its launch is enqueued.  Host
+// state follows what is enqueued: if a later launch of the same call fails,
+// the mapped pages stay mapped on both sides (the next append that reaches
+// them finds them mapped).
+void commit_pages(ps_cache* c, const int* seq_ids, int B,
+                  const std::vector<std::vector<int32_t>>& pages,
+                  const std::vector<int32_t>& avail) {
+  if (!c->paged) return;
+  c->free_pages = avail;
+  for (int b = 0; b < B; ++b) c->seqs[seq_ids[b]].pages = pages[b];
+}
+
 ps::DevMeta to_dev(const SeqHost& s) {
   ps::DevMeta m;
   memset(&m, 0, sizeof(m));
@@ -271,6 +283,7 @@ static int attend_blocks(ps_cache* c, const int* seq_ids, const int64_t* t0, con
   if (append_after && !prompt) {
     if (!idx.empty())
       PS_CUDA(ps::launch_page_set(c->dev, idx.data(), phys.data(), (int)idx.size(), st));
+    commit_pages(c, seq_ids, B, pages, avail);
     int64_t tok = 0;
     for (int b = 0; b < B; ++b) {
       if (n[b] > 0) {
@@ -279,13 +292,9 @@ static int attend_blocks(ps_cache* c, const int* seq_ids, const int64_t* t0, con
         ids.seq[0] = seq_ids[b];
         PS_CUDA(ps::launch_ring_append(c->dev, c->esize, ids, 1, (const char*)k_blk + tok * krow,
                                        (const char*)v_blk + tok * krow, n[b], st));
+        advance(c->seqs[seq_ids[b]], c->W, n[b]);
       }
       tok += n[b];
-    }
-    c->free_pages = avail;
-    for (int b = 0; b < B; ++b) {
-      c->seqs[seq_ids[b]].pages = pages[b];
-      advance(c->seqs[seq_ids[b]], c->W, n[b]);
     }
   }
   return ok();
@@ -499,6 +508,7 @@ int ps_append_kv(ps_cache* c, const int* seq_ids, int B, const void* k, const vo
   cudaStream_t st = (cudaStream_t)stream;
   if (!idx.empty())
     PS_CUDA(ps::launch_page_set(c->dev, idx.data(), phys.data(), (int)idx.size(), st));
+  commit_pages(c, seq_ids, B, pages, avail);
   size_t per_entry = (size_t)n * c->Hkv * c->d * c->esize;
   for (int b0 = 0; b0 < B; b0 += ps::kMaxBatchPerLaunch) {
     int nb = B - b0 < ps::kMaxBatchPerLaunch ? B - b0 : ps::kMaxBatchPerLaunch;
@@ -507,11 +517,7 @@ int ps_append_kv(ps_cache* c, const int* seq_ids, int B, const void* k, const vo
     for (int i = 0; i < nb; ++i) ids.seq[i] = seq_ids[b0 + i];
     PS_CUDA(ps::launch_ring_append(c->dev, c->esize, ids, nb, (const char*)k + b0 * per_entry,
                                    (const char*)v + b0 * per_entry, n, st));
-  }
-  c->free_pages = avail;
-  for (int b = 0; b < B; ++b) {
-    c->seqs[seq_ids[b]].pages = pages[b];
-    advance(c->seqs[seq_ids[b]], c->W, n);
+    for (int i = 0; i < nb; ++i) advance(c->seqs[seq_ids[b0 + i]], c->W, n);
   }
   return ok();
 }
@@ -598,6 +604,7 @@ int ps_decode_step(ps_cache* c, const void* q, const void* k_new, const void* v_
   cudaStream_t st = (cudaStream_t)stream;
   if (!idx.empty())
     PS_CUDA(ps::launch_page_set(c->dev, idx.data(), phys.data(), (int)idx.size(), st));
+  commit_pages(c, seq_ids, B, pages, avail);
   const size_t per_entry = (size_t)Hq * c->d * c->esize;
   const size_t per_row = (size_t)c->Hkv * c->d * c->esize;
   for (int b0 = 0; b0 < B; b0 += ps::kMaxBatchPerLaunch) {
@@ -618,11 +625,7 @@ int ps_decode_step(ps_cache* c, const void* q, const void* k_new, const void* v_
                               (const char*)k_new + b0 * per_row, (const char*)v_new + b0 * per_row,
                               (char*)out + b0 * per_entry, scale, ws, c->sm_count,
                               c->dtype == PS_BF16 ? &c->dmaps : nullptr, st));
-  }
-  c->free_pages = avail;
-  for (int b = 0; b < B; ++b) {
-    c->seqs[seq_ids[b]].pages = pages[b];
-    advance(c->seqs[seq_ids[b]], c->W, 1);
+    for (int i = 0; i < nb; ++i) advance(c->seqs[seq_ids[b0 + i]], c->W, 1);
   }
   return ok();
 }
@@ -689,12 +692,13 @@ int ps_import_window(ps_cache* c, int seq, int64_t next_pos, const void* k, cons
   if (!idx.empty())
     PS_CUDA(ps::launch_page_set(c->dev, idx.data(), phys.data(), (int)idx.size(),
                                 (cudaStream_t)stream));
+  c->free_pages = avail;  // the page-table update is enqueued
+  c->seqs[seq].pages = s.pages;
   s.next_pos = next_pos;
   s.head = ring_head_offset;
   s.count = n;
   PS_CUDA(ps::launch_ring_import(c->dev, c->esize, seq, to_dev(s), k, v, n,
                                  (cudaStream_t)stream));
-  c->free_pages = avail;
   c->seqs[seq] = s;
   return ok();
 }
