@@ -638,6 +638,68 @@ def prefill_measure(steps: int):
 PR_P = 4096  # prompt length of the prompt-prefill measurement
 
 
+def chunk_small_measure(steps: int):
+    """Small chunk blocks: the split decode path against the chunk kernel.
+    The chunk workload's shape (Hq=16, Hkv=8, d=128, P=256, W=4096, t0=100000,
+    window full) with blocks of n queries for B = 1 and 4 sequences, each
+    block size timed with the small-block bound at 0 (chunk kernel) and above
+    n (split decode).  16 sequences' caches (285 MB, larger than L2) are
+    rotated, a batch per step.  One step = one ps_attend_chunk_batch call."""
+    import torch
+
+    import synth
+    from prefix_sliding_window_ring_b200 import PS_BF16, Cache
+
+    def dev(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+
+    Wp, nseq = 4096, 16
+    c = Cache(Wp, PF_P, HKV, D, PS_BF16, nseq)
+    for s in range(nseq):
+        c.seq_reset(s, 0)
+        c.prefill_prefix(s, dev(synth.rows(SEED, synth.TID_K, s, HKV, 0, PF_P, D, "bf16")),
+                         dev(synth.rows(SEED, synth.TID_V, s, HKV, 0, PF_P, D, "bf16")), PF_P)
+        c.import_window(s, PF_T0,
+                        dev(synth.rows(SEED, synth.TID_K, s, HKV, PF_T0 - Wp, Wp, D, "bf16")),
+                        dev(synth.rows(SEED, synth.TID_V, s, HKV, PF_T0 - Wp, Wp, D, "bf16")),
+                        Wp, (977 * s) % Wp)
+    scale = 1.0 / math.sqrt(D)
+    nmax = 64
+    q = dev(synth.rows(SEED, synth.TID_Q, 0, HQ, PF_T0, 4 * nmax, D, "bf16"))
+    kb = dev(synth.rows(SEED, synth.TID_K, 0, HKV, PF_T0, 4 * nmax, D, "bf16"))
+    vb = dev(synth.rows(SEED, synth.TID_V, 0, HKV, PF_T0, 4 * nmax, D, "bf16"))
+    o = torch.empty_like(q)
+    res = {"workload": f"blocks of n queries at t0={PF_T0}, Hq={HQ} Hkv={HKV} d={D} P={PF_P} "
+                       f"W={Wp}, bf16; 16 caches rotated (larger than L2)",
+           "unit": "us per call", "rows": []}
+    for B in (1, 4):
+        for n in (1, 2, 3, 4, 8, 12, 16, 24, 32, 48, 64):
+            row = {"B": B, "n": n}
+            for name, bound in (("chunk_kernel", 0), ("split_decode", 1 << 20)):
+                c.set_chunk_small_max(bound)
+
+                def step(i, st=None):
+                    ids = [((i % (nseq // B)) * B + b) for b in range(B)]
+                    c.attend_chunk_batch(ids, [PF_T0] * B, [n] * B, q[:B * n], kb[:B * n],
+                                         vb[:B * n], HQ, scale, o[:B * n], 0, st)
+
+                for i in range(3):
+                    step(i)
+                torch.cuda.synchronize()
+                if c.device_error():
+                    raise RuntimeError("device error word set by a chunk call")
+                ms = min(time_graph(torch, step, steps) for _ in range(2))
+                row[name] = round(ms * 1e3, 2)
+            res["rows"].append(row)
+    c.set_chunk_small_max(0)
+    for B in (1, 4):
+        rows = [r for r in res["rows"] if r["B"] == B]
+        faster = [r["n"] for r in rows if r["split_decode"] < r["chunk_kernel"]]
+        res[f"split_faster_up_to_B{B}"] = max(faster) if faster else 0
+    c.close()
+    return res
+
+
 def prompt_measure(steps: int, peak: float):
     """Prompt prefill (queries inside the pinned prefix, causal over it) on the
     tensor-core kernel: 4 sequences with a 4096-token prompt each, one
@@ -1076,7 +1138,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--only", choices=["prefill", "prompt", "ragged", "shared", "paged", "t_sweep",
-                                       "gqa"],
+                                       "gqa", "chunk_small"],
                     help="run one side measurement alone and print its record (for profiling "
                          "one kernel under ncu); not a benchmark line")
     args = ap.parse_args()
@@ -1093,6 +1155,7 @@ def main():
               "shared": shared_prefix_measure, "paged": paged_measure,
               "t_sweep": lambda n: t_sweep_measure(max(n, 16)),
               "gqa": lambda n: gqa_measure(max(n, 16)),
+              "chunk_small": lambda n: chunk_small_measure(max(n, 10)),
               "prompt": lambda n: prompt_measure(n, load_bf16_peak()[0])}[args.only]
         print(json.dumps({"only": args.only, "result": fn(k)}), flush=True)
     elif args.impl == "reference":

@@ -108,8 +108,10 @@ PS_API int ps_cache_create(int W, int P_max, int Hkv, int d, int dtype, int max_
  * append or window import first writes one of its slots, and returns to the
  * pool when the sequence is reset; so memory follows the tokens actually held
  * rather than max_seqs * W.  Every call behaves exactly as on an unpaged cache
- * (same results, bit for bit), except that a write needing a page when the
- * pool is empty fails with PS_ENOMEM and changes nothing.  Requires
+ * (same results, bit for bit, when page_rows is a multiple of 8; with other
+ * page sizes the bf16 decode groups a tile's rows page by page, which changes
+ * the float32 summation order only), except that a write needing a page when
+ * the pool is empty fails with PS_ENOMEM and changes nothing.  Requires
  * 1 <= page_rows <= W, W % page_rows == 0, num_pages >= 1; the tensor-core
  * chunk kernel needs page_rows % 128 == 0 (other page sizes use the CUDA-core
  * chunk kernel).  ps_cache_bytes_paged returns 0 for an invalid shape. */
@@ -273,11 +275,29 @@ PS_API int ps_attend_decode_static(ps_cache* c, const void* q, const int* seq_id
  * true before the block is appended.  If append_after != 0 the block is then
  * appended as by ps_append_kv (only its last W tokens survive in the ring).
  * bf16 with d = 128 and Hq/Hkv in {1, 2, 4, 8} runs on the tcgen05 tensor-core
- * kernel; other configurations use a CUDA-core kernel.
+ * kernel; other configurations use a CUDA-core kernel.  Small bf16 blocks
+ * (d = 64 or 128) run instead on the decode kernel when the call qualifies
+ * (ps_set_chunk_small_max): groups of 8 / (Hq/Hkv) queries, each group's
+ * (query, head) pairs as the narrow side of the warp-level products, every
+ * query masked to its own visible set, the key rows of a (group, kv head)
+ * pair split over a cluster of CTAs.
  * Errors: PS_EINVAL, PS_ESTATE, PS_EPOS, PS_EUNSUPPORTED. */
 PS_API int ps_attend_chunk(ps_cache* c, int seq, const void* q, const void* k_blk,
                     const void* v_blk, int64_t t0, int n, int Hq, float scale, void* out,
                     int append_after, void* stream);
+
+/* Small-block bound of the chunk calls (bf16 caches).  A ps_attend_chunk or
+ * ps_attend_chunk_batch call runs on the split decode path when every block
+ * of it has at most n_max queries and its (group of 8 / (Hq/Hkv) queries, kv
+ * head) pairs all fit the GPU at once in clusters of two CTAs (148 on a B200:
+ * e.g. 4 blocks of 16 queries at Hq/Hkv = 2, Hkv = 8); otherwise the whole
+ * call runs on the chunk kernels.  Inside those limits the split path was
+ * measured faster at every block size (W = 4096, one and four sequences); 0
+ * sends every call to the chunk kernels.  The split path's partition, and so
+ * its float32 summation order, follows the call's size, as the decode calls'
+ * does.  Default 64.
+ * Errors: PS_EINVAL (NULL cache, n_max < 0). */
+PS_API int ps_set_chunk_small_max(ps_cache* c, int n_max);
 
 /* Chunked prefill/extend of B sequences in one launch (batched serving):
  * entry b is as ps_attend_chunk for sequence seq_ids[b] (host array of

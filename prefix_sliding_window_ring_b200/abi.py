@@ -46,6 +46,7 @@ SIGNATURES = {
     "ps_attend_decode_static": (_i, [_vp, _vp, _vp, _vp, _i, _i, _f, _vp, _vp]),
     "ps_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _f, _vp, _vp, _sz, _vp]),
     "ps_attend_chunk": (_i, [_vp, _i, _vp, _vp, _vp, _i64, _i, _i, _f, _vp, _i, _vp]),
+    "ps_set_chunk_small_max": (_i, [_vp, _i]),
     "ps_attend_prompt": (_i, [_vp, _i, _vp, _i64, _i, _i, _f, _vp, _vp]),
     "ps_attend_chunk_batch": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _i, _f, _vp, _i, _vp]),
     "ps_attend_prompt_batch": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _i, _f, _vp, _vp]),
@@ -214,6 +215,10 @@ def ps_attend_chunk(cache, seq, q, k_blk, v_blk, t0, n, Hq, scale, out, append_a
     _check("ps_attend_chunk", _lib.ps_attend_chunk(cache, seq, _ptr(q), _ptr(k_blk), _ptr(v_blk),
                                                    t0, n, Hq, scale, _ptr(out), int(append_after),
                                                    _stream(stream)))
+
+
+def ps_set_chunk_small_max(cache, n_max) -> None:
+    _check("ps_set_chunk_small_max", _lib.ps_set_chunk_small_max(cache, int(n_max)))
 
 
 def _entries(seq_ids, t0, n):

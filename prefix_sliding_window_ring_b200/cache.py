@@ -84,6 +84,9 @@ class Cache:
         abi.ps_attend_chunk(self.handle, seq, q, k_blk, v_blk, t0, n, Hq, scale, out, append_after,
                             stream)
 
+    def set_chunk_small_max(self, n_max):
+        abi.ps_set_chunk_small_max(self.handle, n_max)
+
     def attend_chunk_batch(self, seq_ids, t0, n, q, k_blk, v_blk, Hq, scale, out, append_after=0,
                            stream=None):
         abi.ps_attend_chunk_batch(self.handle, seq_ids, t0, n, q, k_blk, v_blk, Hq, scale, out,

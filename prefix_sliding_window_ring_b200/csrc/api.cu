@@ -103,6 +103,7 @@ struct ps_cache {
   int sm_count;
   ps::CacheDev dev;
   ps::DecodeMaps dmaps;  // bf16 caches: tensor maps of K/V for the decode kernel
+  int chunk_small_max;   // chunk blocks of at most this many queries: split decode path
   std::vector<SeqHost> seqs;
 };
 
@@ -243,6 +244,66 @@ static int attend_blocks(ps_cache* c, const int* seq_ids, const int64_t* t0, con
   }
   cudaStream_t st = (cudaStream_t)stream;
   const size_t qrow = (size_t)Hq * c->d * c->esize, krow = (size_t)c->Hkv * c->d * c->esize;
+  // Small blocks (bf16): groups of a few queries on the tensor-core decode
+  // kernel, split over the whole GPU, instead of one 128-row query tile per
+  // kv head on the chunk kernel.
+  // The whole call takes it when every block is small and their (group, kv
+  // head) pairs all fit the GPU at once in clusters of two CTAs; otherwise
+  // the chunk kernel's launch takes the small blocks along (its CTAs run
+  // them in the same waves).
+  std::vector<char> small(B, 0);
+  if (!prompt && c->dtype == PS_BF16 && c->chunk_small_max > 0) {
+    int nmax = 0;
+    int64_t pairs = 0;
+    bool all_small = true;
+    for (int b = 0; b < B; ++b) {
+      if (n[b] == 0) continue;
+      if (n[b] > c->chunk_small_max) all_small = false;
+      nmax = n[b] > nmax ? n[b] : nmax;
+      pairs += (int64_t)((n[b] + 8 / G - 1) / (8 / G)) * c->Hkv;
+    }
+    if (!all_small || nmax == 0 || pairs > ps::chunk_small_pair_capacity(c->d)) nmax = 0;
+    for (int b = 0; b < B; ++b) small[b] = nmax > 0 && n[b] > 0;
+    if (nmax > 0) {
+      // groups of Q = 8 / G queries: the kernel's 8 columns hold a group's
+      // queries x G heads.  Fixed, like the kernel's cluster split, so that an
+      // entry's result does not depend on the rest of the batch.
+      const int cols = 8;
+      const int Q = cols / G;
+      std::vector<ps::SmallChunkEntry> es;
+      auto flush = [&]() -> cudaError_t {
+        if (es.empty()) return cudaSuccess;
+        cudaError_t e = ps::launch_chunk_small_batch(c->dev, cols, G, es.data(), (int)es.size(), Hq,
+                                                     q, k_blk, v_blk, N, out, scale, c->sm_count,
+                                                     c->dmaps, st);
+        es.clear();
+        return e;
+      };
+      int64_t tok = 0;
+      for (int b = 0; b < B; ++b) {
+        if (small[b]) {
+          const SeqHost& sh = c->seqs[seq_ids[b]];
+          for (int i0 = 0; i0 < n[b]; i0 += Q) {
+            ps::SmallChunkEntry e;
+            e.seq = seq_ids[b];
+            e.P = sh.P;
+            e.head = sh.head;
+            e.count = sh.count;
+            e.owner = sh.owner;
+            e.t0 = t0[b];
+            e.i0 = i0;
+            e.nq = n[b] - i0 < Q ? n[b] - i0 : Q;
+            e.qrow = (int32_t)(tok + i0);
+            e.brow = (int32_t)tok;
+            es.push_back(e);
+            if ((int)es.size() == ps::kMaxBatchPerLaunch) PS_CUDA(flush());
+          }
+        }
+        tok += n[b];
+      }
+      PS_CUDA(flush());
+    }
+  }
   if (ps::chunk_tc_supported(c->dev, c->dtype, c->d, G)) {
     // entries with queries, in launches of at most kMaxChunkBatch
     std::vector<ps::ChunkEntry> es;
@@ -258,12 +319,14 @@ static int attend_blocks(ps_cache* c, const int* seq_ids, const int64_t* t0, con
       return e;
     };
     for (int b = 0; b < B; ++b) {
-      if (n[b] > 0) {
+      if (n[b] > 0 && !small[b]) {
         if (es.empty()) tok_first = tok;
         const SeqHost& sh = c->seqs[seq_ids[b]];
         es.push_back(ps::ChunkEntry{seq_ids[b], n[b], t0[b], sh.next_pos, sh.P, sh.head, sh.count,
                                     sh.owner});
         if ((int)es.size() == ps::kMaxChunkBatch) PS_CUDA(flush());
+      } else if (small[b]) {
+        PS_CUDA(flush());  // a launch's entries are consecutive in the packed rows
       }
       tok += n[b];
     }
@@ -271,7 +334,7 @@ static int attend_blocks(ps_cache* c, const int* seq_ids, const int64_t* t0, con
   } else {
     int64_t tok = 0;
     for (int b = 0; b < B; ++b) {
-      if (n[b] > 0)
+      if (n[b] > 0 && !small[b])
         PS_CUDA(ps::launch_chunk_cc(
             c->dev, c->dtype, G, seq_ids[b], t0[b], n[b], Hq, (const char*)q + tok * qrow,
             prompt ? nullptr : (const char*)k_blk + tok * krow,
@@ -360,6 +423,7 @@ int create_cache(int W, int P_max, int Hkv, int d, int dtype, int max_seqs, int 
     delete c;
     return fail(PS_ECUDA, "tensor-map encoding of the cache's K/V failed");
   }
+  c->chunk_small_max = ps::kChunkSmallMaxDefault;
   SeqHost empty{0, 0, 0, 0, 0};
   if (paged) {
     empty.pages.assign(c->dev.npg, -1);
@@ -627,6 +691,13 @@ int ps_decode_step(ps_cache* c, const void* q, const void* k_new, const void* v_
                               c->dtype == PS_BF16 ? &c->dmaps : nullptr, st));
     for (int i = 0; i < nb; ++i) advance(c->seqs[seq_ids[b0 + i]], c->W, 1);
   }
+  return ok();
+}
+
+int ps_set_chunk_small_max(ps_cache* c, int n_max) {
+  if (!c) return fail(PS_EINVAL, "cache is NULL");
+  if (n_max < 0) return fail(PS_EINVAL, "negative n_max=%d", n_max);
+  c->chunk_small_max = n_max;
   return ok();
 }
 

@@ -688,4 +688,39 @@ cudaError_t launch_decode(const CacheDev& c, int dtype, int G, const BatchIds& i
   return launch_decode_mma(a, G, *maps, sm_count, st);
 }
 
+cudaError_t launch_chunk_small_batch(const CacheDev& c, int cols, int gq,
+                                     const SmallChunkEntry* e, int B, int Hq, const void* q,
+                                     const void* k_blk, const void* v_blk, int64_t blk_rows,
+                                     void* out, float scale, int sm_count, const DecodeMaps& maps,
+                                     cudaStream_t st) {
+  if (B < 1 || B > kMaxBatchPerLaunch || gq < 1 || cols != 8 || cols % gq)
+    return cudaErrorInvalidValue;
+  DecodeArgs a;
+  memset(&a, 0, sizeof(a));
+  a.c = c;
+  a.q = q;
+  a.out = out;
+  a.qscale = scale * kLog2e;
+  a.Hq = Hq;
+  a.B = B;
+  ChunkArgs ch;
+  memset(&ch, 0, sizeof(ch));
+  ch.gq = gq;
+  ch.lgq = gq == 8 ? 3 : gq == 4 ? 2 : gq == 2 ? 1 : 0;
+  for (int b = 0; b < B; ++b) {
+    if (e[b].nq < 1 || e[b].nq * gq > cols) return cudaErrorInvalidValue;
+    a.seq[b] = e[b].seq;
+    a.P[b] = e[b].P;
+    a.head[b] = e[b].head;
+    a.count[b] = e[b].count;
+    a.owner[b] = e[b].owner;
+    a.t[b] = e[b].t0 + e[b].i0;
+    ch.i0[b] = e[b].i0;
+    ch.nq[b] = e[b].nq;
+    ch.qrow[b] = e[b].qrow;
+    ch.brow[b] = e[b].brow;
+  }
+  return launch_chunk_small(a, ch, maps, k_blk, v_blk, blk_rows, sm_count, st);
+}
+
 }  // namespace ps

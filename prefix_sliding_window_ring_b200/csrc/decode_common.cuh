@@ -48,6 +48,22 @@ struct DecodeArgs {
   int64_t t[kMaxBatchPerLaunch];
   int32_t tcum[kMaxBatchPerLaunch + 1];  // tcum[b] = Hkv * (tiles per head of entries before b)
 };
+
+// Chunk mode of the tensor-core kernel (small chunk blocks; cluster mode):
+// entry b of the launch's DecodeArgs is a group of nq[b] consecutive queries
+// of a block, the first at position t[b], the i0[b]-th of its block (the ring
+// state is the one before the block); the block's rows start at row brow[b]
+// of the launch's block buffers, the group's q / out rows at row qrow[b].  The
+// kernel's G columns hold the group's queries x gq heads (query k, head h in
+// column k gq + h).  A separate kernel instantiation, so the decode kernels
+// carry none of it.
+struct ChunkArgs {
+  int gq, lgq;  // query heads per kv head, and its log2
+  int32_t qrow[kMaxBatchPerLaunch];
+  int32_t nq[kMaxBatchPerLaunch];
+  int32_t i0[kMaxBatchPerLaunch];
+  int32_t brow[kMaxBatchPerLaunch];
+};
 // Kernel parameters above 4 KB need CUDA 12.1 and sm_70 or later (limit 32764 bytes).
 static_assert(sizeof(DecodeArgs) <= 32764, "decode arguments fit the kernel parameter space");
 
@@ -89,6 +105,7 @@ enum : int32_t {
   TD_LAST = 2,   // last tile of a piece
   TD_END = 4,    // no more tiles
   TD_NEW = 8,    // the tile's last row is the appended token (decode step)
+  TD_QMASK = 16, // chunk mode: per-row query masks in the descriptor
 };
 
 // Pair merge: one thread per four consecutive output elements of one pair.
@@ -181,5 +198,10 @@ cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t st) {
 // decode_mma.cu: the tensor-core streaming kernel (bfloat16) and its merge.
 cudaError_t launch_decode_mma(const dec::DecodeArgs& a, int G, const DecodeMaps& maps,
                               int sm_count, cudaStream_t st);
+// The same kernel in chunk mode (8 columns, cluster mode): block rows from
+// k_blk / v_blk ([blk_rows][Hkv][d], 16-byte aligned).
+cudaError_t launch_chunk_small(const dec::DecodeArgs& a, const dec::ChunkArgs& ch,
+                               const DecodeMaps& maps, const void* k_blk, const void* v_blk,
+                               int64_t blk_rows, int sm_count, cudaStream_t st);
 
 }  // namespace ps

@@ -86,19 +86,33 @@ constexpr int kBox = 64;                    // rows of the large tensor-map box
 constexpr int kMaxCluster = 8;              // CTAs per pair in cluster mode, at most
 constexpr int kTblMax = 256;                // page-table entries staged in shared memory
 static_assert(kTR == 64, "tile rows: 64 (the valid-row mask is one 64-bit word)");
+constexpr float kMaxFloor = -1e30f;         // running max of a column before its first row
 static_assert(PS_DMMA_CTAS_PER_SM <= kDecMaxCtasPerSm, "workspace slots cover every CTA");
 
 struct MmaDecodeArgs {
   DecodeMaps maps;  // first: tensor maps must be 64-byte aligned
   DecodeArgs a;
 };
+struct MmaChunkArgs {
+  DecodeMaps maps;
+  // the launch's block rows k_blk / v_blk [rows][Hkv][D], boxes of 8 rows of
+  // one 64-column block of one kv head
+  CUtensorMap kblk, vblk;
+  DecodeArgs a;
+  ChunkArgs ch;
+};
 static_assert(sizeof(MmaDecodeArgs) <= 32764, "decode arguments fit the kernel parameter space");
+static_assert(sizeof(MmaChunkArgs) <= 32764, "chunk arguments fit the kernel parameter space");
+template <bool CHUNK> struct MmaArgsOf { using type = MmaDecodeArgs; };
+template <> struct MmaArgsOf<true> { using type = MmaChunkArgs; };
+template <bool CHUNK> using MmaArgs = typename MmaArgsOf<CHUNK>::type;
 
 struct TileDescM {
   uint32_t mask[kTR / 32];  // valid rows: bit r % 32 of word r / 32
   int32_t pair, flags;
   int32_t slot;             // partial-result slot of the piece: CTA range + pair
   int32_t new_row;          // TD_NEW: tile row of the appended token
+  uint8_t qv[kTR];          // TD_QMASK: bit k of row r set if the group's query k sees it
 };
 
 // ------------------------------------------------------------- warp MMA --
@@ -143,9 +157,12 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 // Online-softmax state of one consumer lane: lane (g, t) holds, for the
-// query heads 2t and 2t+1, the running max m (log2 units; +inf for a padding
-// head, which then gets weight 0), its partial sum l over the rows it has
-// seen, and O^T rows d = 16 mt + g and 16 mt + g + 8 of both heads.
+// columns 2t and 2t+1 (query heads; in chunk mode query x head), the running
+// max m (log2 units; +inf for a padding column, which then gets weight 0; a
+// valid column starts at the finite floor kMaxFloor, so that a column whose
+// rows so far were all masked gets weight ex2(-inf - floor) = 0, not NaN), its
+// partial sum l over the rows it has seen, and O^T rows d = 16 mt + g and
+// 16 mt + g + 8 of both columns.
 template <int D, int G>
 struct MmaState {
   static constexpr int KS = D / 16;  // k-steps of S^T, m-tiles of O^T
@@ -153,35 +170,39 @@ struct MmaState {
   float o[KS][4];
   float m[2], l[2];
 
-  __device__ __forceinline__ void init(const uint8_t* qs) {
+  // ncols: valid columns (<= G); the others are padding
+  __device__ __forceinline__ void init(const uint8_t* qs, int ncols) {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
 #pragma unroll
     for (int ks = 0; ks < KS; ++ks) {
-      // heads g >= G are padding: zero columns of Q^T (their q rows are not loaded)
-      const uint8_t* row = qs + (size_t)(g < G ? g : 0) * D * 2 + (size_t)(16 * ks + 2 * t) * 2;
+      // columns g >= ncols are padding: zero columns of Q^T (their q rows are not loaded)
+      const uint8_t* row = qs + (size_t)(g < ncols ? g : 0) * D * 2 + (size_t)(16 * ks + 2 * t) * 2;
       const uint32_t lo = *(const uint32_t*)row, hi = *(const uint32_t*)(row + 16);
-      qf[ks][0] = g < G ? lo : 0u;
-      qf[ks][1] = g < G ? hi : 0u;
+      qf[ks][0] = g < ncols ? lo : 0u;
+      qf[ks][1] = g < ncols ? hi : 0u;
 #pragma unroll
       for (int e = 0; e < 4; ++e) o[ks][e] = 0.f;
     }
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
-      m[hh] = 2 * t + hh < G ? -INFINITY : INFINITY;
+      m[hh] = 2 * t + hh < ncols ? kMaxFloor : INFINITY;
       l[hh] = 0.f;
     }
   }
 };
 
+// CHUNK: chunk mode (a pair is a group of a block's queries and one kv head;
+// its columns are the group's queries x gq heads; always with CL).
 // CL: cluster mode.  Pair p is streamed by the csize CTAs of cluster p, CTA
 // rank r taking an equal share of its padded rows (dec_cluster_share); each CTA
 // publishes its merged state in its own shared memory, and rank 0 reads its
 // peers' states through distributed shared memory, writes the pair's output
 // and (decode step) commits the sequence's bookkeeping -- no partials in global
 // memory, no second grid.  Otherwise the flattened split with k_decode_merge.
-template <int D, int G, bool CL>
+template <int D, int G, bool CL, bool CHUNK>
 __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
-    k_decode_mma(const __grid_constant__ MmaDecodeArgs ma) {
+    k_decode_mma(const __grid_constant__ MmaArgs<CHUNK> ma) {
+  static_assert(CL || !CHUNK, "chunk mode runs in cluster mode");
   constexpr int HALVES = D / 64;                       // 128-byte column blocks of a row
   constexpr uint32_t kHalfBytes = kTR * 128;           // one column block of a tile
   constexpr uint32_t kTileBytes = HALVES * kHalfBytes; // K (or V) of one tile
@@ -192,11 +213,18 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
   uint8_t* const vbuf = kbuf + kStagesM * kTileBytes;
   uint8_t* const qbuf = vbuf + kStagesM * kTileBytes;  // [kStagesM][G][D] bf16
   __shared__ __align__(8) uint64_t full[kStagesM], empty[kStagesM];
-  __shared__ __align__(8) uint64_t sync_a, sync_b, sync_c;
+  __shared__ __align__(8) uint64_t sync_a, sync_b, sync_c, sync_m;
   __shared__ __align__(8) uint64_t pub_bar, done_bar;  // cluster: peers published / rank 0 done
   __shared__ TileDescM desc[kStagesM];
   __shared__ int abort_flag;
-  __shared__ MergeSmem<G, D, kMW> sm;
+  // The warps' merge buffer.  In cluster mode a CTA streams one piece, so
+  // once every warp has consumed its last tile the K stages hold nothing more
+  // and the buffer lives there (two CTAs per SM fit at any G); the flattened
+  // split streams the next piece meanwhile and keeps a buffer of its own.
+  using Merge = MergeSmem<G, D, kMW>;
+  static_assert(sizeof(Merge) <= (size_t)kStagesM * kTileBytes, "merge buffer fits the K stages");
+  __shared__ __align__(16) uint8_t sm_own[CL ? 16 : sizeof(Merge)];
+  Merge& sm = *reinterpret_cast<Merge*>(CL ? kbuf : sm_own);
   __shared__ float pub_ml[G][2];  // cluster: this CTA's merged (max, sum) per head
   // paged cache: the page-table row of the piece's sequence (read by the producer only)
   __shared__ __align__(16) int32_t tbl[kTblMax + 4];
@@ -205,6 +233,27 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Hkv = a.c.Hkv;
   const int64_t R = a.total, NC = a.nctas;
+  // Columns of pair (b, g): a decode pair's G query heads; a chunk pair's
+  // nq queries x gq heads.  q and out rows: [rows][Hq][D].
+  constexpr int kLgG = G == 8 ? 3 : G == 4 ? 2 : G == 2 ? 1 : 0;
+  auto lgq = [&]() -> int {
+    if constexpr (CHUNK) return ma.ch.lgq; else return kLgG;
+  };
+  auto nq_of = [&](int b) -> int {
+    if constexpr (CHUNK) return ma.ch.nq[b]; else return 1;
+  };
+  auto qrow_of = [&](int b) -> int {
+    if constexpr (CHUNK) return ma.ch.qrow[b]; else return b;
+  };
+  // ring state the entry's queries see (a chunk group: the state before its block)
+  auto next_pos_of = [&](int b) -> int64_t {
+    if constexpr (CHUNK) return a.t[b] - ma.ch.i0[b]; else return a.t[b] + 1;
+  };
+  auto qo_off = [&](int b, int g, int c) -> size_t {
+    const int gq = 1 << lgq();
+    return ((size_t)(qrow_of(b) + (c >> lgq())) * a.Hq + (size_t)g * gq + (c & (gq - 1))) *
+           (size_t)D;
+  };
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStagesM; ++i) {
       ptx::mbar_init(&full[i], 1);
@@ -213,6 +262,7 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
     ptx::mbar_init(&sync_a, kMW);
     ptx::mbar_init(&sync_b, kMW);
     ptx::mbar_init(&sync_c, kMW);
+    ptx::mbar_init(&sync_m, kMW);
     ptx::mbar_init(&pub_bar, CL ? a.csize - 1 : 1);
     ptx::mbar_init(&done_bar, 1);
     ptx::mbar_init(&tbl_bar, 1);
@@ -231,6 +281,10 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
     if (ma.maps.page_box) {
       ptx::prefetch_tmap(&ma.maps.kring_p);
       ptx::prefetch_tmap(&ma.maps.vring_p);
+    }
+    if constexpr (CHUNK) {
+      ptx::prefetch_tmap(&ma.kblk);
+      ptx::prefetch_tmap(&ma.vblk);
     }
   }
   __syncthreads();
@@ -269,14 +323,29 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
     auto piece = [&](int b, int g, int32_t tph, int32_t j0, int32_t j1, int rank, bool check) {
       const int s = a.seq[b];
       DevMeta m;
-      m.next_pos = a.t[b] + 1;
+      m.next_pos = next_pos_of(b);
       m.P = a.P[b];
       m.head = a.head[b];
       m.count = a.count[b];
       m.owner = a.owner[b];
-      const DecRuns runs = dec_runs(m, a.c.W, a.t[b], page, step);
-      bool bad = runs.rows != m.P + m.count || (rank < 0 && dec_tiles(runs, kTR) != tph);
+      const DecRuns runs = [&]() {
+        if constexpr (CHUNK)
+          return dec_runs_chunk(m, a.c.W, m.next_pos, ma.ch.i0[b], ma.ch.nq[b], page);
+        else
+          return dec_runs(m, a.c.W, a.t[b], page, step);
+      }();
+      bool bad = (!CHUNK && runs.rows != m.P + m.count) ||
+                 (rank < 0 && dec_tiles(runs, kTR) != tph);
       const int pair = b * Hkv + g;
+      // the pair's q rows: one bulk copy per query of the entry, its heads of
+      // kv head g each (a decode entry: one copy of G heads)
+      const uint32_t qbytes = (uint32_t)((nq_of(b) << lgq()) * D * 2);
+      auto load_q = [&](int st) {
+        for (int k = 0; k < nq_of(b); ++k)
+          ptx::bulk_g2s(qbuf + ((size_t)st * G + ((size_t)k << lgq())) * D * 2,
+                        (const uint16_t*)a.q + qo_off(b, g, k << lgq()),
+                        (uint32_t)((1 << lgq()) * D * 2), &full[st]);
+      };
       const int zpre = m.owner * Hkv + g;
       // padded rows [xs, xe) of this piece, in tiles of kTR rows (the last may be short)
       int32_t xs, xe;
@@ -323,7 +392,8 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
         uint8_t* const vd = vbuf + (size_t)st * kTileBytes;
         const int32_t flags0 = (k == 0 ? TD_FIRST : 0) | (k == nt - 1 ? TD_LAST : 0);
         int32_t wsrc, wrow;
-        if (dec_range_whole(runs, kTR, x0, x1, &wsrc, &wrow)) {
+        const bool qdep = CHUNK && dec_tile_qdep(runs, x0, x1);
+        if (!qdep && dec_range_whole(runs, kTR, x0, x1, &wsrc, &wrow)) {
           // the common case: the tile is kTR rows of one run, copied whole
           desc[st].mask[0] = 0xffffffffu;
           desc[st].mask[1] = 0xffffffffu;
@@ -331,12 +401,9 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
           desc[st].flags = flags0;
           desc[st].slot = (int32_t)blockIdx.x + pair;
           desc[st].new_row = -1;
-          ptx::mbar_arrive_expect_tx(
-              &full[st], 2u * kTR * D * 2u + ((flags0 & TD_FIRST) ? (uint32_t)(G * D * 2) : 0u));
-          if (flags0 & TD_FIRST)
-            ptx::bulk_g2s(qbuf + (size_t)st * G * D * 2,
-                          (const uint16_t*)a.q + ((size_t)b * a.Hq + (size_t)g * G) * D,
-                          (uint32_t)(G * D * 2), &full[st]);
+          ptx::mbar_arrive_expect_tx(&full[st],
+                                     2u * kTR * D * 2u + ((flags0 & TD_FIRST) ? qbytes : 0u));
+          if (flags0 & TD_FIRST) load_q(st);
           const bool pre = wsrc == RUN_PREFIX;
           const int32_t y = pre ? wrow : (page ? wrow % page : wrow);
           const int32_t z = pre ? zpre : phys_of(wrow) * Hkv + g;
@@ -356,9 +423,9 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
           continue;
         }
         uint64_t mask = 0;  // valid tile rows
-        int32_t flags = flags0;
+        int32_t flags = flags0 | (qdep ? TD_QMASK : 0);
         int32_t new_row = -1;
-        uint32_t bytes = (flags & TD_FIRST) ? (uint32_t)(G * D * 2) : 0u;
+        uint32_t bytes = (flags & TD_FIRST) ? qbytes : 0u;
         dec_range_pieces(runs, x0, x1, [&](int32_t src, int32_t, int32_t sr, int32_t n) {
           mask |= (n >= 64 ? ~0ull : ((1ull << n) - 1ull)) << sr;
           if (src == RUN_NEW) {
@@ -377,11 +444,19 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
         desc[st].flags = flags;
         desc[st].slot = (int32_t)blockIdx.x + pair;
         desc[st].new_row = new_row;
+        if (CHUNK && qdep) {
+          // chunk mode: which of the group's queries see each row (prefix rows:
+          // all; rows outside the pieces are masked anyway)
+          uint32_t* qw = (uint32_t*)desc[st].qv;
+          for (int w = 0; w < kTR / 4; ++w) qw[w] = 0xffffffffu;
+          dec_range_pieces(runs, x0, x1, [&](int32_t src, int32_t row, int32_t sr, int32_t n) {
+            if (src == RUN_PREFIX) return;
+            for (int32_t r = 0; r < n; ++r)
+              desc[st].qv[sr + r] = (uint8_t)dec_row_queries(runs, src, row + r);
+          });
+        }
         ptx::mbar_arrive_expect_tx(&full[st], bytes);
-        if (flags & TD_FIRST)
-          ptx::bulk_g2s(qbuf + (size_t)st * G * D * 2,
-                        (const uint16_t*)a.q + ((size_t)b * a.Hq + (size_t)g * G) * D,
-                        (uint32_t)(G * D * 2), &full[st]);
+        if (flags & TD_FIRST) load_q(st);
         dec_range_pieces(runs, x0, x1, [&](int32_t src, int32_t row, int32_t sr, int32_t n) {
           if (src == RUN_NEW) {  // the appended token, straight from the caller's rows
             const uint16_t* kn = (const uint16_t*)a.knew + (size_t)pair * D;
@@ -392,6 +467,24 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
               ptx::bulk_g2s(vd + h * kHalfBytes + sr * 128, vn + h * 64, 128u, &full[st]);
             }
             return;
+          }
+          if constexpr (CHUNK) {
+            if (src == RUN_BLK) {
+              // the block's rows from the caller's buffers, whole atoms from
+              // the one holding the piece's first row
+              const int32_t lead = sr & (kPadRows - 1);
+              int32_t y = ma.ch.brow[b] + row - lead;
+              for (int32_t x = sr - lead; x < sr + n; x += kPadRows, y += kPadRows) {
+#pragma unroll
+                for (int h = 0; h < HALVES; ++h) {
+                  ptx::tma_load_3d(kd + h * kHalfBytes + x * 128, &ma.kblk, h * 64, g, y,
+                                   &full[st]);
+                  ptx::tma_load_3d(vd + h * kHalfBytes + x * 128, &ma.vblk, h * 64, g, y,
+                                   &full[st]);
+                }
+              }
+              return;
+            }
           }
           const CUtensorMap* km = src == RUN_PREFIX ? ma.maps.kpre : ma.maps.kring;
           const CUtensorMap* vm = src == RUN_PREFIX ? ma.maps.vpre : ma.maps.vring;
@@ -514,7 +607,8 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
     if (!__all_sync(FULL, ok)) { stopped = true; break; }
     const TileDescM d = desc[stg];
     if (d.flags & TD_END) break;
-    if (d.flags & TD_FIRST) st.init(qbuf + (size_t)stg * G * D * 2);
+    if (d.flags & TD_FIRST)
+      st.init(qbuf + (size_t)stg * G * D * 2, CHUNK ? nq_of(d.pair / Hkv) << lgq() : G);
     uint8_t* const kt = kbuf + (size_t)stg * kTileBytes;
     uint8_t* const vt = vbuf + (size_t)stg * kTileBytes;
     const uint32_t kt_s = ptx::smem_u32(kt), vt_s = ptx::smem_u32(vt);
@@ -546,8 +640,17 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
         mma16816(c, af, st.qf[ks][0], st.qf[ks][1]);
       }
       const bool r0 = (vm >> g) & 1u, r1 = (vm >> (g + 8)) & 1u;
-      const float s0 = r0 ? c[0] * qs : -INFINITY, s1 = r0 ? c[1] * qs : -INFINITY;
-      const float s2 = r1 ? c[2] * qs : -INFINITY, s3 = r1 ? c[3] * qs : -INFINITY;
+      bool v00 = r0, v01 = r0, v10 = r1, v11 = r1;
+      if (CHUNK && (d.flags & TD_QMASK)) {  // column 2tq + hh holds query (2tq + hh) >> lgq
+        const uint32_t qa = desc[stg].qv[R0 + g], qb = desc[stg].qv[R0 + g + 8];
+        const int k0 = (2 * tq) >> lgq(), k1 = (2 * tq + 1) >> lgq();
+        v00 = v00 && ((qa >> k0) & 1u);
+        v01 = v01 && ((qa >> k1) & 1u);
+        v10 = v10 && ((qb >> k0) & 1u);
+        v11 = v11 && ((qb >> k1) & 1u);
+      }
+      const float s0 = v00 ? c[0] * qs : -INFINITY, s1 = v01 ? c[1] * qs : -INFINITY;
+      const float s2 = v10 ? c[2] * qs : -INFINITY, s3 = v11 ? c[3] * qs : -INFINITY;
       const bool need = s0 > st.m[0] + kRaiseLog2 || s2 > st.m[0] + kRaiseLog2 ||
                         s1 > st.m[1] + kRaiseLog2 || s3 > st.m[1] + kRaiseLog2;
       if (__any_sync(FULL, need)) {
@@ -570,7 +673,8 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
           }
         }
       }
-      // every valid head's max is finite here; a padding head's is +inf
+      // every valid column's max is finite here (at least the floor); a
+      // padding column's is +inf
       const float p0 = ex2(s0 - st.m[0]), p1 = ex2(s1 - st.m[1]);
       const float p2 = ex2(s2 - st.m[0]), p3 = ex2(s3 - st.m[1]);
       st.l[0] += p0 + p2;
@@ -615,6 +719,9 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
       st.l[hh] += __shfl_xor_sync(FULL, st.l[hh], 8);
       st.l[hh] += __shfl_xor_sync(FULL, st.l[hh], 16);
     }
+    // cluster mode: the merge buffer is the K stages; every warp must be done
+    // reading its last tile first
+    if (CL && !csync(&sync_m, np)) { stopped = true; break; }
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       const int h = 2 * tq + hh;
@@ -683,7 +790,8 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
       const bool ok = ptx::mbar_wait_cluster_bounded(&pub_bar, 0, &abort_flag, kWaitLimitCycles);
       if (__all_sync(FULL, ok)) {
         const int pair = blockIdx.x / C, b = pair / Hkv, gg = pair % Hkv;
-        for (int idx = threadIdx.x; idx < G * D; idx += kMW * 32) {
+        const int ncols = nq_of(b) << lgq();  // valid columns of the pair
+        for (int idx = threadIdx.x; idx < ncols * D; idx += kMW * 32) {
           const int h = idx / D, e = idx % D;
           float mr[kMaxCluster], lr[kMaxCluster], orr[kMaxCluster];
           float M = -INFINITY;
@@ -705,8 +813,7 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
               A += orr[r] * w;
             }
           }
-          store_out<uint16_t>((uint16_t*)a.out + ((size_t)b * a.Hq + (size_t)gg * G + h) * D + e,
-                              A / L);
+          store_out<uint16_t>((uint16_t*)a.out + qo_off(b, gg, h) + e, A / L);
         }
         // the peers' shared memory has been read: let them exit
         if (csync(&sync_c, np == 0 ? 1 : 0) && threadIdx.x == 0) {
@@ -718,7 +825,7 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
             const DevMeta md = a.c.meta[s];
             DevMeta m;
             memset(&m, 0, sizeof(m));
-            m.next_pos = a.t[b] + 1;
+            m.next_pos = next_pos_of(b);
             m.P = a.P[b];
             m.head = a.head[b];
             m.count = a.count[b];
@@ -743,13 +850,14 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
 }
 
 // Resident CTAs per SM of one instantiation (at most PS_DMMA_CTAS_PER_SM).
-template <int D, int G, bool CL>
+template <int D, int G, bool CL, bool CHUNK>
 int ctas_per_sm(size_t dyn) {
   static std::atomic<int> cached{0};
   int n = cached.load();
   if (n == 0) {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_decode_mma<D, G, CL>, kThreadsM,
-                                                      dyn) != cudaSuccess || n < 1)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_decode_mma<D, G, CL, CHUNK>,
+                                                      kThreadsM, dyn) != cudaSuccess ||
+        n < 1)
       n = 1;
     if (n > PS_DMMA_CTAS_PER_SM) n = PS_DMMA_CTAS_PER_SM;
     cached.store(n);
@@ -757,7 +865,7 @@ int ctas_per_sm(size_t dyn) {
   return n;
 }
 
-template <int D, int G, bool CL>
+template <int D, int G, bool CL, bool CHUNK>
 cudaError_t configure(size_t dyn) {
   static std::atomic<uint64_t> configured{0};  // one bit per device
   int dev = 0;
@@ -765,11 +873,11 @@ cudaError_t configure(size_t dyn) {
   if (e != cudaSuccess) return e;
   const uint64_t bit = 1ull << (dev & 63);
   if (!(configured.load() & bit)) {
-    e = cudaFuncSetAttribute(k_decode_mma<D, G, CL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)dyn);
+    e = cudaFuncSetAttribute(k_decode_mma<D, G, CL, CHUNK>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
     if (e != cudaSuccess) return e;
     // all of the unified L1/shared memory as shared, so that two CTAs fit per SM
-    e = cudaFuncSetAttribute(k_decode_mma<D, G, CL>,
+    e = cudaFuncSetAttribute(k_decode_mma<D, G, CL, CHUNK>,
                              cudaFuncAttributePreferredSharedMemoryCarveout,
                              (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
@@ -778,8 +886,50 @@ cudaError_t configure(size_t dyn) {
   return cudaSuccess;
 }
 
-template <int D, int G>
-cudaError_t launch_mma(MmaDecodeArgs& ma, int sm_count, cudaStream_t st) {
+// Clusters of c CTAs of one instantiation that are resident at once (the
+// occupancy API's count: clusters must fit inside a GPC, so it is below
+// 2 * SMs / c for c = 4 and 8).  Cached per cluster size; 0 on failure.
+template <int D, int G, bool CHUNK>
+int cluster_capacity(int c, size_t dyn) {
+  static std::atomic<int> cached[4] = {{-1}, {-1}, {-1}, {-1}};
+  const int k = c == 8 ? 3 : c == 4 ? 2 : c == 2 ? 1 : 0;
+  int n = cached[k].load();
+  if (n < 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(c * 64));
+    cfg.blockDim = dim3(kThreadsM);
+    cfg.dynamicSmemBytes = dyn;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = (unsigned)c;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, k_decode_mma<D, G, true, CHUNK>, &cfg) != cudaSuccess)
+      n = 0;
+    cached[k].store(n);
+  }
+  return n;
+}
+
+// Clusters of c CTAs that one launch of `pairs` clusters may use: all
+// resident at once, and for c = 8 no more than three quarters of the
+// capacity (measured: 32 clusters of 8, nearly the 33 that fit, ran slower
+// than the same pairs in 64 clusters of 4).
+template <int D, int G, bool CHUNK>
+bool clusters_fit(int64_t pairs, int c, size_t dyn) {
+  const int64_t cap = cluster_capacity<D, G, CHUNK>(c, dyn);
+  return c == 8 ? 4 * pairs <= 3 * cap : pairs <= cap;
+}
+
+template <int D, int G, bool CHUNK>
+constexpr size_t dyn_smem() {
+  return 1024 + (size_t)kStagesM * (2 * (D / 64) * kTR * 128 + G * D * 2);
+}
+
+template <int D, int G, bool CHUNK>
+cudaError_t launch_mma(MmaArgs<CHUNK>& ma, int sm_count, cudaStream_t st) {
   DecodeArgs& a = ma.a;
   const int32_t page = a.c.page_table ? a.c.page_rows : 0;
   const bool step = a.knew != nullptr;
@@ -788,39 +938,51 @@ cudaError_t launch_mma(MmaDecodeArgs& ma, int sm_count, cudaStream_t st) {
   for (int b = 0; b < a.B; ++b) {
     DevMeta m;
     memset(&m, 0, sizeof(m));
-    m.next_pos = a.t[b] + 1;
     m.P = a.P[b];
     m.head = a.head[b];
     m.count = a.count[b];
     m.owner = a.owner[b];
-    const DecRuns r = dec_runs(m, a.c.W, a.t[b], page, step);
+    DecRuns r;
+    if constexpr (CHUNK) {
+      m.next_pos = a.t[b] - ma.ch.i0[b];
+      r = dec_runs_chunk(m, a.c.W, m.next_pos, ma.ch.i0[b], ma.ch.nq[b], page);
+    } else {
+      m.next_pos = a.t[b] + 1;
+      r = dec_runs(m, a.c.W, a.t[b], page, step);
+    }
     const int32_t tph = dec_tiles(r, kTR);
     a.tcum[b + 1] = a.tcum[b] + a.c.Hkv * tph;
     tmin = tph < tmin ? tph : tmin;
     tmax = tph > tmax ? tph : tmax;
   }
   a.total = a.tcum[a.B];
-  constexpr size_t dyn = 1024 + (size_t)kStagesM * (2 * (D / 64) * kTR * 128 + G * D * 2);
-  // Cluster mode when there are few pairs of about equal length: csize CTAs
-  // per pair with csize the largest of 8, 4, 2 that keeps every CTA resident
-  // at once, provided that fills at least half of the resident slots and gives
-  // each CTA a few tiles.  Otherwise the flattened split.
+  constexpr size_t dyn = dyn_smem<D, G, CHUNK>();
   const int64_t pairs = (int64_t)a.B * a.c.Hkv;
   cudaError_t e;
-  if ((e = configure<D, G, true>(dyn)) != cudaSuccess) return e;
-  if ((e = configure<D, G, false>(dyn)) != cudaSuccess) return e;
+  if ((e = configure<D, G, true, CHUNK>(dyn)) != cudaSuccess) return e;
   int csize = 0;
+  if constexpr (CHUNK) {
+    // no workspace: always clusters, of the largest size that fits (else
+    // pairs of CTAs, in waves)
+    csize = 2;
+    for (int c = kMaxCluster; c >= 2; c /= 2)
+      if (clusters_fit<D, G, true>(pairs, c, dyn)) { csize = c; break; }
+  } else {
+    if ((e = configure<D, G, false, false>(dyn)) != cudaSuccess) return e;
 #ifndef PS_DMMA_NO_CLUSTER
-  {
-    const int64_t slots = (int64_t)sm_count * ctas_per_sm<D, G, true>(dyn);
+    // Cluster mode when there are few pairs of about equal length: csize CTAs
+    // per pair with csize the largest of 8, 4, 2 that fits (clusters_fit),
+    // provided that fills at least half of the resident slots and gives each
+    // CTA a few tiles.  Otherwise the flattened split.
+    const int64_t slots = (int64_t)sm_count * ctas_per_sm<D, G, true, false>(dyn);
     for (int c = kMaxCluster; c >= 2; c /= 2) {
-      if (pairs * c <= slots) {
+      if (clusters_fit<D, G, false>(pairs, c, dyn)) {
         if (2 * pairs * c >= slots && tmin >= 2 * c && 4 * tmax <= 5 * tmin) csize = c;
         break;
       }
     }
-  }
 #endif
+  }
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -838,19 +1000,22 @@ cudaError_t launch_mma(MmaDecodeArgs& ma, int sm_count, cudaStream_t st) {
     attr[1].val.clusterDim.z = 1;
     dcfg.numAttrs = 2;
     dcfg.gridDim = dim3((unsigned)a.nctas);
-    return cudaLaunchKernelEx(&dcfg, k_decode_mma<D, G, true>, ma);
+    return cudaLaunchKernelEx(&dcfg, k_decode_mma<D, G, true, CHUNK>, ma);
   }
-  a.csize = 0;
-  int64_t nc = ((int64_t)a.total + kMinTilesPerCta - 1) / kMinTilesPerCta;
-  const int64_t maxc = (int64_t)sm_count * ctas_per_sm<D, G, false>(dyn);
-  if (nc > maxc) nc = maxc;
-  if (nc < 1) nc = 1;
-  a.nctas = (int)nc;
-  dcfg.numAttrs = 1;
-  dcfg.gridDim = dim3((unsigned)a.nctas);
-  e = cudaLaunchKernelEx(&dcfg, k_decode_mma<D, G, false>, ma);
-  if (e != cudaSuccess) return e;
-  return launch_merge<uint16_t, D, G>(a, st);
+  if constexpr (!CHUNK) {
+    a.csize = 0;
+    int64_t nc = ((int64_t)a.total + kMinTilesPerCta - 1) / kMinTilesPerCta;
+    const int64_t maxc = (int64_t)sm_count * ctas_per_sm<D, G, false, false>(dyn);
+    if (nc > maxc) nc = maxc;
+    if (nc < 1) nc = 1;
+    a.nctas = (int)nc;
+    dcfg.numAttrs = 1;
+    dcfg.gridDim = dim3((unsigned)a.nctas);
+    e = cudaLaunchKernelEx(&dcfg, k_decode_mma<D, G, false, false>, ma);
+    if (e != cudaSuccess) return e;
+    return launch_merge<uint16_t, D, G>(a, st);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace
@@ -901,6 +1066,42 @@ bool make_decode_maps(const CacheDev& c, DecodeMaps* m) {
   return ok;
 }
 
+int chunk_small_pair_capacity(int d) {
+  if (d == 128) {
+    constexpr size_t dyn = dyn_smem<128, 8, true>();
+    if (configure<128, 8, true, true>(dyn) != cudaSuccess) return 0;
+    return cluster_capacity<128, 8, true>(2, dyn);
+  }
+  if (d == 64) {
+    constexpr size_t dyn = dyn_smem<64, 8, true>();
+    if (configure<64, 8, true, true>(dyn) != cudaSuccess) return 0;
+    return cluster_capacity<64, 8, true>(2, dyn);
+  }
+  return 0;
+}
+
+cudaError_t launch_chunk_small(const DecodeArgs& a, const ChunkArgs& ch, const DecodeMaps& maps,
+                               const void* k_blk, const void* v_blk, int64_t blk_rows,
+                               int sm_count, cudaStream_t st) {
+  MmaChunkArgs ma;
+  memset(&ma, 0, sizeof(ma));
+  ma.maps = maps;
+  ma.a = a;
+  ma.ch = ch;
+  const int D = a.c.d;
+  const uint64_t row = (uint64_t)D * 2;
+  // block rows [rows][Hkv][D]: dimensions (column, kv head, row), boxes of 8
+  // rows of one 64-column block of one head (the ring tiles' atom layout)
+  if (!encode_map3d_bf16(&ma.kblk, k_blk, (uint64_t)D, (uint64_t)a.c.Hkv, (uint64_t)blk_rows, row,
+                         row * a.c.Hkv, 64, 1, kPadRows, PS_DMMA_L2_PROMOTION) ||
+      !encode_map3d_bf16(&ma.vblk, v_blk, (uint64_t)D, (uint64_t)a.c.Hkv, (uint64_t)blk_rows, row,
+                         row * a.c.Hkv, 64, 1, kPadRows, PS_DMMA_L2_PROMOTION))
+    return cudaErrorInvalidValue;
+  if (D == 128) return launch_mma<128, 8, true>(ma, sm_count, st);
+  if (D == 64) return launch_mma<64, 8, true>(ma, sm_count, st);
+  return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_decode_mma(const DecodeArgs& a, int G, const DecodeMaps& maps, int sm_count,
                               cudaStream_t st) {
   MmaDecodeArgs ma;
@@ -909,7 +1110,7 @@ cudaError_t launch_decode_mma(const DecodeArgs& a, int G, const DecodeMaps& maps
   ma.a = a;
   const int D = a.c.d;
 #define PS_DMMA_CASE(DD, GG) \
-  if (D == DD && G == GG) return launch_mma<DD, GG>(ma, sm_count, st);
+  if (D == DD && G == GG) return launch_mma<DD, GG, false>(ma, sm_count, st);
   PS_DMMA_CASE(128, 1) PS_DMMA_CASE(128, 2) PS_DMMA_CASE(128, 4) PS_DMMA_CASE(128, 8)
   PS_DMMA_CASE(64, 1) PS_DMMA_CASE(64, 2) PS_DMMA_CASE(64, 4) PS_DMMA_CASE(64, 8)
 #undef PS_DMMA_CASE

@@ -20,6 +20,13 @@
 // range and the window range are walked separately and the evicted middle is
 // never visited).
 //
+// Chunk mode (a small block of queries routed off the 128-row tensor-core
+// tile): a pair is one group of up to 8 consecutive queries of the block and
+// one kv head; its runs are the union of the group's visible sets -- the
+// prefix, the ring window of its first query, and the block's own rows (read
+// from the caller's buffer) -- and a per-row query mask (dec_row_queries)
+// cuts that union back to each query's set.
+//
 // Host-callable, so that the layout can be checked on the CPU.
 #pragma once
 #include <stdint.h>
@@ -36,6 +43,7 @@ enum : int32_t {
   RUN_PREFIX = 0,  // prefix rows of the owner's slab, row0 = first prefix row
   RUN_RING = 1,    // ring slots of the sequence, row0 = first slot
   RUN_NEW = 2,     // the appended token (decode step), from the caller's buffer
+  RUN_BLK = 3,     // chunk mode: rows of the caller's block, row0 = first block row
 };
 
 struct DecRuns {
@@ -48,6 +56,14 @@ struct DecRuns {
   int32_t rows;       // valid rows of the pair
   int32_t page;       // ring page rows of a paged cache, 0 when unpaged
   int32_t ring_ok;    // 0 if the window reaches below what the ring holds
+  // chunk mode (dec_runs_chunk; a plain decode leaves qb0 = qd0 = qd1 = 0 and
+  // no tile is query-dependent): the group's queries are at t0 + qi0 + k,
+  // k < qnq; qlo = t0 + qi0 - W + 1; ring slot s holds position
+  // rbase + (s - rhead) mod W.  Padded rows [qd0, qd1) and [qb0, padded) may
+  // hold rows that not every query of the group sees.
+  int64_t qlo, rbase;
+  int32_t qi0, qnq, qW, rhead;
+  int32_t qd0, qd1, qb0;
 };
 
 // Pages whose edges fall on atom boundaries keep the unpaged layout.
@@ -118,6 +134,8 @@ __host__ __device__ __forceinline__ DecRuns dec_runs(const DevMeta& m, int32_t W
       --lenA;
     }
   }
+  r.qlo = 0; r.rbase = 0; r.qi0 = 0; r.qnq = 1; r.qW = W; r.rhead = 0;
+  r.qd0 = 0; r.qd1 = 0; r.qb0 = 0;
   int32_t n = 0, padded = 0, rows = 0;
   auto add = [&](int32_t src, int32_t row0, int32_t len, int32_t pre, int32_t padlen) {
 #pragma unroll
@@ -141,7 +159,125 @@ __host__ __device__ __forceinline__ DecRuns dec_runs(const DevMeta& m, int32_t W
   r.n = n;
   r.padded = padded;
   r.rows = rows;
+  r.qb0 = padded;
   return r;
+}
+
+// Runs of a chunk-mode pair: the group of nq (1..8) queries at positions
+// t0 + i0 + k of a block whose rows j sit at positions t0 + j in the caller's
+// buffer, with m the ring state before the block (next_pos == t0).  Query i
+// of the block sees (digest section 03, 0-indexed) the prefix [0, P), the ring
+// rows at positions >= max(P, t0 + i - W + 1), and the block rows j with
+// i - W + 1 <= j <= i.  The runs hold the union over the group: the prefix,
+// the ring window of its first query as at most two slot runs, and block rows
+// [max(0, i0 - W + 1), i0 + nq) as one run from an atom boundary.
+__host__ __device__ __forceinline__ DecRuns dec_runs_chunk(const DevMeta& m, int32_t W, int64_t t0,
+                                                           int32_t i0, int32_t nq, int32_t page) {
+  DecRuns r;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    r.src[i] = 0; r.row0[i] = 0; r.len[i] = 0; r.pstart[i] = 0;
+  }
+  r.page = page;
+  r.ring_ok = 1;
+  const int64_t base = m.next_pos - m.count;
+  const int64_t qlo = t0 + i0 - (int64_t)W + 1;
+  int64_t lo = qlo < m.P ? (int64_t)m.P : qlo;
+  const int64_t hi = m.next_pos - 1;
+  int32_t s0 = 0, lenA = 0, lenB = 0;
+  if (hi >= lo) {
+    if (lo < base) {
+      r.ring_ok = 0;
+      lo = base;
+    }
+    if (hi >= lo) {
+      const int64_t nw = hi - lo + 1;
+      s0 = m.head + (int32_t)(lo - base);
+      if (s0 >= W) s0 -= W;
+      lenA = (int32_t)(nw < (int64_t)(W - s0) ? nw : (int64_t)(W - s0));
+      lenB = (int32_t)(nw - lenA);
+    }
+  }
+  const int32_t jlo = i0 - W + 1 > 0 ? i0 - W + 1 : 0;
+  const int32_t nblk = i0 + nq - jlo;
+  int32_t n = 0, padded = 0, rows = 0;
+  int32_t pA = 0, pB = 0;
+  auto add = [&](int32_t src, int32_t row0, int32_t len, int32_t pre, int32_t padlen) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if (k == n) {
+        r.src[k] = src;
+        r.row0[k] = row0;
+        r.len[k] = len;
+        r.pstart[k] = padded + pre;
+      }
+    }
+    ++n;
+    padded += padlen;
+    rows += len;
+  };
+  if (m.P > 0) add(RUN_PREFIX, 0, m.P, 0, pad8(m.P));
+  const bool al = page_aligned(page);
+  pA = padded;
+  if (lenA > 0) add(RUN_RING, s0, lenA, al ? s0 % kPadRows : 0, ring_run_padded(s0, lenA, page));
+  pB = padded;
+  if (lenB > 0) add(RUN_RING, 0, lenB, 0, ring_run_padded(0, lenB, page));
+  const int32_t pK = padded;
+  add(RUN_BLK, jlo, nblk, 0, pad8(nblk));
+  r.n = n;
+  r.padded = padded;
+  r.rows = rows;
+  r.qlo = qlo;
+  r.rbase = base;
+  r.qi0 = i0;
+  r.qnq = nq;
+  r.qW = W;
+  r.rhead = m.head;
+  // Ring rows whose visibility differs within the group: positions
+  // [lo, qlo + nq - 1), the window's first rows (run A, then run B).
+  int64_t dep = qlo + nq - 1 - lo;
+  if (dep < 0) dep = 0;
+  if (dep > (int64_t)lenA + lenB) dep = (int64_t)lenA + lenB;
+  r.qd0 = pA;
+  r.qd1 = pA;
+  if (dep > 0) {
+    if (dep <= lenA) {
+      r.qd1 = pA + ring_run_padded(s0, (int32_t)dep, page);
+    } else {
+      r.qd1 = pB + ring_run_padded(0, (int32_t)(dep - lenA), page);
+    }
+  }
+  // Block rows: j > i0 (causal inside the block), and with a window shorter
+  // than the group, j < i0 + nq - W.
+  const int32_t jd = i0 + nq - W > jlo ? jlo : i0 + 1;
+  r.qb0 = pK + (jd - jlo);
+  return r;
+}
+
+// Queries of a chunk-mode group (bit k: query t0 + qi0 + k) that see the row
+// `row` of a run of source src (prefix row, ring slot, or block row).
+__host__ __device__ __forceinline__ uint32_t dec_row_queries(const DecRuns& r, int32_t src,
+                                                             int32_t row) {
+  int64_t lo_k = 0, hi_k = 7;  // queries k in [lo_k, hi_k] see the row
+  if (src == RUN_RING) {
+    int32_t off = row - r.rhead;
+    if (off < 0) off += r.qW;
+    hi_k = r.rbase + off - r.qlo;  // position >= qlo + k
+  } else if (src == RUN_BLK) {
+    const int32_t d = row - r.qi0;  // block row j <= i0 + k and j >= i0 + k - W + 1
+    lo_k = d;
+    hi_k = (int64_t)d + r.qW - 1;
+  }
+  if (lo_k < 0) lo_k = 0;
+  if (hi_k > 7) hi_k = 7;
+  if (hi_k < lo_k) return 0u;
+  return ((2u << hi_k) - 1u) & ~((1u << lo_k) - 1u);
+}
+
+// True if the tile of padded rows [x0, x1) may hold a row that not every query
+// of a chunk-mode group sees (never in a plain decode or a decode step).
+__host__ __device__ __forceinline__ bool dec_tile_qdep(const DecRuns& r, int32_t x0, int32_t x1) {
+  return (x0 < r.qd1 && x1 > r.qd0) || x1 > r.qb0;
 }
 
 __host__ __device__ __forceinline__ int32_t dec_tiles(const DecRuns& r, int32_t TR) {
@@ -158,7 +294,8 @@ __host__ __device__ __forceinline__ bool dec_range_whole(const DecRuns& r, int32
   if (x1 - x0 != TR) return false;
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    if (k < r.n && r.src[k] != RUN_NEW && x0 >= r.pstart[k] && x0 + TR <= r.pstart[k] + r.len[k]) {
+    if (k < r.n && r.src[k] <= RUN_RING && x0 >= r.pstart[k] &&
+        x0 + TR <= r.pstart[k] + r.len[k]) {
       const int32_t rw = r.row0[k] + (x0 - r.pstart[k]);
       const int32_t pg = r.src[k] == RUN_RING ? r.page : 0;
       if (pg <= 0 || rw % pg + TR <= pg) {

@@ -84,6 +84,27 @@ cudaError_t launch_decode(const CacheDev& c, int dtype, int G, const BatchIds& i
                           float scale, const DecodeWs& ws, int sm_count, const DecodeMaps* maps,
                           cudaStream_t st);
 
+// Small chunk blocks on the tensor-core decode kernel (bf16, head_dim 64 or
+// 128): entry e is a group of nq (1..8) consecutive queries of one sequence's
+// block, the first at position t0 + i0 (i0-th of the block); its q / out rows
+// start at packed row qrow and its block's key rows at packed row brow of
+// k_blk / v_blk.  cols (1, 2, 4 or 8) = the kernel's columns, >= nq * Hq/Hkv.
+// Default largest block of the small path (ps_set_chunk_small_max).
+constexpr int kChunkSmallMaxDefault = 64;
+struct SmallChunkEntry {
+  int seq, P, head, count, owner;  // the ring state before the block
+  int64_t t0;
+  int32_t i0, nq, qrow, brow;
+};
+// (group, kv head) pairs of the small-block path that are resident at once
+// in clusters of two CTAs (one wave); 0 if the occupancy query fails.
+int chunk_small_pair_capacity(int d);
+cudaError_t launch_chunk_small_batch(const CacheDev& c, int cols, int gq,
+                                     const SmallChunkEntry* e, int B, int Hq, const void* q,
+                                     const void* k_blk, const void* v_blk, int64_t blk_rows,
+                                     void* out, float scale, int sm_count, const DecodeMaps& maps,
+                                     cudaStream_t st);
+
 // chunk_tc.cu (tcgen05 chunk kernel: bf16, head_dim 128)
 bool chunk_tc_supported(const CacheDev& c, int dtype, int d, int G);
 // One sequence's block in a batched chunk or prompt launch: n >= 1 queries at

@@ -22,12 +22,17 @@ def _bits(x):
 
 
 def _setup(dtype, d, Hq, Hkv, W, P, starts, heads, page=0, seed=41):
+    """Two identical caches.  Small blocks stay on the chunk kernels (bound 0):
+    a call takes the split decode path for small blocks only when all its
+    blocks are small, so a batch and its single calls may take different paths
+    (tests/test_gpu_chunk_small.py covers that path)."""
     S = len(starts)
     sds = [SeqData(seed, s, Hq, Hkv, d, dtype) for s in range(S)]
     caches = []
     for _ in range(2):
         c = Cache(W, P, Hkv, d, ps_dtype(dtype), S, page_rows=page,
                   num_pages=S * (W // page) if page else 0)
+        c.set_chunk_small_max(0)
         for s, (sd, t) in enumerate(zip(sds, starts)):
             c.seq_reset(s, heads[s])
             c.prefill_prefix(s, to_torch(sd.k(0, P)), to_torch(sd.v(0, P)), P)
