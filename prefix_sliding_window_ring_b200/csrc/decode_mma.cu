@@ -204,8 +204,12 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
     k_decode_mma(const __grid_constant__ MmaArgs<CHUNK> ma) {
   static_assert(CL || !CHUNK, "chunk mode runs in cluster mode");
   constexpr int HALVES = D / 64;                       // 128-byte column blocks of a row
-  constexpr uint32_t kHalfBytes = kTR * 128;           // one column block of a tile
-  constexpr uint32_t kTileBytes = HALVES * kHalfBytes; // K (or V) of one tile
+  // Tile layout in shared memory: 8-row atoms one after the other, each
+  // holding its rows of every 64-column block ([atom][block][8 rows][128
+  // bytes], 128-byte swizzle inside each 1 KiB block), so one atom-map copy
+  // brings whole atoms of all column blocks.
+  constexpr uint32_t kAtomBytes = HALVES * 1024;       // one 8-row atom, all column blocks
+  constexpr uint32_t kTileBytes = (kTR / 8) * kAtomBytes;  // K (or V) of one tile
   constexpr int KS = D / 16;
   const DecodeArgs& a = ma.a;
   extern __shared__ uint8_t dsm_raw[];
@@ -273,15 +277,21 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
     // fetch the tensor maps' descriptors while the previous grid drains
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
-      ptx::prefetch_tmap(&ma.maps.kpre[k]);
-      ptx::prefetch_tmap(&ma.maps.vpre[k]);
-      ptx::prefetch_tmap(&ma.maps.kring[k]);
-      ptx::prefetch_tmap(&ma.maps.vring[k]);
+      if (ma.maps.prefix_atoms) {
+        ptx::prefetch_tmap(&ma.maps.kpa[k]);
+        ptx::prefetch_tmap(&ma.maps.vpa[k]);
+      }
+      if (ma.maps.ring_atoms) {
+        ptx::prefetch_tmap(&ma.maps.kra[k]);
+        ptx::prefetch_tmap(&ma.maps.vra[k]);
+      }
     }
     if (ma.maps.page_box) {
-      ptx::prefetch_tmap(&ma.maps.kring_p);
-      ptx::prefetch_tmap(&ma.maps.vring_p);
+      ptx::prefetch_tmap(&ma.maps.kra[2]);
+      ptx::prefetch_tmap(&ma.maps.vra[2]);
     }
+    ptx::prefetch_tmap(&ma.maps.kring8);
+    ptx::prefetch_tmap(&ma.maps.vring8);
     if constexpr (CHUNK) {
       ptx::prefetch_tmap(&ma.kblk);
       ptx::prefetch_tmap(&ma.vblk);
@@ -377,7 +387,12 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
         ++tbl_n;
       }
       auto phys_of = [&](int32_t slot) -> int {
-        return tab ? tab[slot / page] : ring_page(a.c, s, slot);
+        return tab ? tab[pg_div(slot, page, runs.plg)] : ring_page(a.c, s, slot);
+      };
+      // the atom maps of a prefix (pre) or ring copy
+      auto amap = [&](bool pre, bool isv, int k) -> const CUtensorMap* {
+        return pre ? (isv ? &ma.maps.vpa[k] : &ma.maps.kpa[k])
+                   : (isv ? &ma.maps.vra[k] : &ma.maps.kra[k]);
       };
       for (int32_t k = 0; k < nt && alive; ++k) {
         const int32_t x0 = xs + k * kTR, x1 = min(x0 + kTR, xe);
@@ -405,18 +420,20 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
                                      2u * kTR * D * 2u + ((flags0 & TD_FIRST) ? qbytes : 0u));
           if (flags0 & TD_FIRST) load_q(st);
           const bool pre = wsrc == RUN_PREFIX;
-          const int32_t y = pre ? wrow : (page ? wrow % page : wrow);
+          const int32_t y = pre ? wrow : (page ? pg_mod(wrow, page, runs.plg) : wrow);
           const int32_t z = pre ? zpre : phys_of(wrow) * Hkv + g;
-          if (HALVES == 2 && ma.maps.whole) {
-            ptx::tma_load_4d(kd, pre ? &ma.maps.kpre_w : &ma.maps.kring_w, 0, y, 0, z, &full[st]);
-            ptx::tma_load_4d(vd, pre ? &ma.maps.vpre_w : &ma.maps.vring_w, 0, y, 0, z, &full[st]);
-          } else {
+          if (pre ? ma.maps.prefix_atoms : ma.maps.ring_atoms) {  // one copy per operand: 8 atoms
+            ptx::tma_load_5d(kd, amap(pre, false, 0), 0, 0, 0, y >> 3, z, &full[st]);
+            ptx::tma_load_5d(vd, amap(pre, true, 0), 0, 0, 0, y >> 3, z, &full[st]);
+          } else {  // an atom of a column block per copy
+            for (int t = 0; t < kTR / 8; ++t) {
 #pragma unroll
-            for (int h = 0; h < HALVES; ++h) {
-              ptx::tma_load_3d(kd + h * kHalfBytes, pre ? &ma.maps.kpre[0] : &ma.maps.kring[0],
-                               h * 64, y, z, &full[st]);
-              ptx::tma_load_3d(vd + h * kHalfBytes, pre ? &ma.maps.vpre[0] : &ma.maps.vring[0],
-                               h * 64, y, z, &full[st]);
+              for (int h = 0; h < HALVES; ++h) {
+                ptx::tma_load_3d(kd + t * kAtomBytes + h * 1024, pre ? &ma.maps.kpre8 : &ma.maps.kring8,
+                                 h * 64, y + 8 * t, z, &full[st]);
+                ptx::tma_load_3d(vd + t * kAtomBytes + h * 1024, pre ? &ma.maps.vpre8 : &ma.maps.vring8,
+                                 h * 64, y + 8 * t, z, &full[st]);
+              }
             }
           }
           ++i;
@@ -425,17 +442,104 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
         uint64_t mask = 0;  // valid tile rows
         int32_t flags = flags0 | (qdep ? TD_QMASK : 0);
         int32_t new_row = -1;
-        uint32_t bytes = (flags & TD_FIRST) ? qbytes : 0u;
-        dec_range_pieces(runs, x0, x1, [&](int32_t src, int32_t, int32_t sr, int32_t n) {
+        // One pass: each copy is issued as the tile's pieces are walked and
+        // its bytes counted; the barrier's arrival with the byte count comes
+        // last (an mbarrier's tx-count may run below zero until then, and the
+        // phase cannot complete before the arrival).
+        uint32_t bytes = 0;
+        if (flags & TD_FIRST) {
+          load_q(st);
+          bytes += qbytes;
+        }
+        dec_range_pieces(runs, x0, x1, [&](int32_t src, int32_t row, int32_t sr, int32_t n) {
           mask |= (n >= 64 ? ~0ull : ((1ull << n) - 1ull)) << sr;
-          if (src == RUN_NEW) {
+          if (src == RUN_NEW) {  // the appended token, straight from the caller's rows
             flags |= TD_NEW;
             new_row = sr;
+            const uint16_t* kn = (const uint16_t*)a.knew + (size_t)pair * D;
+            const uint16_t* vn = (const uint16_t*)a.vnew + (size_t)pair * D;
+#pragma unroll
+            for (int h = 0; h < HALVES; ++h) {  // row sr % 8 == 0: the swizzle is the identity
+              ptx::bulk_g2s(kd + (sr >> 3) * kAtomBytes + h * 1024, kn + h * 64, 128u, &full[st]);
+              ptx::bulk_g2s(vd + (sr >> 3) * kAtomBytes + h * 1024, vn + h * 64, 128u, &full[st]);
+            }
             bytes += 2u * D * 2u;
-          } else {  // whole atoms from the one holding the piece's first row
-            const int32_t nb = (sr & (kPadRows - 1)) + n;
-            const int32_t boxed = (nb / kBox) * kBox + pad8(nb % kBox);
-            bytes += 2u * (uint32_t)boxed * D * 2u;
+            return;
+          }
+          if constexpr (CHUNK) {
+            if (src == RUN_BLK) {
+              // the block's rows from the caller's buffers, whole atoms from
+              // the one holding the piece's first row
+              const int32_t lead = sr & (kPadRows - 1);
+              int32_t y = ma.ch.brow[b] + row - lead;
+              for (int32_t x = sr - lead; x < sr + n; x += kPadRows, y += kPadRows) {
+#pragma unroll
+                for (int h = 0; h < HALVES; ++h) {
+                  ptx::tma_load_3d(kd + (x >> 3) * kAtomBytes + h * 1024, &ma.kblk, h * 64, g, y,
+                                   &full[st]);
+                  ptx::tma_load_3d(vd + (x >> 3) * kAtomBytes + h * 1024, &ma.vblk, h * 64, g, y,
+                                   &full[st]);
+                }
+                bytes += 2u * kPadRows * D * 2u;
+              }
+              return;
+            }
+          }
+          const bool pre = src == RUN_PREFIX;
+          int32_t y, z;
+          if (pre) {
+            y = row;
+            z = zpre;
+          } else {  // a ring piece lies within one page
+            y = page ? pg_mod(row, page, runs.plg) : row;
+            z = phys_of(row) * Hkv + g;
+          }
+          // copy whole atoms, from the one that holds the piece's first row
+          // (its row or slot minus the offset within the atom: same page)
+          const int32_t lead = sr & (kPadRows - 1);
+          sr -= lead;
+          y -= lead;
+          n += lead;
+          // Atom-map copies when the copy starts on an atom of its slab (prefix
+          // rows always; ring rows of whole-atom slabs, except the newest row
+          // of a plain decode, which starts an atom of the tile whatever its
+          // slot); otherwise 8-row boxes of each column block.
+          if ((pre ? ma.maps.prefix_atoms : ma.maps.ring_atoms) && (y & (kPadRows - 1)) == 0) {
+            if (!pre && ma.maps.page_box && lead == 0 && n == page) {
+              // a whole small page: one copy per operand
+              ptx::tma_load_5d(kd + (sr >> 3) * kAtomBytes, &ma.maps.kra[2], 0, 0, 0, y >> 3, z,
+                               &full[st]);
+              ptx::tma_load_5d(vd + (sr >> 3) * kAtomBytes, &ma.maps.vra[2], 0, 0, 0, y >> 3, z,
+                               &full[st]);
+              bytes += 2u * (uint32_t)page * D * 2u;
+              return;
+            }
+            while (n > 0) {  // 8 atoms or 1 atom per copy
+              const bool big = n >= kBox;
+              const int32_t rows = big ? kBox : kPadRows;
+              ptx::tma_load_5d(kd + (sr >> 3) * kAtomBytes, amap(pre, false, big ? 0 : 1), 0, 0, 0,
+                               y >> 3, z, &full[st]);
+              ptx::tma_load_5d(vd + (sr >> 3) * kAtomBytes, amap(pre, true, big ? 0 : 1), 0, 0, 0,
+                               y >> 3, z, &full[st]);
+              bytes += 2u * (uint32_t)rows * D * 2u;
+              sr += rows;
+              y += rows;
+              n -= rows;
+            }
+            return;
+          }
+          while (n > 0) {  // an atom of a column block per copy
+#pragma unroll
+            for (int h = 0; h < HALVES; ++h) {
+              ptx::tma_load_3d(kd + (sr >> 3) * kAtomBytes + h * 1024,
+                               pre ? &ma.maps.kpre8 : &ma.maps.kring8, h * 64, y, z, &full[st]);
+              ptx::tma_load_3d(vd + (sr >> 3) * kAtomBytes + h * 1024,
+                               pre ? &ma.maps.vpre8 : &ma.maps.vring8, h * 64, y, z, &full[st]);
+            }
+            bytes += 2u * kPadRows * D * 2u;
+            sr += kPadRows;
+            y += kPadRows;
+            n -= kPadRows;
           }
         });
         desc[st].mask[0] = (uint32_t)mask;
@@ -456,78 +560,6 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
           });
         }
         ptx::mbar_arrive_expect_tx(&full[st], bytes);
-        if (flags & TD_FIRST) load_q(st);
-        dec_range_pieces(runs, x0, x1, [&](int32_t src, int32_t row, int32_t sr, int32_t n) {
-          if (src == RUN_NEW) {  // the appended token, straight from the caller's rows
-            const uint16_t* kn = (const uint16_t*)a.knew + (size_t)pair * D;
-            const uint16_t* vn = (const uint16_t*)a.vnew + (size_t)pair * D;
-#pragma unroll
-            for (int h = 0; h < HALVES; ++h) {  // row sr % 8 == 0: the swizzle is the identity
-              ptx::bulk_g2s(kd + h * kHalfBytes + sr * 128, kn + h * 64, 128u, &full[st]);
-              ptx::bulk_g2s(vd + h * kHalfBytes + sr * 128, vn + h * 64, 128u, &full[st]);
-            }
-            return;
-          }
-          if constexpr (CHUNK) {
-            if (src == RUN_BLK) {
-              // the block's rows from the caller's buffers, whole atoms from
-              // the one holding the piece's first row
-              const int32_t lead = sr & (kPadRows - 1);
-              int32_t y = ma.ch.brow[b] + row - lead;
-              for (int32_t x = sr - lead; x < sr + n; x += kPadRows, y += kPadRows) {
-#pragma unroll
-                for (int h = 0; h < HALVES; ++h) {
-                  ptx::tma_load_3d(kd + h * kHalfBytes + x * 128, &ma.kblk, h * 64, g, y,
-                                   &full[st]);
-                  ptx::tma_load_3d(vd + h * kHalfBytes + x * 128, &ma.vblk, h * 64, g, y,
-                                   &full[st]);
-                }
-              }
-              return;
-            }
-          }
-          const CUtensorMap* km = src == RUN_PREFIX ? ma.maps.kpre : ma.maps.kring;
-          const CUtensorMap* vm = src == RUN_PREFIX ? ma.maps.vpre : ma.maps.vring;
-          int32_t y, z;
-          if (src == RUN_PREFIX) {
-            y = row;
-            z = zpre;
-          } else {  // a ring piece lies within one page
-            y = page ? row % page : row;
-            z = phys_of(row) * Hkv + g;
-          }
-          // copy whole atoms, from the one that holds the piece's first row
-          // (its row or slot minus the offset within the atom: same page)
-          const int32_t lead = sr & (kPadRows - 1);
-          sr -= lead;
-          y -= lead;
-          n += lead;
-          if (src == RUN_RING && ma.maps.page_box && lead == 0 && n == page) {
-            // a whole small page: one box per column block
-#pragma unroll
-            for (int h = 0; h < HALVES; ++h) {
-              ptx::tma_load_3d(kd + h * kHalfBytes + sr * 128, &ma.maps.kring_p, h * 64, y, z,
-                               &full[st]);
-              ptx::tma_load_3d(vd + h * kHalfBytes + sr * 128, &ma.maps.vring_p, h * 64, y, z,
-                               &full[st]);
-            }
-            return;
-          }
-          while (n > 0) {
-            const bool big = n >= kBox;
-            const int32_t rows = big ? kBox : kPadRows;
-#pragma unroll
-            for (int h = 0; h < HALVES; ++h) {
-              ptx::tma_load_3d(kd + h * kHalfBytes + sr * 128, big ? &km[0] : &km[1], h * 64, y, z,
-                               &full[st]);
-              ptx::tma_load_3d(vd + h * kHalfBytes + sr * 128, big ? &vm[0] : &vm[1], h * 64, y, z,
-                               &full[st]);
-            }
-            sr += rows;
-            y += rows;
-            n -= rows;
-          }
-        });
         ++i;
       }
       if (check) {
@@ -625,7 +657,8 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
         for (int idx = lane; idx < 16 * HALVES * 8; idx += 32) {
           const int r = idx / (HALVES * 8), h = (idx / 8) % HALVES, ch = idx % 8;
           if (!((vm >> r) & 1u))
-            *(uint4*)(vt + h * kHalfBytes + (R0 + r) * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
+            *(uint4*)(vt + ((R0 + r) >> 3) * kAtomBytes + h * 1024 + ((R0 + r) & 7) * 128 + ch * 16) =
+                make_uint4(0, 0, 0, 0);
         }
         __syncwarp();
         wrote = true;
@@ -636,7 +669,9 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
       for (int ks = 0; ks < KS; ++ks) {
         const int h = ks >> 2, chunk = (ks & 3) * 2 + kchk;
         uint32_t af[4];
-        ldsm4(kt_s + h * kHalfBytes + (R0 + krow) * 128 + ((chunk ^ sw) << 4), af);
+        ldsm4(kt_s + ((R0 + krow) >> 3) * kAtomBytes + h * 1024 + ((R0 + krow) & 7) * 128 +
+                  ((chunk ^ sw) << 4),
+              af);
         mma16816(c, af, st.qf[ks][0], st.qf[ks][1]);
       }
       const bool r0 = (vm >> g) & 1u, r1 = (vm >> (g + 8)) & 1u;
@@ -685,7 +720,9 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
       for (int mt = 0; mt < KS; ++mt) {
         const int h = mt >> 2, chunk = (mt & 3) * 2 + vchk;
         uint32_t af[4];
-        ldsm4_t(vt_s + h * kHalfBytes + (R0 + vrow) * 128 + ((chunk ^ sw) << 4), af);
+        ldsm4_t(vt_s + ((R0 + vrow) >> 3) * kAtomBytes + h * 1024 + ((R0 + vrow) & 7) * 128 +
+                    ((chunk ^ sw) << 4),
+                af);
         mma16816(st.o[mt], af, b0, b1);
       }
     }
@@ -702,7 +739,8 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
         const bool isv = x >= V16;
         const int xi = isv ? x - V16 : x;
         const uint4 val =
-            *(const uint4*)((isv ? vt : kt) + (xi / 8) * kHalfBytes + d.new_row * 128 + (xi % 8) * 16);
+            *(const uint4*)((isv ? vt : kt) + (d.new_row >> 3) * kAtomBytes + (xi / 8) * 1024 +
+                            (xi % 8) * 16);
         ((uint4*)((uint16_t*)(isv ? a.c.V : a.c.K) + row))[xi] = val;
       }
       if (lane == 0 && gg == 0) a.c.pos[pos_index(a.c, phys, slot)] = a.t[b];
@@ -1026,42 +1064,60 @@ bool make_decode_maps(const CacheDev& c, DecodeMaps* m) {
   const char* kring = (const char*)c.K + (size_t)c.rbase * row;
   const char* vring = (const char*)c.V + (size_t)c.rbase * row;
   const uint64_t nslab = (uint64_t)c.S * c.Hkv, nring = (uint64_t)c.nphys * c.Hkv;
-  bool ok = true;
-  for (int k = 0; k < 2; ++k) {
-    const uint32_t box = k == 0 ? (uint32_t)kBox : (uint32_t)kPadRows;
-    const int pr = PS_DMMA_L2_PROMOTION;
-    ok = ok && encode_map3d_bf16(&m->kpre[k], c.K, c.d, prows, nslab, row, prows * row, 64, box, 1,
-                                 pr);
-    ok = ok && encode_map3d_bf16(&m->vpre[k], c.V, c.d, prows, nslab, row, prows * row, 64, box, 1,
-                                 pr);
-    ok = ok && encode_map3d_bf16(&m->kring[k], kring, c.d, (uint64_t)c.page_rows, nring, row,
-                                 (uint64_t)c.rstride * row, 64, box, 1, pr);
-    ok = ok && encode_map3d_bf16(&m->vring[k], vring, c.d, (uint64_t)c.page_rows, nring, row,
-                                 (uint64_t)c.rstride * row, 64, box, 1, pr);
+  const uint64_t rstride = (uint64_t)c.rstride * row;
+  const int pr = PS_DMMA_L2_PROMOTION;
+  bool ok = encode_map3d_bf16(&m->kpre8, c.K, c.d, prows, nslab, row, prows * row, 64, kPadRows,
+                              1, pr) &&
+            encode_map3d_bf16(&m->vpre8, c.V, c.d, prows, nslab, row, prows * row, 64, kPadRows,
+                              1, pr) &&
+            encode_map3d_bf16(&m->kring8, kring, c.d, (uint64_t)c.page_rows, nring, row, rstride,
+                              64, kPadRows, 1, pr) &&
+            encode_map3d_bf16(&m->vring8, vring, c.d, (uint64_t)c.page_rows, nring, row, rstride,
+                              64, kPadRows, 1, pr);
+  const uint32_t halves = (uint32_t)(c.d / 64);
+  const uint64_t astr[4] = {row, 128, (uint64_t)kPadRows * row, 0};
+  // Prefix slabs: atoms covering rows [0, P_max) rounded up to a whole atom.
+  // A copy of the last atom reads up to 7 rows past P_max: the slab's own
+  // ring rows (unpaged), the next slab or the ring pages (paged).  Used only
+  // when even the last slab's last atom ends inside the buffer (V, the last
+  // region, has as many rows as K); otherwise prefix copies take the 3D maps.
+  m->prefix_atoms = 0;
+  const uint64_t pat = (uint64_t)(c.P_max > 0 ? (c.P_max + kPadRows - 1) / kPadRows : 1);
+  const uint64_t pre_rows = nslab * (uint64_t)c.pstride;
+  const uint64_t ring_end = (uint64_t)c.rbase + (nring - 1) * (uint64_t)c.rstride + c.page_rows;
+  const uint64_t buf_rows = pre_rows > ring_end ? pre_rows : ring_end;
+  if (ok && (nslab - 1) * prows + pat * kPadRows <= buf_rows) {
+    const uint64_t dims[5] = {64, (uint64_t)kPadRows, halves, pat, nslab};
+    const uint64_t str[4] = {astr[0], astr[1], astr[2], prows * row};
+    bool pok = true;
+    for (int k = 0; k < 2 && pok; ++k) {
+      const uint32_t box[5] = {64, (uint32_t)kPadRows, halves, k == 0 ? 8u : 1u, 1};
+      pok = encode_map_bf16(&m->kpa[k], c.K, 5, dims, str, box, pr) &&
+            encode_map_bf16(&m->vpa[k], c.V, 5, dims, str, box, pr);
+    }
+    m->prefix_atoms = pok ? 1 : 0;
   }
-  // Whole-tile maps (head_dim 128): dimensions (64 columns, rows, column
-  // block, slab); the column block is the outer box dimension, so one copy
-  // writes the tile's two 64-column blocks one after the other, as the kernel
-  // lays them out.
+  // Ring slabs: only when a slab (a page, or the whole ring) is whole atoms,
+  // so that no copy leaves it.
+  m->ring_atoms = 0;
   m->page_box = 0;
-  if (ok && c.page_table && c.page_rows >= 16 && c.page_rows < kBox && c.page_rows % kPadRows == 0) {
-    const int pr = PS_DMMA_L2_PROMOTION;
-    m->page_box = encode_map3d_bf16(&m->kring_p, kring, c.d, (uint64_t)c.page_rows, nring, row,
-                                    (uint64_t)c.rstride * row, 64, (uint32_t)c.page_rows, 1, pr) &&
-                  encode_map3d_bf16(&m->vring_p, vring, c.d, (uint64_t)c.page_rows, nring, row,
-                                    (uint64_t)c.rstride * row, 64, (uint32_t)c.page_rows, 1, pr);
-  }
-  m->whole = 0;
-  if (ok && c.d == 128) {
-    const uint32_t box[4] = {64, (uint32_t)kBox, 2, 1};
-    const uint64_t dp[4] = {64, prows, 2, nslab}, sp[3] = {row, 128, prows * row};
-    const uint64_t dr[4] = {64, (uint64_t)c.page_rows, 2, nring},
-                   sr[3] = {row, 128, (uint64_t)c.rstride * row};
-    const int pr = PS_DMMA_L2_PROMOTION;
-    m->whole = encode_map_bf16(&m->kpre_w, c.K, 4, dp, sp, box, pr) &&
-               encode_map_bf16(&m->vpre_w, c.V, 4, dp, sp, box, pr) &&
-               encode_map_bf16(&m->kring_w, kring, 4, dr, sr, box, pr) &&
-               encode_map_bf16(&m->vring_w, vring, 4, dr, sr, box, pr);
+  if (ok && c.page_rows % kPadRows == 0) {
+    const uint64_t dims[5] = {64, (uint64_t)kPadRows, halves,
+                              (uint64_t)(c.page_rows / kPadRows), nring};
+    const uint64_t str[4] = {astr[0], astr[1], astr[2], rstride};
+    bool rok = true;
+    for (int k = 0; k < 2 && rok; ++k) {
+      const uint32_t box[5] = {64, (uint32_t)kPadRows, halves, k == 0 ? 8u : 1u, 1};
+      rok = encode_map_bf16(&m->kra[k], kring, 5, dims, str, box, pr) &&
+            encode_map_bf16(&m->vra[k], vring, 5, dims, str, box, pr);
+    }
+    m->ring_atoms = rok ? 1 : 0;
+    if (rok && c.page_table && c.page_rows > kPadRows && c.page_rows < kBox) {
+      const uint32_t box[5] = {64, (uint32_t)kPadRows, halves,
+                               (uint32_t)(c.page_rows / kPadRows), 1};
+      m->page_box = encode_map_bf16(&m->kra[2], kring, 5, dims, str, box, pr) &&
+                    encode_map_bf16(&m->vra[2], vring, 5, dims, str, box, pr);
+    }
   }
   return ok;
 }

@@ -55,6 +55,7 @@ struct DecRuns {
   int32_t padded;     // padded rows of the pair (a multiple of 8)
   int32_t rows;       // valid rows of the pair
   int32_t page;       // ring page rows of a paged cache, 0 when unpaged
+  int32_t plg;        // log2(page) for a power-of-two page, else -1 (divisions)
   int32_t ring_ok;    // 0 if the window reaches below what the ring holds
   // chunk mode (dec_runs_chunk; a plain decode leaves qb0 = qd0 = qd1 = 0 and
   // no tile is query-dependent): the group's queries are at t0 + qi0 + k,
@@ -65,6 +66,23 @@ struct DecRuns {
   int32_t qi0, qnq, qW, rhead;
   int32_t qd0, qd1, qb0;
 };
+
+// log2 of a power-of-two page size, -1 otherwise; x mod page and x / page
+// with shifts when it is one (the common sizes), divisions otherwise.
+__host__ __device__ __forceinline__ int32_t page_log2(int32_t page) {
+  if (page <= 0 || (page & (page - 1))) return -1;
+#ifdef __CUDA_ARCH__
+  return __ffs(page) - 1;
+#else
+  return __builtin_ctz((unsigned)page);
+#endif
+}
+__host__ __device__ __forceinline__ int32_t pg_mod(int32_t x, int32_t page, int32_t lg) {
+  return lg >= 0 ? (x & (page - 1)) : x % page;
+}
+__host__ __device__ __forceinline__ int32_t pg_div(int32_t x, int32_t page, int32_t lg) {
+  return lg >= 0 ? (x >> lg) : x / page;
+}
 
 // Pages whose edges fall on atom boundaries keep the unpaged layout.
 __host__ __device__ __forceinline__ bool page_aligned(int32_t page) {
@@ -98,6 +116,7 @@ __host__ __device__ __forceinline__ DecRuns dec_runs(const DevMeta& m, int32_t W
     r.src[i] = 0; r.row0[i] = 0; r.len[i] = 0; r.pstart[i] = 0;
   }
   r.page = page;
+  r.plg = page_log2(page);
   r.ring_ok = 1;
   // the window part: positions [lo, hi] of the ring, oldest at slot `head`
   const int64_t base = m.next_pos - m.count;
@@ -179,6 +198,7 @@ __host__ __device__ __forceinline__ DecRuns dec_runs_chunk(const DevMeta& m, int
     r.src[i] = 0; r.row0[i] = 0; r.len[i] = 0; r.pstart[i] = 0;
   }
   r.page = page;
+  r.plg = page_log2(page);
   r.ring_ok = 1;
   const int64_t base = m.next_pos - m.count;
   const int64_t qlo = t0 + i0 - (int64_t)W + 1;
@@ -298,7 +318,7 @@ __host__ __device__ __forceinline__ bool dec_range_whole(const DecRuns& r, int32
         x0 + TR <= r.pstart[k] + r.len[k]) {
       const int32_t rw = r.row0[k] + (x0 - r.pstart[k]);
       const int32_t pg = r.src[k] == RUN_RING ? r.page : 0;
-      if (pg <= 0 || rw % pg + TR <= pg) {
+      if (pg <= 0 || pg_mod(rw, pg, r.plg) + TR <= pg) {
         whole = true;
         *src = r.src[k];
         *row = rw;
@@ -330,7 +350,7 @@ __host__ __device__ __forceinline__ void dec_range_pieces(const DecRuns& r, int3
       for (int32_t x = a; x < b;) {  // one piece, or one per page edge crossed
         int32_t n = b - x;
         if (pg > 0) {
-          const int32_t to_edge = pg - row % pg;
+          const int32_t to_edge = pg - pg_mod(row, pg, r.plg);
           if (n > to_edge) n = to_edge;
         }
         f(src, row, x - x0, n);
@@ -340,7 +360,7 @@ __host__ __device__ __forceinline__ void dec_range_pieces(const DecRuns& r, int3
     } else {
       // small pages: the first (partial) page, then page after page, each
       // from its own atom
-      const int32_t f0 = pg - row0 % pg;
+      const int32_t f0 = pg - pg_mod(row0, pg, r.plg);
       const int32_t first = f0 < len ? f0 : len;
       const int32_t step = pad8(pg);
       int32_t pos = ps, row = row0, n = first;

@@ -69,13 +69,20 @@ size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int sm_count);
 // both column blocks of a 128-column row, which fills a whole tile with one
 // copy.
 struct DecodeMaps {
-  CUtensorMap kpre[2], vpre[2], kring[2], vring[2];
-  CUtensorMap kpre_w, vpre_w, kring_w, vring_w;
-  // paged caches with pages of 16..56 rows (a multiple of 8): a box of one
-  // page of one 64-column block
-  CUtensorMap kring_p, vring_p;
-  int whole;     // 1 if the whole-tile maps exist (head_dim 128)
-  int page_box;  // 1 if the one-page maps exist
+  // Atom maps: 5D views (64 columns, 8 rows, 64-column block, atom of the
+  // slab, slab) of the prefix slabs and of the ring slabs, 128-byte swizzle.
+  // A box of A atoms lands as A groups of [column block][8 rows] -- the
+  // decode kernel's tile layout -- so one copy brings A atoms of every column
+  // block.  Boxes of 8 atoms (a 64-row tile) and 1 atom; ring slabs also one
+  // page (page_rows / 8 atoms; paged caches with 8 < page_rows < 64).
+  CUtensorMap kpa[2], vpa[2];  // prefix slabs (prefix_atoms)
+  CUtensorMap kra[3], vra[3];  // ring slabs (ring_atoms)
+  // 3D maps with one 8-row box of one 64-column block: copies that do not
+  // start on an atom of their slab, and ring slabs that are not whole atoms
+  CUtensorMap kpre8, vpre8, kring8, vring8;
+  int prefix_atoms;  // 1 if the prefix atom maps exist (every prefix atom inside the buffer)
+  int ring_atoms;  // 1 if the ring atom maps exist (page_rows a multiple of 8)
+  int page_box;    // 1 if the one-page ring atom maps exist
 };
 bool make_decode_maps(const CacheDev& c, DecodeMaps* m);
 // maps: the cache's decode maps (bf16 caches; NULL for float32).

@@ -177,6 +177,16 @@ __device__ __forceinline__ void tma_load_4d(void* smem_dst, const void* tmap, in
       : "memory");
 }
 
+// 5-D tiled TMA load (no multicast) of the box at (x, y, z, w, v).
+__device__ __forceinline__ void tma_load_5d(void* smem_dst, const void* tmap, int32_t x, int32_t y,
+                                            int32_t z, int32_t w, int32_t v, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(smem_dst)),
+      "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(w), "r"(v), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // ------------------------------------------------------------ tensor memory --
 // Allocation is warp-wide; the allocated base address is written to *slot.
 __device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
