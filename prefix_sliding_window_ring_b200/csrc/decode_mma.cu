@@ -19,12 +19,15 @@
 // 8-row atom that its row or slot has modulo 8, so that whole atoms can be
 // loaded by tensor-map copies; no atom holds rows of two pieces.
 //
-// Streaming.  One lane of warp kMW is the producer: per tile it issues
-// tensor-map copies (cp.async.bulk.tensor, 128-byte swizzle, no multicast) of
-// the atoms holding each piece's K and V rows -- 64-row boxes, then 8-row
-// boxes for the rest -- into a kStages-deep ring of shared-memory stages; the
-// pair's q rows come with the first tile of a piece and the appended token of
-// a decode step by plain bulk copies.  Rows a box reads before or after its
+// Streaming.  Two producers (one lane of each of warps kMW and kMW + 1) take
+// alternate tiles: per tile a producer issues tensor-map copies
+// (cp.async.bulk.tensor, 128-byte swizzle, no multicast) of the 8-row atoms
+// holding each piece's K and V rows into a kStages-deep ring of shared-memory
+// stages -- one copy per 64-row tile, per small page or per atom, all column
+// blocks at once through 5D maps of the prefix and ring slabs (8-row boxes of
+// one column block where a copy cannot start on an atom of its slab) -- and
+// the pair's q rows with the first tile of a piece and the appended token of a
+// decode step by plain bulk copies.  Rows a copy brings before or after its
 // piece are masked.
 // No evicted row is a valid row of any tile ("Prefix Sliding" digest, section
 // 06: the prefix and the window are walked separately).
@@ -78,7 +81,8 @@ namespace {
 using namespace dec;
 
 constexpr int kMW = 4;                      // consumer warps
-constexpr int kThreadsM = (kMW + 1) * 32;   // plus one producer warp
+constexpr int kProd = 2;                    // producer warps (one lane each), alternate tiles
+constexpr int kThreadsM = (kMW + kProd) * 32;
 constexpr int kTR = PS_DMMA_TR;             // rows per tile
 constexpr int kStagesM = PS_DMMA_STAGES;
 constexpr int kGroups = kTR / 16;           // 16-row MMA groups per tile
@@ -231,8 +235,8 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
   Merge& sm = *reinterpret_cast<Merge*>(CL ? kbuf : sm_own);
   __shared__ float pub_ml[G][2];  // cluster: this CTA's merged (max, sum) per head
   // paged cache: the page-table row of the piece's sequence (read by the producer only)
-  __shared__ __align__(16) int32_t tbl[kTblMax + 4];
-  __shared__ __align__(8) uint64_t tbl_bar;
+  __shared__ __align__(16) int32_t tbl[kProd][kTblMax + 4];  // one per producer
+  __shared__ __align__(8) uint64_t tbl_bar[kProd];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Hkv = a.c.Hkv;
@@ -269,7 +273,7 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
     ptx::mbar_init(&sync_m, kMW);
     ptx::mbar_init(&pub_bar, CL ? a.csize - 1 : 1);
     ptx::mbar_init(&done_bar, 1);
-    ptx::mbar_init(&tbl_bar, 1);
+    for (int p = 0; p < kProd; ++p) ptx::mbar_init(&tbl_bar[p], 1);
     abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -310,9 +314,12 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
   // the first piece overlaps the previous grid's tail.
   ptx::pdl_launch_dependents();
 
-  if (warp == kMW) {
+  if (warp >= kMW) {
     if (lane != 0) return;
-    // ------------------------------------------------------------ producer --
+    // ----------------------------------------------------------- producers --
+    // Producer pw issues the tiles i with i % kProd == pw; both walk every
+    // piece and tile so that each knows every tile's stage and phase.
+    const int pw = warp - kMW;
     const bool step = a.knew != nullptr;
     const int32_t page = a.c.page_table ? a.c.page_rows : 0;
     int i = 0;  // tiles handed out so far
@@ -377,10 +384,10 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
         const int lead = (int)((src - src16) / 4);
         const uint32_t bytes = (uint32_t)(((src - src16) + (size_t)a.c.npg * 4 + 15) & ~(size_t)15);
         if (tbl_n > 0) fence_proxy_async_smem();  // earlier reads before the copy overwrites
-        ptx::mbar_arrive_expect_tx(&tbl_bar, bytes);
-        ptx::bulk_g2s(tbl, (const void*)src16, bytes, &tbl_bar);
-        if (ptx::mbar_wait_bounded(&tbl_bar, tbl_n & 1, &abort_flag, kWaitLimitCycles)) {
-          tab = tbl + lead;
+        ptx::mbar_arrive_expect_tx(&tbl_bar[pw], bytes);
+        ptx::bulk_g2s(tbl[pw], (const void*)src16, bytes, &tbl_bar[pw]);
+        if (ptx::mbar_wait_bounded(&tbl_bar[pw], tbl_n & 1, &abort_flag, kWaitLimitCycles)) {
+          tab = tbl[pw] + lead;
         } else {
           alive = false;
         }
@@ -395,6 +402,10 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
                    : (isv ? &ma.maps.vra[k] : &ma.maps.kra[k]);
       };
       for (int32_t k = 0; k < nt && alive; ++k) {
+        if (i % kProd != pw) {  // the other producer's tile
+          ++i;
+          continue;
+        }
         const int32_t x0 = xs + k * kTR, x1 = min(x0 + kTR, xe);
         const int st = i % kStagesM;
         if (i >= kStagesM && !ptx::mbar_wait_bounded(&empty[st], ((i / kStagesM) - 1) & 1,
@@ -562,7 +573,7 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
         ptx::mbar_arrive_expect_tx(&full[st], bytes);
         ++i;
       }
-      if (check) {
+      if (check && pw == 0) {
         const DevMeta md = a.c.meta[s];
         DevMeta me = md;  // the device record before this launch (a step advances it by one)
         if (step) {
@@ -575,8 +586,8 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
             me.count != m.count || me.owner != m.owner)
           bad = true;
       }
-      if (bad) atomicOr(a.c.err, ERR_BATCH);
-      if (!runs.ring_ok) atomicOr(a.c.err, ERR_RING);
+      if (pw == 0 && bad) atomicOr(a.c.err, ERR_BATCH);
+      if (pw == 0 && !runs.ring_ok) atomicOr(a.c.err, ERR_RING);
     };
     if (CL) {
       const int pair = blockIdx.x / a.csize, rank = (int)ptx::cluster_ctarank();
@@ -591,7 +602,7 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
         piece(pt.b, pt.g, pt.tph, j0, j1, -1, true);
       }
     }
-    if (alive) {  // end marker: a descriptor with no bytes
+    if (alive && i % kProd == pw) {  // end marker (its producer): a descriptor with no bytes
       wait_primary();
       const int st = i % kStagesM;
       if (i < kStagesM || ptx::mbar_wait_bounded(&empty[st], ((i / kStagesM) - 1) & 1,
@@ -607,7 +618,8 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
     if (abort_flag) {  // let the copies already issued land before the CTA exits
       int quiet = 0;
       for (int k = max(0, i - kStagesM); k < i; ++k)
-        ptx::mbar_wait_bounded(&full[k % kStagesM], (k / kStagesM) & 1, &quiet, kWaitLimitCycles);
+        if (k % kProd == pw)
+          ptx::mbar_wait_bounded(&full[k % kStagesM], (k / kStagesM) & 1, &quiet, kWaitLimitCycles);
     }
     return;
   }
