@@ -198,11 +198,15 @@ struct MmaState {
 // CHUNK: chunk mode (a pair is a group of a block's queries and one kv head;
 // its columns are the group's queries x gq heads; always with CL).
 // CL: cluster mode.  Pair p is streamed by the csize CTAs of cluster p, CTA
-// rank r taking an equal share of its padded rows (dec_cluster_share); each CTA
-// publishes its merged state in its own shared memory, and rank 0 reads its
-// peers' states through distributed shared memory, writes the pair's output
-// and (decode step) commits the sequence's bookkeeping -- no partials in global
-// memory, no second grid.  Otherwise the flattened split with k_decode_merge.
+// rank r taking an equal share of its padded rows (dec_cluster_share).  Each
+// CTA then pushes its merged state into its peers' shared memory (remote
+// stores: its (max, sum) per column to all, its accumulator values of output
+// slice r to rank r), waits for theirs and combines its own slice of the
+// pair's output from local shared memory -- no partials in global memory, no
+// second grid, no CTA reading another's memory.  The sequence's record is
+// checked (and a decode step's new state committed) by rank 0 of kv head 0
+// once its copies are issued.  Otherwise the flattened split with
+// k_decode_merge.
 template <int D, int G, bool CL, bool CHUNK>
 __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
     k_decode_mma(const __grid_constant__ MmaArgs<CHUNK> ma) {
@@ -221,8 +225,8 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
   uint8_t* const vbuf = kbuf + kStagesM * kTileBytes;
   uint8_t* const qbuf = vbuf + kStagesM * kTileBytes;  // [kStagesM][G][D] bf16
   __shared__ __align__(8) uint64_t full[kStagesM], empty[kStagesM];
-  __shared__ __align__(8) uint64_t sync_a, sync_b, sync_c, sync_m;
-  __shared__ __align__(8) uint64_t pub_bar, done_bar;  // cluster: peers published / rank 0 done
+  __shared__ __align__(8) uint64_t sync_a, sync_b, sync_c, sync_m, sync_w;
+  __shared__ __align__(8) uint64_t pub_bar;  // cluster: the peers' states have arrived
   __shared__ TileDescM desc[kStagesM];
   __shared__ int abort_flag;
   // The warps' merge buffer.  In cluster mode a CTA streams one piece, so
@@ -233,7 +237,13 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
   static_assert(sizeof(Merge) <= (size_t)kStagesM * kTileBytes, "merge buffer fits the K stages");
   __shared__ __align__(16) uint8_t sm_own[CL ? 16 : sizeof(Merge)];
   Merge& sm = *reinterpret_cast<Merge*>(CL ? kbuf : sm_own);
-  __shared__ float pub_ml[G][2];  // cluster: this CTA's merged (max, sum) per head
+  __shared__ float pub_ml[G][2];  // cluster: this CTA's merged (max, sum) per column
+  // cluster: the states the peers push here -- each rank's (max, sum) per
+  // column, and its accumulator values of the output slice this CTA combines
+  // (slice r of the G*D outputs belongs to rank r)
+  __shared__ float rcv_ml[kMaxCluster][G][2];
+  __shared__ float rcv_o[G * D];
+  __shared__ float cw[kMaxCluster][G];  // each rank's combine weight per column
   // paged cache: the page-table row of the piece's sequence (read by the producer only)
   __shared__ __align__(16) int32_t tbl[kProd][kTblMax + 4];  // one per producer
   __shared__ __align__(8) uint64_t tbl_bar[kProd];
@@ -271,8 +281,8 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
     ptx::mbar_init(&sync_b, kMW);
     ptx::mbar_init(&sync_c, kMW);
     ptx::mbar_init(&sync_m, kMW);
+    ptx::mbar_init(&sync_w, kMW);
     ptx::mbar_init(&pub_bar, CL ? a.csize - 1 : 1);
-    ptx::mbar_init(&done_bar, 1);
     for (int p = 0; p < kProd; ++p) ptx::mbar_init(&tbl_bar[p], 1);
     abort_flag = 0;
     ptx::fence_mbar_init();
@@ -336,7 +346,10 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
     // One piece of pair (b, g): its tiles [j0, j1) (flattened split, tph
     // tiles in all), or with rank >= 0 the cluster share of CTA `rank`.
     // check: compare the device record with the launch's state (flattened
-    // split; in cluster mode rank 0 of kv head 0 does it at the end).
+    // split: every piece; cluster mode: rank 0 of kv head 0, which also
+    // commits a decode step's new state -- no other CTA of the launch reads
+    // or writes the record, so it is done once the copies are issued, off the
+    // output's path).
     auto piece = [&](int b, int g, int32_t tph, int32_t j0, int32_t j1, int rank, bool check) {
       const int s = a.seq[b];
       DevMeta m;
@@ -585,6 +598,16 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
         if (me.next_pos != m.next_pos || me.P != m.P || me.head != m.head ||
             me.count != m.count || me.owner != m.owner)
           bad = true;
+        if (CL && step) {
+          DevMeta mn;
+          memset(&mn, 0, sizeof(mn));
+          mn.next_pos = m.next_pos;
+          mn.P = m.P;
+          mn.head = m.head;
+          mn.count = m.count;
+          mn.owner = m.owner;
+          a.c.meta[s] = mn;
+        }
       }
       if (pw == 0 && bad) atomicOr(a.c.err, ERR_BATCH);
       if (pw == 0 && !runs.ring_ok) atomicOr(a.c.err, ERR_RING);
@@ -592,7 +615,7 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
     if (CL) {
       const int pair = blockIdx.x / a.csize, rank = (int)ptx::cluster_ctarank();
       const int b = pair / Hkv, g = pair % Hkv;
-      piece(b, g, 0, 0, 0, rank, false);
+      piece(b, g, 0, 0, 0, rank, rank == 0 && g == 0);
     } else {
       const int32_t x1 = range_start(blockIdx.x + 1, R, NC);
       for (int32_t x = range_start(blockIdx.x, R, NC); x < x1 && alive;) {
@@ -829,68 +852,75 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
       if (!csync(&sync_c, 0)) stopped = true;
     }
     const int rank = (int)ptx::cluster_ctarank(), C = a.csize;
-    if (!stopped && rank != 0) {
-      // publish to rank 0, then keep this CTA's shared memory alive until it has read it
-      if (threadIdx.x == 0) {
-        ptx::fence_acq_rel_cluster();
-        ptx::mbar_arrive_cluster(ptx::map_to_rank(&pub_bar, 0));
-        ptx::mbar_wait_cluster_bounded(&done_bar, 0, &abort_flag, kWaitLimitCycles);
+    const int SL = G * D / C;  // outputs per slice
+    if (!stopped) {
+      // push: every peer gets this CTA's (max, sum) and the values of its slice
+      for (int idx = threadIdx.x; idx < G * D; idx += kMW * 32) {
+        const int r = idx / SL;
+        if (r != rank) {
+          const int h = idx / D, e = idx % D;
+          ptx::st_cluster_f32(ptx::map_to_rank(&rcv_o[rank * SL + (idx - r * SL)], r),
+                              sm.o[0][h][e]);
+        }
       }
-    } else if (!stopped) {
+      for (int idx = threadIdx.x; idx < C * G * 2; idx += kMW * 32) {
+        const int r = idx / (G * 2), h = (idx / 2) % G, w = idx & 1;
+        if (r != rank) ptx::st_cluster_f32(ptx::map_to_rank(&rcv_ml[rank][h][w], r), pub_ml[h][w]);
+      }
+      // every thread's stores before the arrivals (cumulative release by thread 0)
+      if (csync(&sync_w, 0)) {
+        if (threadIdx.x == 0) {
+          ptx::fence_acq_rel_cluster();
+          for (int r = 0; r < C; ++r)
+            if (r != rank) ptx::mbar_arrive_cluster(ptx::map_to_rank(&pub_bar, r));
+        }
+      } else {
+        stopped = true;
+      }
+    }
+    if (!stopped) {
+      // the peers' states are here once all C - 1 have arrived
       const bool ok = ptx::mbar_wait_cluster_bounded(&pub_bar, 0, &abort_flag, kWaitLimitCycles);
       if (__all_sync(FULL, ok)) {
         const int pair = blockIdx.x / C, b = pair / Hkv, gg = pair % Hkv;
         const int ncols = nq_of(b) << lgq();  // valid columns of the pair
-        for (int idx = threadIdx.x; idx < ncols * D; idx += kMW * 32) {
-          const int h = idx / D, e = idx % D;
-          float mr[kMaxCluster], lr[kMaxCluster], orr[kMaxCluster];
+        // each rank's weight 2^(m_r - M) / L per column, L = sum_r l_r 2^(m_r - M)
+        if (threadIdx.x < ncols) {
+          const int h = threadIdx.x;
+          float mr[kMaxCluster], lr[kMaxCluster];
           float M = -INFINITY;
 #pragma unroll
           for (int r = 0; r < kMaxCluster; ++r) {
             if (r < C) {
-              mr[r] = r == 0 ? pub_ml[h][0] : ptx::ld_cluster_f32(ptx::map_to_rank(&pub_ml[h][0], r));
-              lr[r] = r == 0 ? pub_ml[h][1] : ptx::ld_cluster_f32(ptx::map_to_rank(&pub_ml[h][1], r));
-              orr[r] = r == 0 ? sm.o[0][h][e] : ptx::ld_cluster_f32(ptx::map_to_rank(&sm.o[0][h][e], r));
+              mr[r] = r == rank ? pub_ml[h][0] : rcv_ml[r][h][0];
+              lr[r] = r == rank ? pub_ml[h][1] : rcv_ml[r][h][1];
               M = fmaxf(M, mr[r]);
             }
           }
-          float L = 0.f, A = 0.f;
+          float L = 0.f;
 #pragma unroll
           for (int r = 0; r < kMaxCluster; ++r) {
             if (r < C) {
-              const float w = (mr[r] == -INFINITY) ? 0.f : exp2f(mr[r] - M);
-              L += lr[r] * w;
-              A += orr[r] * w;
+              mr[r] = (mr[r] == -INFINITY) ? 0.f : exp2f(mr[r] - M);
+              L += lr[r] * mr[r];
             }
           }
-          store_out<uint16_t>((uint16_t*)a.out + qo_off(b, gg, h) + e, A / L);
+          const float inv = 1.f / L;
+#pragma unroll
+          for (int r = 0; r < kMaxCluster; ++r)
+            if (r < C) cw[r][h] = mr[r] * inv;
         }
-        // the peers' shared memory has been read: let them exit
-        if (csync(&sync_c, np == 0 ? 1 : 0) && threadIdx.x == 0) {
-          for (int r = 1; r < C; ++r) ptx::mbar_arrive_cluster(ptx::map_to_rank(&done_bar, r));
-          if (gg == 0) {
-            // the sequence's bookkeeping: check the device record, then (decode
-            // step) commit the state after the append
-            const int s = a.seq[b];
-            const DevMeta md = a.c.meta[s];
-            DevMeta m;
-            memset(&m, 0, sizeof(m));
-            m.next_pos = next_pos_of(b);
-            m.P = a.P[b];
-            m.head = a.head[b];
-            m.count = a.count[b];
-            m.owner = a.owner[b];
-            DevMeta me = md;
-            if (a.knew != nullptr) {
-              const int64_t W = a.c.W, cn = (int64_t)md.count + 1;
-              me.next_pos = md.next_pos + 1;
-              me.count = (int32_t)(cn < W ? cn : W);
-              me.head = (int32_t)((md.head + (cn > W ? 1 : 0)) % W);
+        if (csync(&sync_c, np == 0 ? 1 : 0)) {
+          // this CTA's slice of the outputs
+          for (int k = threadIdx.x; k < SL; k += kMW * 32) {
+            const int idx = rank * SL + k, h = idx / D, e = idx % D;
+            if (h < ncols) {
+              float A = 0.f;
+#pragma unroll
+              for (int r = 0; r < kMaxCluster; ++r)
+                if (r < C) A += (r == rank ? sm.o[0][h][e] : rcv_o[r * SL + k]) * cw[r][h];
+              store_out<uint16_t>((uint16_t*)a.out + qo_off(b, gg, h) + e, A);
             }
-            if (me.next_pos != m.next_pos || me.P != m.P || me.head != m.head ||
-                me.count != m.count || me.owner != m.owner)
-              atomicOr(a.c.err, ERR_BATCH);
-            if (a.knew != nullptr) a.c.meta[s] = m;
           }
         }
       }
