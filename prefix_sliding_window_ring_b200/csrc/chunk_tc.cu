@@ -102,6 +102,13 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// max of three (max.f32 with three sources, sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
@@ -327,14 +334,18 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
             if (!vis) x[c] = -INFINITY;
           }
         }
-        // row max of the raw scores (the scale is positive), as a tree
+        // row max of the raw scores (the scale is positive), as a tree of
+        // three-input maxima
         float t8[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) t8[u] = x[u];
+        for (int u = 0; u < 8; ++u) t8[u] = fmax3(x[u], x[8 + u], x[16 + u]);
 #pragma unroll
-        for (int c = 8; c < 64; ++c) t8[c & 7] = fmaxf(t8[c & 7], x[c]);
-        mloc = fmaxf(fmaxf(fmaxf(t8[0], t8[1]), fmaxf(t8[2], t8[3])),
-                     fmaxf(fmaxf(t8[4], t8[5]), fmaxf(t8[6], t8[7])));
+        for (int u = 0; u < 8; ++u) t8[u] = fmax3(t8[u], x[24 + u], x[32 + u]);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) t8[u] = fmax3(t8[u], x[40 + u], x[48 + u]);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) t8[u] = fmaxf(t8[u], x[56 + u]);
+        mloc = fmax3(fmax3(t8[0], t8[1], t8[2]), fmax3(t8[3], t8[4], t8[5]), fmaxf(t8[6], t8[7]));
       }
       xchg[st][half][r] = mloc;
       pair_sync();
@@ -367,15 +378,22 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
       }
       m_run = m_new;
       const float mu = m_run == -INFINITY ? 0.f : m_run;
-      float s8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      // two columns per packed f32x2 FMA / add (sm_100): scale and shift,
+      // then the running sums; the exponentials one by one
+      const float2 sc2 = make_float2(sc, sc), nmu2 = make_float2(-mu, -mu);
+      float2 s4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                      make_float2(0.f, 0.f)};
       uint32_t pk[32];
 #pragma unroll
       for (int c = 0; c < 64; c += 2) {
-        const float p0 = ex2(fmaf(x[c], sc, -mu)), p1 = ex2(fmaf(x[c + 1], sc, -mu));
-        s8[(c >> 1) & 7] += p0 + p1;
+        const float2 y = __ffma2_rn(make_float2(x[c], x[c + 1]), sc2, nmu2);
+        const float p0 = ex2(y.x), p1 = ex2(y.y);
+        s4[(c >> 1) & 3] = __fadd2_rn(s4[(c >> 1) & 3], make_float2(p0, p1));
         pk[c >> 1] = pack_bf16(p0, p1);
       }
-      l_run += ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
+      const float2 s01 = __fadd2_rn(s4[0], s4[1]), s23 = __fadd2_rn(s4[2], s4[3]);
+      const float2 sall = __fadd2_rn(s01, s23);
+      l_run += sall.x + sall.y;
       // P occupies the first 64 columns of the S buffer; my 64 keys are 32 of them.
       // The partner read its scores from those columns before the pair barrier.
       ptx::tmem_st32(tmem + lane_base + col_s(st) + half * 32, pk);
