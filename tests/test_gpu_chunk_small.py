@@ -120,9 +120,17 @@ def test_short_windows_and_edges(W, P, L, n):
     run_blocks(W, P, [(L, n), (L + 3, max(1, n - 2))], Hkv=2, small_max=32)
 
 
-@pytest.mark.parametrize("page", [8, 16, 256])
+@pytest.mark.parametrize("page", [4, 8, 16, 256])
 def test_paged_ring(page):
+    """Pages of 4 rows start an atom each (their own layout); 8, 16 and 256
+    keep the unpaged one."""
     run_blocks(512, 64, [(1000, 3), (37, 12), (600, 1)], Hkv=4, page=page, h0=77)
+
+
+def test_paged_ring_non_power_of_two_pages():
+    """24-row pages: a multiple of 8 (the unpaged layout) whose page numbers
+    need a division, not a shift."""
+    run_blocks(480, 40, [(900, 5), (100, 9), (481, 1)], Hkv=4, page=24, h0=13)
 
 
 def test_mixed_batch():
