@@ -638,6 +638,63 @@ def prefill_measure(steps: int):
 PR_P = 4096  # prompt length of the prompt-prefill measurement
 
 
+def paged_prefill_measure(steps: int):
+    """The chunk workload (4 sequences x 2048-query blocks at t0=100000,
+    W=4096, P=256, Hq=16, Hkv=8, d=128, bf16) on an unpaged cache and on paged
+    caches with 256-, 64- and 16-row pages (each window imported whole).
+    One step = one ps_attend_chunk_batch call."""
+    import torch
+
+    import synth
+    from prefix_sliding_window_ring_b200 import PS_BF16, Cache
+    peak, _ = load_bf16_peak()
+
+    def dev(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+
+    Wp = 4096
+    ids = list(range(PF_SEQS))
+    kw_ = dev(np.stack([synth.rows(SEED, synth.TID_K, s, HKV, PF_T0 - Wp, Wp, D, "bf16")
+                        for s in range(PF_SEQS)]))
+    vw_ = dev(np.stack([synth.rows(SEED, synth.TID_V, s, HKV, PF_T0 - Wp, Wp, D, "bf16")
+                        for s in range(PF_SEQS)]))
+    q = torch.cat([dev(synth.rows(SEED, synth.TID_Q, s, HQ, PF_T0, PF_N, D, "bf16"))
+                   for s in range(PF_SEQS)])
+    kb = torch.cat([dev(synth.rows(SEED, synth.TID_K, s, HKV, PF_T0, PF_N, D, "bf16"))
+                    for s in range(PF_SEQS)])
+    vb = torch.cat([dev(synth.rows(SEED, synth.TID_V, s, HKV, PF_T0, PF_N, D, "bf16"))
+                    for s in range(PF_SEQS)])
+    o = torch.empty_like(q)
+    scale = 1.0 / math.sqrt(D)
+    res = {"workload": f"{PF_SEQS} sequences x {PF_N}-query blocks at t0={PF_T0}, W={Wp}, "
+                       f"P={PF_P}, Hq={HQ} Hkv={HKV} d={D}, bf16",
+           "unit": "ms per call"}
+    for page in (0, 256, 64, 16):
+        c = Cache(Wp, PF_P, HKV, D, PS_BF16, PF_SEQS, page_rows=page,
+                  num_pages=PF_SEQS * Wp // page if page else 0)
+        for s in range(PF_SEQS):
+            c.seq_reset(s, (977 * s) % Wp)
+            c.prefill_prefix(s, dev(synth.rows(SEED, synth.TID_K, s, HKV, 0, PF_P, D, "bf16")),
+                             dev(synth.rows(SEED, synth.TID_V, s, HKV, 0, PF_P, D, "bf16")), PF_P)
+            c.import_window(s, PF_T0, kw_[s].contiguous(), vw_[s].contiguous(), Wp, (977 * s) % Wp)
+
+        def step(i, st=None):
+            c.attend_chunk_batch(ids, [PF_T0] * PF_SEQS, [PF_N] * PF_SEQS, q, kb, vb, HQ, scale,
+                                 o, 0, st)
+
+        for i in range(3):
+            step(i)
+        torch.cuda.synchronize()
+        if c.device_error():
+            raise RuntimeError("device error word set by a chunk call")
+        ms = min(time_graph(torch, step, steps) for _ in range(2))
+        tf = prefill_flops(Wp) / (ms / 1e3) / 1e12
+        res[f"page_rows_{page}" if page else "unpaged"] = {
+            "ms": round(ms, 4), "achieved_tflops": round(tf, 1), "frac": round(tf / peak, 4)}
+        c.close()
+    return res
+
+
 def chunk_small_measure(steps: int):
     """Small chunk blocks: the split decode path against the chunk kernel.
     The chunk workload's shape (Hq=16, Hkv=8, d=128, P=256, W=4096, t0=100000,
@@ -1138,7 +1195,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--only", choices=["prefill", "prompt", "ragged", "shared", "paged", "t_sweep",
-                                       "gqa", "chunk_small"],
+                                       "gqa", "chunk_small", "paged_prefill"],
                     help="run one side measurement alone and print its record (for profiling "
                          "one kernel under ncu); not a benchmark line")
     args = ap.parse_args()
@@ -1156,6 +1213,7 @@ def main():
               "t_sweep": lambda n: t_sweep_measure(max(n, 16)),
               "gqa": lambda n: gqa_measure(max(n, 16)),
               "chunk_small": lambda n: chunk_small_measure(max(n, 10)),
+              "paged_prefill": lambda n: paged_prefill_measure(max(n, 5)),
               "prompt": lambda n: prompt_measure(n, load_bf16_peak()[0])}[args.only]
         print(json.dumps({"only": args.only, "result": fn(k)}), flush=True)
     elif args.impl == "reference":

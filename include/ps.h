@@ -113,8 +113,9 @@ PS_API int ps_cache_create(int W, int P_max, int Hkv, int d, int dtype, int max_
  * the float32 summation order only), except that a write needing a page when
  * the pool is empty fails with PS_ENOMEM and changes nothing.  Requires
  * 1 <= page_rows <= W, W % page_rows == 0, num_pages >= 1; the tensor-core
- * chunk kernel needs page_rows % 128 == 0 (other page sizes use the CUDA-core
- * chunk kernel).  ps_cache_bytes_paged returns 0 for an invalid shape. */
+ * chunk kernel takes page_rows that are multiples of 128 or that divide 128
+ * and are multiples of 8 (8, 16, 32, 64); other page sizes use the CUDA-core
+ * chunk kernel.  ps_cache_bytes_paged returns 0 for an invalid shape. */
 PS_API size_t ps_cache_bytes_paged(int W, int P_max, int Hkv, int d, int dtype, int max_seqs,
                                    int page_rows, int num_pages);
 PS_API int ps_cache_create_paged(int W, int P_max, int Hkv, int d, int dtype, int max_seqs,

@@ -1,7 +1,12 @@
 // Key-tile schedule of the tensor-core chunk kernel: which 128-row key tiles
 // a query tile reads, in order (prefix rows, the ring window as at most two
-// slot runs split at the physical wrap and, for a paged cache, at page edges,
-// then the block rows).  Host-callable so that it can be checked on the CPU.
+// slot runs split at the physical wrap, then the block rows).  A ring run of
+// a paged cache with pages of 128 rows or more is also cut at page edges.
+// With smaller pages (8 to 64 rows, dividing 128) the run is tiled from the
+// page edge at or below its first slot instead, so that every tile is whole
+// pages; the rows before the run hold positions below KSched::rlo, which the
+// kernel masks by position like the window's edge.  Host-callable so that it
+// can be checked on the CPU.
 #pragma once
 #include <stdint.h>
 
@@ -17,6 +22,7 @@ constexpr int kBN = 128;  // key rows per tile
 struct KSched {
   int n;
   int ntiles;
+  int64_t rlo;      // lowest position a ring or block tile presents as a key
   int src[4];       // 0: ring slot, 1: block row, 2: prefix row (owner's slab)
   int64_t row0[4];  // first ring slot / block row / prefix row of the range
   int64_t pos0[4];  // position of that row
@@ -32,10 +38,20 @@ struct KTile {
   int valid;
 };
 
+// Pages smaller than a key tile (they divide it): ring tiles are whole pages.
+__host__ __device__ __forceinline__ bool small_pages(int64_t page) { return page > 0 && page < kBN; }
+
 // page: ring page size for a ring range of a paged cache (0: no page cuts)
 __host__ __device__ __forceinline__ void add_range(KSched& s, int src, int64_t row0, int64_t pos0,
                                           int64_t len, int64_t page = 0) {
   if (len <= 0) return;
+  if (small_pages(page)) {  // start at the page edge at or below row0 (a slot, below 2^28)
+    const int32_t lead = (int32_t)row0 % (int32_t)page;
+    row0 -= lead;
+    pos0 -= lead;
+    len += lead;
+    page = 0;
+  }
   int64_t first = len;
   if (page > 0) {  // a ring range: row0 is a slot, below 2^28
     const int64_t to_edge = page - (int32_t)row0 % (int32_t)page;
@@ -69,6 +85,7 @@ __host__ __device__ __forceinline__ KSched make_sched(const DevMeta& m, int W, i
   KSched s;
   s.n = 0;
   s.ntiles = 0;
+  s.rlo = 0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     s.src[i] = 0; s.row0[i] = 0; s.pos0[i] = 0; s.len[i] = 0;
@@ -83,6 +100,7 @@ __host__ __device__ __forceinline__ KSched make_sched(const DevMeta& m, int W, i
   if (lo < m.P) lo = m.P;
   const int64_t base = m.next_pos - m.count;
   int64_t rlo = lo < base ? base : lo;  // never below what the ring holds
+  s.rlo = rlo;  // block rows start at or above it too (base <= t0)
   if (t0 - 1 >= rlo) {
     const int64_t nw = t0 - rlo;
     int64_t s0 = (int64_t)m.head + (rlo - base);  // head < W, rlo - base < W: one wrap at most

@@ -62,6 +62,8 @@ struct ChunkArgs {
   CUtensorMap vpre;
   CUtensorMap kring;  // cache K ring pages [nphys*Hkv][page_rows][128]: box (64, 128, 1)
   CUtensorMap vring;
+  CUtensorMap kring_p;  // pages smaller than a key tile: box (64, page_rows, 1)
+  CUtensorMap vring_p;
   CUtensorMap kblk;   // k_blk [N][Hkv][128] (entries packed): box (64, 1, 128)
   CUtensorMap vblk;
   CacheDev c;
@@ -115,6 +117,8 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return r;
 }
 
+// SP: a paged cache whose pages are smaller than a key tile (8 to 64 rows)
+template <bool SP>
 __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constant__ ChunkArgs a) {
   extern __shared__ uint8_t dsm_raw[];
   TcSmem& sm = *reinterpret_cast<TcSmem*>(
@@ -151,8 +155,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
   m.owner = a.owner[eb];
   const int64_t plo = t0 + i0;
   const int64_t phi = t0 + min(i0 + PT, n) - 1;
-  const KSched ks = make_sched(m, a.c.W, a.c.page_table ? a.c.page_rows : 0, t0, plo, phi,
-                               a.prompt != 0);
+  const int spage = a.c.page_table ? a.c.page_rows : 0;  // ring page size of the schedule
+  const KSched ks = make_sched(m, a.c.W, spage, t0, plo, phi, a.prompt != 0);
   const int T = ks.ntiles;
 
   if (threadIdx.x == 0) {
@@ -181,9 +185,14 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer --
+    // Lane 0 waits for free stages and issues the copies.  With pages smaller
+    // than a tile (SP) a ring tile is kBN / spage whole pages, one box each,
+    // which the lanes map and copy one page apiece (their page-table reads
+    // run side by side); a page past the ring's end or not yet mapped gets
+    // slab -1, which the copy fills with zeros, and its rows are masked.
+    const int prefix_z = m.owner * a.c.Hkv + g;  // prefix rows live in the owner's slab
+    int issued_k = 0, issued_v = 0;
     if (lane == 0) {
-      const int prefix_z = m.owner * a.c.Hkv + g;  // prefix rows live in the owner's slab
-      int issued_k = 0, issued_v = 0;
       ptx::mbar_arrive_expect_tx(&q_full, 2 * kBM * 128);
       for (int hh = 0; hh < a.G; ++hh)
         for (int b = 0; b < 2; ++b)
@@ -196,45 +205,106 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
                          (a.prompt ? t0 + n > m.P : m.next_pos != t0);
         if (bad) atomicOr(a.c.err, ERR_BATCH);
       }
-      for (int j = 0; j < T && !abort_flag; ++j) {
+    }
+    if constexpr (!SP) {
+      if (lane == 0) {
+        for (int j = 0; j < T && !abort_flag; ++j) {
+          const int st = j & 1;
+          const KTile kt = tile_of(ks, j);
+          if (j >= 2 && !wait_bar(&k_empty[st], ((j >> 1) - 1) & 1, &abort_flag)) break;
+          // a ring tile lies within one page: (slot within the page, page's slab)
+          const int32_t kslot = (int32_t)kt.row;  // ring slot (ring tiles)
+          const int ring_z = kt.src == 0 ? ring_page(a.c, seq, kslot) * a.c.Hkv + g : 0;
+          const int32_t ring_y = kt.src == 0 ? kslot % a.c.page_rows : 0;
+          const int32_t blk_row = (int32_t)(tok0 + kt.row);  // block tiles: packed row
+          ptx::mbar_arrive_expect_tx(&k_full[st], kTileBytes);
+          for (int b = 0; b < 2; ++b) {
+            if (kt.src == 2)
+              ptx::tma_load_3d(sm.k[st][b], &a.kpre, b * 64, (int32_t)kt.row, prefix_z,
+                               &k_full[st]);
+            else if (kt.src == 0)
+              ptx::tma_load_3d(sm.k[st][b], &a.kring, b * 64, ring_y, ring_z, &k_full[st]);
+            else
+              ptx::tma_load_3d(sm.k[st][b], &a.kblk, b * 64, g, blk_row, &k_full[st]);
+          }
+          issued_k = j + 1;
+          if (j >= 2 && !wait_bar(&v_empty[st], ((j >> 1) - 1) & 1, &abort_flag)) break;
+          ptx::mbar_arrive_expect_tx(&v_full[st], kTileBytes);
+          for (int b = 0; b < 2; ++b) {
+            if (kt.src == 2)
+              ptx::tma_load_3d(sm.v[st][b], &a.vpre, b * 64, (int32_t)kt.row, prefix_z,
+                               &v_full[st]);
+            else if (kt.src == 0)
+              ptx::tma_load_3d(sm.v[st][b], &a.vring, b * 64, ring_y, ring_z, &v_full[st]);
+            else
+              ptx::tma_load_3d(sm.v[st][b], &a.vblk, b * 64, g, blk_row, &v_full[st]);
+          }
+          issued_v = j + 1;
+        }
+      }
+    } else {
+      const bool plane = lane * spage < kBN;  // this lane copies a page of a tile
+      for (int j = 0; j < T; ++j) {
         const int st = j & 1;
         const KTile kt = tile_of(ks, j);
-        if (j >= 2 && !wait_bar(&k_empty[st], ((j >> 1) - 1) & 1, &abort_flag)) break;
-        // a ring tile lies within one page: (slot within the page, page's slab)
-        const int32_t kslot = (int32_t)kt.row;  // ring slot (ring tiles)
-        const int ring_z = kt.src == 0 ? ring_page(a.c, seq, kslot) * a.c.Hkv + g : 0;
-        const int32_t ring_y = kt.src == 0 ? kslot % a.c.page_rows : 0;
+        const bool ptile = kt.src == 0;  // a ring tile: whole pages
+        const int32_t kslot = (int32_t)kt.row;  // its first slot, a page edge
+        int pz = -1;  // this lane's page of a small-page tile: its slab
+        if (ptile && plane && kslot + lane * spage < a.c.W) {
+          const int ph = ring_page(a.c, seq, kslot + lane * spage);
+          pz = ph >= 0 ? ph * a.c.Hkv + g : -1;
+        }
         const int32_t blk_row = (int32_t)(tok0 + kt.row);  // block tiles: packed row
-        ptx::mbar_arrive_expect_tx(&k_full[st], kTileBytes);
-        for (int b = 0; b < 2; ++b) {
-          if (kt.src == 2)
-            ptx::tma_load_3d(sm.k[st][b], &a.kpre, b * 64, (int32_t)kt.row, prefix_z, &k_full[st]);
-          else if (kt.src == 0)
-            ptx::tma_load_3d(sm.k[st][b], &a.kring, b * 64, ring_y, ring_z, &k_full[st]);
-          else
-            ptx::tma_load_3d(sm.k[st][b], &a.kblk, b * 64, g, blk_row, &k_full[st]);
+        // lane 0 waits; the warp follows its verdict
+        int go = 1;
+        if (lane == 0)
+          go = !abort_flag && (j < 2 || wait_bar(&k_empty[st], ((j >> 1) - 1) & 1, &abort_flag));
+        if (!__shfl_sync(0xffffffffu, go, 0)) break;
+        if (lane == 0) {
+          ptx::mbar_arrive_expect_tx(&k_full[st], kTileBytes);
+          if (!ptile)  // prefix or block rows: one box per column block
+            for (int b = 0; b < 2; ++b) {
+              if (kt.src == 2)
+                ptx::tma_load_3d(sm.k[st][b], &a.kpre, b * 64, (int32_t)kt.row, prefix_z,
+                                 &k_full[st]);
+              else
+                ptx::tma_load_3d(sm.k[st][b], &a.kblk, b * 64, g, blk_row, &k_full[st]);
+            }
+        }
+        if (ptile && plane) {
+          const int off = lane * spage * 128;
+          ptx::tma_load_3d(sm.k[st][0] + off, &a.kring_p, 0, 0, pz, &k_full[st]);
+          ptx::tma_load_3d(sm.k[st][1] + off, &a.kring_p, 64, 0, pz, &k_full[st]);
         }
         issued_k = j + 1;
-        if (j >= 2 && !wait_bar(&v_empty[st], ((j >> 1) - 1) & 1, &abort_flag)) break;
-        ptx::mbar_arrive_expect_tx(&v_full[st], kTileBytes);
-        for (int b = 0; b < 2; ++b) {
-          if (kt.src == 2)
-            ptx::tma_load_3d(sm.v[st][b], &a.vpre, b * 64, (int32_t)kt.row, prefix_z, &v_full[st]);
-          else if (kt.src == 0)
-            ptx::tma_load_3d(sm.v[st][b], &a.vring, b * 64, ring_y, ring_z, &v_full[st]);
-          else
-            ptx::tma_load_3d(sm.v[st][b], &a.vblk, b * 64, g, blk_row, &v_full[st]);
+        if (lane == 0) go = j < 2 || wait_bar(&v_empty[st], ((j >> 1) - 1) & 1, &abort_flag);
+        if (!__shfl_sync(0xffffffffu, go, 0)) break;
+        if (lane == 0) {
+          ptx::mbar_arrive_expect_tx(&v_full[st], kTileBytes);
+          if (!ptile)  // prefix or block rows: one box per column block
+            for (int b = 0; b < 2; ++b) {
+              if (kt.src == 2)
+                ptx::tma_load_3d(sm.v[st][b], &a.vpre, b * 64, (int32_t)kt.row, prefix_z,
+                                 &v_full[st]);
+              else
+                ptx::tma_load_3d(sm.v[st][b], &a.vblk, b * 64, g, blk_row, &v_full[st]);
+            }
+        }
+        if (ptile && plane) {
+          const int off = lane * spage * 128;
+          ptx::tma_load_3d(sm.v[st][0] + off, &a.vring_p, 0, 0, pz, &v_full[st]);
+          ptx::tma_load_3d(sm.v[st][1] + off, &a.vring_p, 64, 0, pz, &v_full[st]);
         }
         issued_v = j + 1;
       }
-      if (abort_flag) {  // let the copies already issued land before the CTA exits
-        int quiet = 0;
-        ptx::mbar_wait_bounded(&q_full, 0, &quiet, kWaitLimit);
-        for (int j = issued_k > 2 ? issued_k - 2 : 0; j < issued_k; ++j)
-          ptx::mbar_wait_bounded(&k_full[j & 1], (j >> 1) & 1, &quiet, kWaitLimit);
-        for (int j = issued_v > 2 ? issued_v - 2 : 0; j < issued_v; ++j)
-          ptx::mbar_wait_bounded(&v_full[j & 1], (j >> 1) & 1, &quiet, kWaitLimit);
-      }
+    }
+    if (lane == 0 && abort_flag) {  // let the copies already issued land before the CTA exits
+      int quiet = 0;
+      ptx::mbar_wait_bounded(&q_full, 0, &quiet, kWaitLimit);
+      for (int j = issued_k > 2 ? issued_k - 2 : 0; j < issued_k; ++j)
+        ptx::mbar_wait_bounded(&k_full[j & 1], (j >> 1) & 1, &quiet, kWaitLimit);
+      for (int j = issued_v > 2 ? issued_v - 2 : 0; j < issued_v; ++j)
+        ptx::mbar_wait_bounded(&v_full[j & 1], (j >> 1) & 1, &quiet, kWaitLimit);
     }
     __syncwarp();  // the whole warp meets the final block barrier together
   } else if (warp == 1) {
@@ -293,6 +363,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
     const int cbase = half * 64;          // first S/O column of this thread
     // A prompt query t sees [0, t]: the mask below with the prefix taken as [0, t].
     const int W = a.c.W, P = a.prompt ? (int)(tq + 1) : m.P;
+    // lowest ring or block key of this query / of any query of the tile: the
+    // window's start, or the schedule's rlo where that is higher (the first
+    // ring tile over pages smaller than a tile starts at a page edge below it)
+    const int64_t qlo = max(tq - W + 1, ks.rlo);
+    const int64_t tlo = max(phi - W + 1, ks.rlo);
     const float sc = a.sc;
     const int pair_bar = 2 + quad;        // named barrier of the two warps of this quadrant
     auto pair_sync = [&]() { asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory"); };
@@ -321,11 +396,12 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
         const bool full = kt.valid == kBN &&
                           (kt.src == 2 && kt.pos0 + kBN <= P
                                ? true
-                               : (kt.pos0 >= phi - W + 1 && kt.pos0 + kBN - 1 <= plo));
+                               : (kt.pos0 >= tlo && kt.pos0 + kBN - 1 <= plo));
         if (!full) {
           auto clampc = [](int64_t v) -> int { return v < -1 ? -1 : (v > kBN ? kBN : (int)v); };
-          const int pre_c = clampc(P - kt.pos0) - cbase;          // c < pre_c: pinned prefix
-          const int lo_c = clampc(tq - W + 1 - kt.pos0) - cbase;  // window start
+          // c < pre_c: pinned prefix (prefix tiles only)
+          const int pre_c = kt.src == 2 ? clampc(P - kt.pos0) - cbase : 0;
+          const int lo_c = clampc(qlo - kt.pos0) - cbase;  // window start
           const int hi_c = clampc(tq - kt.pos0) - cbase;          // causal end
           const int vc = kt.valid - cbase;
 #pragma unroll
@@ -446,8 +522,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
 }  // namespace
 
 bool chunk_tc_supported(const CacheDev& c, int dtype, int d, int G) {
-  // ring tiles of a paged cache must not straddle pages: 128-row multiples
-  const bool pages_ok = !c.page_table || c.page_rows % kBN == 0;
+  // ring tiles of a paged cache: pages of 128-row multiples, or whole pages of
+  // 8 to 64 rows that divide the tile
+  const bool pages_ok = !c.page_table || c.page_rows % kBN == 0 ||
+                        (kBN % c.page_rows == 0 && c.page_rows % 8 == 0);
   return pages_ok && dtype == 1 && d == kHD && (G == 1 || G == 2 || G == 4 || G == 8);
 }
 
@@ -489,6 +567,14 @@ cudaError_t launch_chunk_tc(const CacheDev& c, int G, const ChunkEntry* e, int n
                    (uint64_t)c.rstride * row, 64, kBN, 1);
   ok = ok && encode_map3d_bf16(&a.vring, vring, kHD, (uint64_t)c.page_rows, (uint64_t)c.nphys * c.Hkv, row,
                    (uint64_t)c.rstride * row, 64, kBN, 1);
+  if (c.page_table && small_pages(c.page_rows)) {  // whole-page boxes
+    ok = ok && encode_map3d_bf16(&a.kring_p, kring, kHD, (uint64_t)c.page_rows,
+                                 (uint64_t)c.nphys * c.Hkv, row, (uint64_t)c.rstride * row, 64,
+                                 (uint32_t)c.page_rows, 1);
+    ok = ok && encode_map3d_bf16(&a.vring_p, vring, kHD, (uint64_t)c.page_rows,
+                                 (uint64_t)c.nphys * c.Hkv, row, (uint64_t)c.rstride * row, 64,
+                                 (uint32_t)c.page_rows, 1);
+  }
   // a prompt launch loads no block rows; its block maps describe the cache
   // K/V (never used) so that every map is well formed
   const uint64_t nblk = prompt ? prows : (uint64_t)N;
@@ -511,12 +597,19 @@ cudaError_t launch_chunk_tc(const CacheDev& c, int G, const ChunkEntry* e, int n
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (!(configured.load() & (1ull << (dev & 63)))) {
-    err = cudaFuncSetAttribute(k_chunk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
+    err = cudaFuncSetAttribute(k_chunk_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)dyn);
+    if (err == cudaSuccess)
+      err = cudaFuncSetAttribute(k_chunk_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)dyn);
     if (err != cudaSuccess) return err;
     configured.fetch_or(1ull << (dev & 63));
   }
   dim3 grid(a.qtc[nb], c.Hkv);
-  k_chunk_tc<<<grid, kThreadsTC, dyn, st>>>(a);
+  if (c.page_table && small_pages(c.page_rows))
+    k_chunk_tc<true><<<grid, kThreadsTC, dyn, st>>>(a);
+  else
+    k_chunk_tc<false><<<grid, kThreadsTC, dyn, st>>>(a);
   return cudaGetLastError();
 }
 

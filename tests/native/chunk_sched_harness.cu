@@ -1,7 +1,8 @@
 // Host-side harness for the tensor-core chunk kernel's key-tile schedule
 // (prefix_sliding_window_ring_b200/csrc/chunk_sched.cuh), compiled by the CPU
 // tests and run without a GPU.  For each case read from stdin it prints the
-// key tiles a query tile reads: source, first row, first position, rows.
+// lowest ring or block key position (rlo) and the key tiles a query tile
+// reads: source, first row, first position, rows.
 //
 // Input lines:  P W head count next_pos t0 plo phi prompt page
 #include <stdio.h>
@@ -21,7 +22,7 @@ int main() {
     m.head = head;
     m.count = count;
     const ps::KSched s = ps::make_sched(m, W, page, t0, plo, phi, prompt != 0);
-    printf("%d", s.ntiles);
+    printf("%d %lld", s.ntiles, (long long)s.rlo);
     for (int j = 0; j < s.ntiles; ++j) {
       const ps::KTile t = ps::tile_of(s, j);
       printf(" %d,%lld,%lld,%d", t.src, (long long)t.row, (long long)t.pos0, t.valid);

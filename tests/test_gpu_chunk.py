@@ -24,12 +24,14 @@ def chunk_history(P, W, t0, n, i_rows):
 
 
 def run_chunk(W, P, L, n, dtype, d, G, Hkv=2, seed=0, rows=None, seqs=1, h0=0, append=True,
-              batched=False):
+              batched=False, page=0):
     """batched: all sequences' blocks in one ps_attend_chunk_batch call (the
-    launch the benchmark times); otherwise one ps_attend_chunk call each."""
+    launch the benchmark times); otherwise one ps_attend_chunk call each.
+    page > 0: a paged ring of page-row pages."""
     Hq = G * Hkv
     scale = default_scale(d)
-    c = Cache(W, max(P, 1), Hkv, d, ps_dtype(dtype), seqs)
+    kw = dict(page_rows=page, num_pages=seqs * (W // page)) if page else {}
+    c = Cache(W, max(P, 1), Hkv, d, ps_dtype(dtype), seqs, **kw)
     t0 = P + L
     sds = [SeqData(seed, s, Hq, Hkv, d, dtype) for s in range(seqs)]
     outs, qs, kbs, vbs = [], [], [], []
@@ -129,3 +131,23 @@ def test_chunk_full_size(W):
                       set(rng.integers(0, n, 6).tolist()))
     run_chunk(W, s.P, t0 - s.P, n, s.dtype, s.d, s.G, Hkv=s.Hkv, rows=rows, seqs=cfg["B"],
               h0=1234, append=True, batched=True)
+
+
+@pytest.mark.parametrize("page", [8, 16, 32, 64])
+def test_chunk_small_pages(page):
+    """Paged rings whose pages are smaller than a 128-row key tile: the
+    tensor-core kernel reads each ring tile as whole pages from a page edge
+    (window full and wrapping, then window filling inside the block)."""
+    run_chunk(512, 40, 700, 300, "bf16", 128, 2, h0=37, seqs=2, page=page, batched=True)
+    run_chunk(256, 24, 100, 200, "bf16", 128, 4, h0=5, page=page)
+
+
+def test_chunk_full_size_16_row_pages():
+    """The chunk workload (4 sequences x 2048 queries at t0=100000, W=4096) on
+    a ring of 16-row pages, sampled rows of every query-tile edge class."""
+    cfg = workloads.CHUNK
+    s = cfg["shape_for"](4096)
+    n, t0 = cfg["n"], cfg["t0"]
+    rows = [0, 1, 63, 64, 127, 128, 129, 1023, 1024, n - 2, n - 1]
+    run_chunk(4096, s.P, t0 - s.P, n, s.dtype, s.d, s.G, Hkv=s.Hkv, rows=rows, seqs=cfg["B"],
+              h0=1234, append=True, batched=True, page=16)
