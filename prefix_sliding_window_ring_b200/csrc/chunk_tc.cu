@@ -104,6 +104,37 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// 2^y for two values on the FMA pipe, so that part of a tile's exponentials
+// leaves the special-function unit.  Cody and Waite's reduction: 2^y =
+// 2^floor(y) * 2^f with f = y - floor(y) in [0, 1), and 2^f from a cubic
+// 1 + c1 f + c2 f^2 + c3 f^3 whose coefficients were fitted here by
+// least squares on relative error over [0, 1) (largest relative error
+// 2.7e-4, well below the rounding of the bf16 P it feeds).  floor(y) comes
+// from adding 1.5 * 2^23 rounded down, which leaves it in the low bits of the
+// sum; shifting those bits by 23 adds it to the exponent field of the cubic's
+// value.  y is clamped at -127: there f = 0, the cubic is exactly 1, and the
+// exponent field drops to zero, so y <= -127 (a masked -inf included) gives
+// +0 exactly; the scaled scores never exceed 2^8 (the lazy maximum).
+constexpr float kExpC1 = 0.6951161f, kExpC2 = 0.22877206f, kExpC3 = 0.0755871f;
+__device__ __forceinline__ float2 exp2_fma2(float2 y) {
+  constexpr float kMagic = 12582912.f;  // 1.5 * 2^23
+  y.x = fmaxf(y.x, -127.f);
+  y.y = fmaxf(y.y, -127.f);
+  const float2 t = __fadd2_rd(y, make_float2(kMagic, kMagic));  // 1.5 * 2^23 + floor(y)
+  const float2 fl = __fadd2_rn(t, make_float2(-kMagic, -kMagic));  // floor(y), exact
+  const float2 f = __ffma2_rn(fl, make_float2(-1.f, -1.f), y);     // y - floor(y), exact
+  float2 q = __ffma2_rn(make_float2(kExpC3, kExpC3), f, make_float2(kExpC2, kExpC2));
+  q = __ffma2_rn(q, f, make_float2(kExpC1, kExpC1));
+  q = __ffma2_rn(q, f, make_float2(1.f, 1.f));
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+}
+#ifndef PS_CHUNK_EXP_FMA_EVERY
+#define PS_CHUNK_EXP_FMA_EVERY 8
+#endif
+// one column pair in kExpFmaEvery takes its exponentials on the FMA pipe (0: none)
+constexpr int kExpFmaEvery = PS_CHUNK_EXP_FMA_EVERY;
+
 // max of three (max.f32 with three sources, sm_100)
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
@@ -463,7 +494,16 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
 #pragma unroll
       for (int c = 0; c < 64; c += 2) {
         const float2 y = __ffma2_rn(make_float2(x[c], x[c + 1]), sc2, nmu2);
-        const float p0 = ex2(y.x), p1 = ex2(y.y);
+        float p0, p1;
+        if (kExpFmaEvery > 0 && (c >> 1) % (kExpFmaEvery > 0 ? kExpFmaEvery : 1) ==
+                                    kExpFmaEvery - 1) {
+          const float2 e = exp2_fma2(y);
+          p0 = e.x;
+          p1 = e.y;
+        } else {
+          p0 = ex2(y.x);
+          p1 = ex2(y.y);
+        }
         s4[(c >> 1) & 3] = __fadd2_rn(s4[(c >> 1) & 3], make_float2(p0, p1));
         pk[c >> 1] = pack_bf16(p0, p1);
       }
