@@ -214,16 +214,18 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
   ptx::tc_fence_after();
   const uint32_t tmem = tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer --
+  if (warp == 0 || (SP && warp == 3)) {
+    // ----------------------------------------------------------- producers --
     // Lane 0 waits for free stages and issues the copies.  With pages smaller
     // than a tile (SP) a ring tile is kBN / spage whole pages, one box each,
     // which the lanes map and copy one page apiece (their page-table reads
     // run side by side); a page past the ring's end or not yet mapped gets
     // slab -1, which the copy fills with zeros, and its rows are masked.
+    // There warp 0 copies the K tiles and warp 3 the V tiles, so that the
+    // tile's page copies are issued by two warps at once.
     const int prefix_z = m.owner * a.c.Hkv + g;  // prefix rows live in the owner's slab
     int issued_k = 0, issued_v = 0;
-    if (lane == 0) {
+    if (lane == 0 && warp == 0) {
       ptx::mbar_arrive_expect_tx(&q_full, 2 * kBM * 128);
       for (int hh = 0; hh < a.G; ++hh)
         for (int b = 0; b < 2; ++b)
@@ -274,6 +276,15 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
         }
       }
     } else {
+      const bool isv = warp == 3;  // this warp's operand
+      const CUtensorMap* mpre = isv ? &a.vpre : &a.kpre;
+      const CUtensorMap* mblk = isv ? &a.vblk : &a.kblk;
+      const CUtensorMap* mring_p = isv ? &a.vring_p : &a.kring_p;
+      uint64_t* full = isv ? v_full : k_full;
+      uint64_t* empty = isv ? v_empty : k_empty;
+      uint8_t* const buf = isv ? &sm.v[0][0][0] : &sm.k[0][0][0];
+      constexpr int kColBlk = kBN * 128;  // bytes of one 64-column block of a tile
+      int issued = 0;
       const bool plane = lane * spage < kBN;  // this lane copies a page of a tile
       for (int j = 0; j < T; ++j) {
         const int st = j & 1;
@@ -289,45 +300,27 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
         // lane 0 waits; the warp follows its verdict
         int go = 1;
         if (lane == 0)
-          go = !abort_flag && (j < 2 || wait_bar(&k_empty[st], ((j >> 1) - 1) & 1, &abort_flag));
+          go = !abort_flag && (j < 2 || wait_bar(&empty[st], ((j >> 1) - 1) & 1, &abort_flag));
         if (!__shfl_sync(0xffffffffu, go, 0)) break;
         if (lane == 0) {
-          ptx::mbar_arrive_expect_tx(&k_full[st], kTileBytes);
+          ptx::mbar_arrive_expect_tx(&full[st], kTileBytes);
           if (!ptile)  // prefix or block rows: one box per column block
             for (int b = 0; b < 2; ++b) {
+              uint8_t* dst = buf + (st * 2 + b) * kColBlk;
               if (kt.src == 2)
-                ptx::tma_load_3d(sm.k[st][b], &a.kpre, b * 64, (int32_t)kt.row, prefix_z,
-                                 &k_full[st]);
+                ptx::tma_load_3d(dst, mpre, b * 64, (int32_t)kt.row, prefix_z, &full[st]);
               else
-                ptx::tma_load_3d(sm.k[st][b], &a.kblk, b * 64, g, blk_row, &k_full[st]);
+                ptx::tma_load_3d(dst, mblk, b * 64, g, blk_row, &full[st]);
             }
         }
         if (ptile && plane) {
-          const int off = lane * spage * 128;
-          ptx::tma_load_3d(sm.k[st][0] + off, &a.kring_p, 0, 0, pz, &k_full[st]);
-          ptx::tma_load_3d(sm.k[st][1] + off, &a.kring_p, 64, 0, pz, &k_full[st]);
+          uint8_t* dst = buf + st * 2 * kColBlk + lane * spage * 128;
+          ptx::tma_load_3d(dst, mring_p, 0, 0, pz, &full[st]);
+          ptx::tma_load_3d(dst + kColBlk, mring_p, 64, 0, pz, &full[st]);
         }
-        issued_k = j + 1;
-        if (lane == 0) go = j < 2 || wait_bar(&v_empty[st], ((j >> 1) - 1) & 1, &abort_flag);
-        if (!__shfl_sync(0xffffffffu, go, 0)) break;
-        if (lane == 0) {
-          ptx::mbar_arrive_expect_tx(&v_full[st], kTileBytes);
-          if (!ptile)  // prefix or block rows: one box per column block
-            for (int b = 0; b < 2; ++b) {
-              if (kt.src == 2)
-                ptx::tma_load_3d(sm.v[st][b], &a.vpre, b * 64, (int32_t)kt.row, prefix_z,
-                                 &v_full[st]);
-              else
-                ptx::tma_load_3d(sm.v[st][b], &a.vblk, b * 64, g, blk_row, &v_full[st]);
-            }
-        }
-        if (ptile && plane) {
-          const int off = lane * spage * 128;
-          ptx::tma_load_3d(sm.v[st][0] + off, &a.vring_p, 0, 0, pz, &v_full[st]);
-          ptx::tma_load_3d(sm.v[st][1] + off, &a.vring_p, 64, 0, pz, &v_full[st]);
-        }
-        issued_v = j + 1;
+        issued = j + 1;
       }
+      if (isv) issued_v = issued; else issued_k = issued;
     }
     if (lane == 0 && abort_flag) {  // let the copies already issued land before the CTA exits
       int quiet = 0;
