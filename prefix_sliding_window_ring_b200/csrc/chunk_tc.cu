@@ -214,15 +214,16 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
   ptx::tc_fence_after();
   const uint32_t tmem = tmem_slot;
 
-  if (warp == 0 || (SP && warp == 3)) {
+  if (warp == 0 || warp == 3) {
     // ----------------------------------------------------------- producers --
     // Lane 0 waits for free stages and issues the copies.  With pages smaller
     // than a tile (SP) a ring tile is kBN / spage whole pages, one box each,
     // which the lanes map and copy one page apiece (their page-table reads
     // run side by side); a page past the ring's end or not yet mapped gets
     // slab -1, which the copy fills with zeros, and its rows are masked.
-    // There warp 0 copies the K tiles and warp 3 the V tiles, so that the
-    // tile's page copies are issued by two warps at once.
+    // Warp 0 copies the K tiles and warp 3 the V tiles, each into its own
+    // 2-stage ring, so that a K tile never waits behind a V tile's free
+    // stage (and a tile's page copies are issued by two warps at once).
     const int prefix_z = m.owner * a.c.Hkv + g;  // prefix rows live in the owner's slab
     int issued_k = 0, issued_v = 0;
     if (lane == 0 && warp == 0) {
@@ -239,52 +240,41 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
         if (bad) atomicOr(a.c.err, ERR_BATCH);
       }
     }
+    const bool isv = warp == 3;  // this warp's operand
+    const CUtensorMap* mpre = isv ? &a.vpre : &a.kpre;
+    const CUtensorMap* mblk = isv ? &a.vblk : &a.kblk;
+    uint64_t* full = isv ? v_full : k_full;
+    uint64_t* empty = isv ? v_empty : k_empty;
+    uint8_t* const buf = isv ? &sm.v[0][0][0] : &sm.k[0][0][0];
+    constexpr int kColBlk = kBN * 128;  // bytes of one 64-column block of a tile
+    int issued = 0;
     if constexpr (!SP) {
+      const CUtensorMap* mring = isv ? &a.vring : &a.kring;
       if (lane == 0) {
         for (int j = 0; j < T && !abort_flag; ++j) {
           const int st = j & 1;
           const KTile kt = tile_of(ks, j);
-          if (j >= 2 && !wait_bar(&k_empty[st], ((j >> 1) - 1) & 1, &abort_flag)) break;
+          if (j >= 2 && !wait_bar(&empty[st], ((j >> 1) - 1) & 1, &abort_flag)) break;
           // a ring tile lies within one page: (slot within the page, page's slab)
           const int32_t kslot = (int32_t)kt.row;  // ring slot (ring tiles)
           const int ring_z = kt.src == 0 ? ring_page(a.c, seq, kslot) * a.c.Hkv + g : 0;
           const int32_t ring_y = kt.src == 0 ? kslot % a.c.page_rows : 0;
           const int32_t blk_row = (int32_t)(tok0 + kt.row);  // block tiles: packed row
-          ptx::mbar_arrive_expect_tx(&k_full[st], kTileBytes);
+          ptx::mbar_arrive_expect_tx(&full[st], kTileBytes);
           for (int b = 0; b < 2; ++b) {
+            uint8_t* dst = buf + (st * 2 + b) * kColBlk;
             if (kt.src == 2)
-              ptx::tma_load_3d(sm.k[st][b], &a.kpre, b * 64, (int32_t)kt.row, prefix_z,
-                               &k_full[st]);
+              ptx::tma_load_3d(dst, mpre, b * 64, (int32_t)kt.row, prefix_z, &full[st]);
             else if (kt.src == 0)
-              ptx::tma_load_3d(sm.k[st][b], &a.kring, b * 64, ring_y, ring_z, &k_full[st]);
+              ptx::tma_load_3d(dst, mring, b * 64, ring_y, ring_z, &full[st]);
             else
-              ptx::tma_load_3d(sm.k[st][b], &a.kblk, b * 64, g, blk_row, &k_full[st]);
+              ptx::tma_load_3d(dst, mblk, b * 64, g, blk_row, &full[st]);
           }
-          issued_k = j + 1;
-          if (j >= 2 && !wait_bar(&v_empty[st], ((j >> 1) - 1) & 1, &abort_flag)) break;
-          ptx::mbar_arrive_expect_tx(&v_full[st], kTileBytes);
-          for (int b = 0; b < 2; ++b) {
-            if (kt.src == 2)
-              ptx::tma_load_3d(sm.v[st][b], &a.vpre, b * 64, (int32_t)kt.row, prefix_z,
-                               &v_full[st]);
-            else if (kt.src == 0)
-              ptx::tma_load_3d(sm.v[st][b], &a.vring, b * 64, ring_y, ring_z, &v_full[st]);
-            else
-              ptx::tma_load_3d(sm.v[st][b], &a.vblk, b * 64, g, blk_row, &v_full[st]);
-          }
-          issued_v = j + 1;
+          issued = j + 1;
         }
       }
     } else {
-      const bool isv = warp == 3;  // this warp's operand
-      const CUtensorMap* mpre = isv ? &a.vpre : &a.kpre;
-      const CUtensorMap* mblk = isv ? &a.vblk : &a.kblk;
       const CUtensorMap* mring_p = isv ? &a.vring_p : &a.kring_p;
-      uint64_t* full = isv ? v_full : k_full;
-      uint64_t* empty = isv ? v_empty : k_empty;
-      uint8_t* const buf = isv ? &sm.v[0][0][0] : &sm.k[0][0][0];
-      constexpr int kColBlk = kBN * 128;  // bytes of one 64-column block of a tile
-      int issued = 0;
       const bool plane = lane * spage < kBN;  // this lane copies a page of a tile
       for (int j = 0; j < T; ++j) {
         const int st = j & 1;
@@ -320,8 +310,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
         }
         issued = j + 1;
       }
-      if (isv) issued_v = issued; else issued_k = issued;
     }
+    if (isv) issued_v = issued; else issued_k = issued;
     if (lane == 0 && abort_flag) {  // let the copies already issued land before the CTA exits
       int quiet = 0;
       ptx::mbar_wait_bounded(&q_full, 0, &quiet, kWaitLimit);
