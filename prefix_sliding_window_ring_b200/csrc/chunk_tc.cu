@@ -18,8 +18,9 @@
 // or causal edge are masked element by element.
 //
 // Roles (12 warps):
-//   warp 0   TMA producer: Q once, then K and V tiles into 2-stage rings
+//   warp 0   TMA producer: Q once, then the K tiles into a 2-stage ring
 //            (tensor-map tiled loads with 128-byte swizzle, no multicast);
+//   warp 3   TMA producer of the V tiles (its own 2-stage ring);
 //   warp 1   MMA issuer: S_j = Q K_j^T into one of two TMEM buffers, then
 //            O += P_j V_j with P_j read from TMEM (kind::f16, f32 accumulate);
 //   warp 2   owns the TMEM allocation (S in two 128-column buffers, O);
@@ -28,7 +29,8 @@
 //            and sums through shared memory.  They load S_j from TMEM, mask,
 //            keep a running max (raised lazily, rescaling O in TMEM only when
 //            it grows by more than 2^8), write P_j (bf16) back over S_j and
-//            finally normalise O into the output.
+//            finally normalise O into the output.  One column pair in eight
+//            takes its exponentials on the FMA pipe (exp2_fma2).
 // Every wait is bounded: a time-out sets ERR_TIMEOUT, every role stops, the
 // MMA issuer waits for its issued work and the TMEM is freed.
 #include <math.h>
