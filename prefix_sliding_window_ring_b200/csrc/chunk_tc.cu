@@ -289,7 +289,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1) k_chunk_tc(const __grid_constan
           pz = ph >= 0 ? ph * a.c.Hkv + g : -1;
         }
         const int32_t blk_row = (int32_t)(tok0 + kt.row);  // block tiles: packed row
-        // lane 0 waits; the warp follows its verdict
+        // lane 0 waits; the warp follows its decision
         int go = 1;
         if (lane == 0)
           go = !abort_flag && (j < 2 || wait_bar(&empty[st], ((j >> 1) - 1) & 1, &abort_flag));
