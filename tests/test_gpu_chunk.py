@@ -142,6 +142,15 @@ def test_chunk_small_pages(page):
     run_chunk(256, 24, 100, 200, "bf16", 128, 4, h0=5, page=page)
 
 
+@pytest.mark.parametrize("W,page", [(200, 8), (344, 8), (208, 16), (320, 64), (448, 64)])
+def test_chunk_small_pages_ragged_ring(W, page):
+    """A ring that is not a whole number of 128-row key tiles: the last ring
+    tile of a run ends inside a tile, and its pages past the ring's end are
+    copied as zeros and masked (window full and wrapping; window filling)."""
+    run_chunk(W, 16, 3 * W + 11, 150, "bf16", 128, 2, h0=W // 3, seqs=2, page=page, batched=True)
+    run_chunk(W, 40, W // 2, 90, "bf16", 128, 1, h0=7, page=page)
+
+
 def test_chunk_full_size_16_row_pages():
     """The chunk workload (4 sequences x 2048 queries at t0=100000, W=4096) on
     a ring of 16-row pages, sampled rows of every query-tile edge class."""
