@@ -199,8 +199,9 @@ struct MmaState {
 // its columns are the group's queries x gq heads; always with CL).
 // CL: cluster mode.  Pair p is streamed by the csize CTAs of cluster p, CTA
 // rank r taking an equal share of its padded rows (dec_cluster_share).  Each
-// CTA then pushes its merged state into its peers' shared memory (remote
-// stores: its (max, sum) per column to all, its accumulator values of output
+// CTA then pushes its merged state into its peers' shared memory
+// (asynchronous remote stores that count their bytes on the receiver's
+// barrier: its (max, sum) per column to all, its accumulator values of output
 // slice r to rank r), waits for theirs and combines its own slice of the
 // pair's output from local shared memory -- no partials in global memory, no
 // second grid, no CTA reading another's memory.  The sequence's record is
@@ -225,7 +226,7 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
   uint8_t* const vbuf = kbuf + kStagesM * kTileBytes;
   uint8_t* const qbuf = vbuf + kStagesM * kTileBytes;  // [kStagesM][G][D] bf16
   __shared__ __align__(8) uint64_t full[kStagesM], empty[kStagesM];
-  __shared__ __align__(8) uint64_t sync_a, sync_b, sync_c, sync_m, sync_w;
+  __shared__ __align__(8) uint64_t sync_a, sync_b, sync_c, sync_m;
   __shared__ __align__(8) uint64_t pub_bar;  // cluster: the peers' states have arrived
   __shared__ TileDescM desc[kStagesM];
   __shared__ int abort_flag;
@@ -242,7 +243,7 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
   // column, and its accumulator values of the output slice this CTA combines
   // (slice r of the G*D outputs belongs to rank r)
   __shared__ float rcv_ml[kMaxCluster][G][2];
-  __shared__ float rcv_o[G * D];
+  __shared__ __align__(16) float rcv_o[G * D];
   __shared__ float cw[kMaxCluster][G];  // each rank's combine weight per column
   // paged cache: the page-table row of the piece's sequence (read by the producer only)
   __shared__ __align__(16) int32_t tbl[kProd][kTblMax + 4];  // one per producer
@@ -281,11 +282,16 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
     ptx::mbar_init(&sync_b, kMW);
     ptx::mbar_init(&sync_c, kMW);
     ptx::mbar_init(&sync_m, kMW);
-    ptx::mbar_init(&sync_w, kMW);
-    ptx::mbar_init(&pub_bar, CL ? a.csize - 1 : 1);
+    ptx::mbar_init(&pub_bar, 1);
     for (int p = 0; p < kProd; ++p) ptx::mbar_init(&tbl_bar[p], 1);
     abort_flag = 0;
     ptx::fence_mbar_init();
+    // cluster: the peers' states arrive as asynchronous stores that count
+    // their bytes on pub_bar -- from each of the csize - 1 peers its slice of
+    // G * D / csize values and its (max, sum) per column
+    if (CL)
+      ptx::mbar_arrive_expect_tx(
+          &pub_bar, (uint32_t)((a.csize - 1) * (G * D / a.csize + 2 * G) * sizeof(float)));
   }
   if (warp == kMW && lane == 0) {
     // fetch the tensor maps' descriptors while the previous grid drains
@@ -854,28 +860,25 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
     const int rank = (int)ptx::cluster_ctarank(), C = a.csize;
     const int SL = G * D / C;  // outputs per slice
     if (!stopped) {
-      // push: every peer gets this CTA's (max, sum) and the values of its slice
-      for (int idx = threadIdx.x; idx < G * D; idx += kMW * 32) {
+      // push: every peer gets this CTA's (max, sum) and the values of its
+      // slice, as asynchronous stores that complete their bytes on the peer's
+      // pub_bar (no fence, no separate arrival).  D and SL are multiples of
+      // 4, so four consecutive values stay inside one row and one slice and go
+      // in one store.
+      for (int idx = 4 * threadIdx.x; idx < G * D; idx += 4 * kMW * 32) {
         const int r = idx / SL;
         if (r != rank) {
           const int h = idx / D, e = idx % D;
-          ptx::st_cluster_f32(ptx::map_to_rank(&rcv_o[rank * SL + (idx - r * SL)], r),
-                              sm.o[0][h][e]);
+          ptx::st_async_v4_f32(ptx::map_to_rank(&rcv_o[rank * SL + (idx - r * SL)], r),
+                               sm.o[0][h][e], sm.o[0][h][e + 1], sm.o[0][h][e + 2],
+                               sm.o[0][h][e + 3], ptx::map_to_rank(&pub_bar, r));
         }
       }
       for (int idx = threadIdx.x; idx < C * G * 2; idx += kMW * 32) {
         const int r = idx / (G * 2), h = (idx / 2) % G, w = idx & 1;
-        if (r != rank) ptx::st_cluster_f32(ptx::map_to_rank(&rcv_ml[rank][h][w], r), pub_ml[h][w]);
-      }
-      // every thread's stores before the arrivals (cumulative release by thread 0)
-      if (csync(&sync_w, 0)) {
-        if (threadIdx.x == 0) {
-          ptx::fence_acq_rel_cluster();
-          for (int r = 0; r < C; ++r)
-            if (r != rank) ptx::mbar_arrive_cluster(ptx::map_to_rank(&pub_bar, r));
-        }
-      } else {
-        stopped = true;
+        if (r != rank)
+          ptx::st_async_f32(ptx::map_to_rank(&rcv_ml[rank][h][w], r), pub_ml[h][w],
+                            ptx::map_to_rank(&pub_bar, r));
       }
     }
     if (!stopped) {
