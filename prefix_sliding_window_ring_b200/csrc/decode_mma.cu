@@ -226,7 +226,7 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
   uint8_t* const vbuf = kbuf + kStagesM * kTileBytes;
   uint8_t* const qbuf = vbuf + kStagesM * kTileBytes;  // [kStagesM][G][D] bf16
   __shared__ __align__(8) uint64_t full[kStagesM], empty[kStagesM];
-  __shared__ __align__(8) uint64_t sync_a, sync_b, sync_c, sync_m;
+  __shared__ __align__(8) uint64_t sync_a, sync_b, sync_m;
   __shared__ __align__(8) uint64_t pub_bar;  // cluster: the peers' states have arrived
   __shared__ TileDescM desc[kStagesM];
   __shared__ int abort_flag;
@@ -244,7 +244,6 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
   // (slice r of the G*D outputs belongs to rank r)
   __shared__ float rcv_ml[kMaxCluster][G][2];
   __shared__ __align__(16) float rcv_o[G * D];
-  __shared__ float cw[kMaxCluster][G];  // each rank's combine weight per column
   // paged cache: the page-table row of the piece's sequence (read by the producer only)
   __shared__ __align__(16) int32_t tbl[kProd][kTblMax + 4];  // one per producer
   __shared__ __align__(8) uint64_t tbl_bar[kProd];
@@ -280,7 +279,6 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
     }
     ptx::mbar_init(&sync_a, kMW);
     ptx::mbar_init(&sync_b, kMW);
-    ptx::mbar_init(&sync_c, kMW);
     ptx::mbar_init(&sync_m, kMW);
     ptx::mbar_init(&pub_bar, 1);
     for (int p = 0; p < kProd; ++p) ptx::mbar_init(&tbl_bar[p], 1);
@@ -672,6 +670,35 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
   const float qs = a.qscale;
   MmaState<D, G> st;
   int np = 0;
+  // cluster mode: this CTA's rank, the cluster size and the outputs per slice
+  // (slice r of the G * D outputs belongs to rank r)
+  const int rank = CL ? (int)ptx::cluster_ctarank() : 0, C = CL ? a.csize : 1;
+  const int SL = G * D / C;
+  // cluster mode: hand four merged values of outputs idx..idx+3 (one row,
+  // one slice: D and SL are multiples of 4) to the slice's owner -- kept here
+  // for this CTA's slice, else an asynchronous store that counts its bytes on
+  // the owner's pub_bar -- and, from the thread holding a row's first values,
+  // the row's (max, sum) to every peer.  No fence, no separate arrival.
+  auto publish = [&](int idx, const float (&v)[4], float mx, float l) {
+    const int r = idx / SL, h = idx / D, e = idx % D;
+    if (r == rank) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) sm.o[0][h][e + q] = v[q];
+    } else {
+      ptx::st_async_v4_f32(ptx::map_to_rank(&rcv_o[rank * SL + (idx - r * SL)], r), v[0], v[1],
+                           v[2], v[3], ptx::map_to_rank(&pub_bar, r));
+    }
+    if (e == 0) {
+      pub_ml[h][0] = mx;
+      pub_ml[h][1] = l;
+      for (int r2 = 0; r2 < C; ++r2) {
+        if (r2 == rank) continue;
+        const uint32_t bar = ptx::map_to_rank(&pub_bar, r2);
+        ptx::st_async_f32(ptx::map_to_rank(&rcv_ml[rank][h][0], r2), mx, bar);
+        ptx::st_async_f32(ptx::map_to_rank(&rcv_ml[rank][h][1], r2), l, bar);
+      }
+    }
+  };
   bool stopped = false;
   for (int i = 0;; ++i) {
     const int stg = i % kStagesM;
@@ -820,22 +847,37 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
     const int64_t slot = d.slot;
     float* pml = a.part_ml + (size_t)slot * G * 2;
     float* po = a.part_o + (size_t)slot * G * D;
-    for (int idx = threadIdx.x; idx < G * D; idx += kMW * 32) {
-      const int h = idx / D, e = idx % D;
-      float mx = -INFINITY;
+    if constexpr (CL) {
+      // four values per thread, published as soon as merged; this CTA's slice
+      // is kept in place (each thread rewrites only its own values)
+      for (int idx = 4 * threadIdx.x; idx < G * D; idx += 4 * kMW * 32) {
+        const int h = idx / D, e = idx % D;
+        float mx = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < kMW; ++w) mx = fmaxf(mx, sm.m[w][h]);
-      float l = 0.f, acc = 0.f;
+        for (int w = 0; w < kMW; ++w) mx = fmaxf(mx, sm.m[w][h]);
+        float l = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int w = 0; w < kMW; ++w) {
-        const float wt = (mx == -INFINITY) ? 0.f : exp2f(sm.m[w][h] - mx);
-        l += sm.l[w][h] * wt;
-        acc += sm.o[w][h][e] * wt;
+        for (int w = 0; w < kMW; ++w) {
+          const float wt = (mx == -INFINITY) ? 0.f : exp2f(sm.m[w][h] - mx);
+          l += sm.l[w][h] * wt;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) acc[q] += sm.o[w][h][e + q] * wt;
+        }
+        publish(idx, acc, mx, l);
       }
-      if (CL) {  // this CTA's state, in place (each thread rewrites only its own (h, e))
-        sm.o[0][h][e] = acc;
-        if (e == 0) { pub_ml[h][0] = mx; pub_ml[h][1] = l; }
-      } else {
+    } else {
+      for (int idx = threadIdx.x; idx < G * D; idx += kMW * 32) {
+        const int h = idx / D, e = idx % D;
+        float mx = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kMW; ++w) mx = fmaxf(mx, sm.m[w][h]);
+        float l = 0.f, acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < kMW; ++w) {
+          const float wt = (mx == -INFINITY) ? 0.f : exp2f(sm.m[w][h] - mx);
+          l += sm.l[w][h] * wt;
+          acc += sm.o[w][h][e] * wt;
+        }
         po[idx] = acc;
         if (e == 0) {
           pml[h * 2] = mx;
@@ -843,87 +885,56 @@ __global__ void __launch_bounds__(kThreadsM, PS_DMMA_CTAS_PER_SM)
         }
       }
     }
+    // the merged state in shared memory before it is read (next piece's
+    // merge; cluster mode: this CTA's slice and (max, sum) in the combine)
     if (!csync(&sync_b, np)) { stopped = true; break; }
     ++np;
   }
 
   if (CL && !stopped && !abort_flag) {
     // ---- cluster: combine the pair's csize states into its output ----
-    if (np == 0) {  // no tiles in this CTA's share: an empty state
-      for (int idx = threadIdx.x; idx < G * D; idx += kMW * 32) {
-        const int h = idx / D, e = idx % D;
-        sm.o[0][h][e] = 0.f;
-        if (e == 0) { pub_ml[h][0] = -INFINITY; pub_ml[h][1] = 0.f; }
-      }
-      if (!csync(&sync_c, 0)) stopped = true;
-    }
-    const int rank = (int)ptx::cluster_ctarank(), C = a.csize;
-    const int SL = G * D / C;  // outputs per slice
-    if (!stopped) {
-      // push: every peer gets this CTA's (max, sum) and the values of its
-      // slice, as asynchronous stores that complete their bytes on the peer's
-      // pub_bar (no fence, no separate arrival).  D and SL are multiples of
-      // 4, so four consecutive values stay inside one row and one slice and go
-      // in one store.
-      for (int idx = 4 * threadIdx.x; idx < G * D; idx += 4 * kMW * 32) {
-        const int r = idx / SL;
-        if (r != rank) {
-          const int h = idx / D, e = idx % D;
-          ptx::st_async_v4_f32(ptx::map_to_rank(&rcv_o[rank * SL + (idx - r * SL)], r),
-                               sm.o[0][h][e], sm.o[0][h][e + 1], sm.o[0][h][e + 2],
-                               sm.o[0][h][e + 3], ptx::map_to_rank(&pub_bar, r));
-        }
-      }
-      for (int idx = threadIdx.x; idx < C * G * 2; idx += kMW * 32) {
-        const int r = idx / (G * 2), h = (idx / 2) % G, w = idx & 1;
-        if (r != rank)
-          ptx::st_async_f32(ptx::map_to_rank(&rcv_ml[rank][h][w], r), pub_ml[h][w],
-                            ptx::map_to_rank(&pub_bar, r));
-      }
+    if (np == 0) {  // no tiles in this CTA's share: publish an empty state
+      const float zero[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int idx = 4 * threadIdx.x; idx < G * D; idx += 4 * kMW * 32)
+        publish(idx, zero, -INFINITY, 0.f);
+      if (!csync(&sync_b, 0)) stopped = true;
     }
     if (!stopped) {
-      // the peers' states are here once all C - 1 have arrived
+      // the peers' states are here once all their bytes have landed
       const bool ok = ptx::mbar_wait_cluster_bounded(&pub_bar, 0, &abort_flag, kWaitLimitCycles);
       if (__all_sync(FULL, ok)) {
         const int pair = blockIdx.x / C, b = pair / Hkv, gg = pair % Hkv;
         const int ncols = nq_of(b) << lgq();  // valid columns of the pair
-        // each rank's weight 2^(m_r - M) / L per column, L = sum_r l_r 2^(m_r - M)
-        if (threadIdx.x < ncols) {
-          const int h = threadIdx.x;
-          float mr[kMaxCluster], lr[kMaxCluster];
-          float M = -INFINITY;
+        // this CTA's slice of the outputs: each rank's weight 2^(m_r - M) / L
+        // per column (L = sum_r l_r 2^(m_r - M)), found by every output thread
+        // of the column for itself
+        for (int k = threadIdx.x; k < SL; k += kMW * 32) {
+          const int idx = rank * SL + k, h = idx / D, e = idx % D;
+          if (h < ncols) {
+            float mr[kMaxCluster], lr[kMaxCluster];
+            float M = -INFINITY;
 #pragma unroll
-          for (int r = 0; r < kMaxCluster; ++r) {
-            if (r < C) {
-              mr[r] = r == rank ? pub_ml[h][0] : rcv_ml[r][h][0];
-              lr[r] = r == rank ? pub_ml[h][1] : rcv_ml[r][h][1];
-              M = fmaxf(M, mr[r]);
+            for (int r = 0; r < kMaxCluster; ++r) {
+              if (r < C) {
+                mr[r] = r == rank ? pub_ml[h][0] : rcv_ml[r][h][0];
+                lr[r] = r == rank ? pub_ml[h][1] : rcv_ml[r][h][1];
+                M = fmaxf(M, mr[r]);
+              }
             }
-          }
-          float L = 0.f;
+            float L = 0.f;
 #pragma unroll
-          for (int r = 0; r < kMaxCluster; ++r) {
-            if (r < C) {
-              mr[r] = (mr[r] == -INFINITY) ? 0.f : exp2f(mr[r] - M);
-              L += lr[r] * mr[r];
+            for (int r = 0; r < kMaxCluster; ++r) {
+              if (r < C) {
+                mr[r] = (mr[r] == -INFINITY) ? 0.f : exp2f(mr[r] - M);
+                L += lr[r] * mr[r];
+              }
             }
-          }
-          const float inv = 1.f / L;
+            const float inv = 1.f / L;
+            float A = 0.f;
 #pragma unroll
-          for (int r = 0; r < kMaxCluster; ++r)
-            if (r < C) cw[r][h] = mr[r] * inv;
-        }
-        if (csync(&sync_c, np == 0 ? 1 : 0)) {
-          // this CTA's slice of the outputs
-          for (int k = threadIdx.x; k < SL; k += kMW * 32) {
-            const int idx = rank * SL + k, h = idx / D, e = idx % D;
-            if (h < ncols) {
-              float A = 0.f;
-#pragma unroll
-              for (int r = 0; r < kMaxCluster; ++r)
-                if (r < C) A += (r == rank ? sm.o[0][h][e] : rcv_o[r * SL + k]) * cw[r][h];
-              store_out<uint16_t>((uint16_t*)a.out + qo_off(b, gg, h) + e, A);
-            }
+            for (int r = 0; r < kMaxCluster; ++r)
+              if (r < C) A += (r == rank ? sm.o[0][h][e] : rcv_o[r * SL + k]) * (mr[r] * inv);
+            store_out<uint16_t>((uint16_t*)a.out + qo_off(b, gg, h) + e, A);
           }
         }
       }
