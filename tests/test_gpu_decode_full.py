@@ -67,6 +67,22 @@ def test_ragged_serving_batch():
                      "ragged")
 
 
+@pytest.mark.parametrize("B,Hq,d", [(3, 16, 128), (10, 16, 128), (3, 64, 128), (10, 8, 64)],
+                         ids=["24pairs-G2", "80pairs-G2", "24pairs-G8", "80pairs-G1-d64"])
+def test_cluster_sizes(B, Hq, d):
+    """Few equal pairs run in cluster mode, where each CTA hands its merged
+    state to the peers that own the output slices.  24 (sequence, kv head)
+    pairs take clusters of 8 CTAs, 80 pairs clusters of 2 (the headline
+    decode, 64 pairs, takes 4); G = 8 makes a slice span whole rows of the
+    outputs, d = 64 halves them.  Every output against the float64 oracle."""
+    W, P, t, Hkv = 2048, 64, 3000, 8
+    c = Cache(W, P, Hkv, d, ps_dtype("bf16"), B)
+    sds = [SeqData(11, b, Hq, Hkv, d, "bf16") for b in range(B)]
+    for b, sd in enumerate(sds):
+        setup_seq(c, sd, b, P, t, W, (331 * b) % W)
+    decode_and_check(c, sds, [P] * B, [t] * B, W, Hq, d, "bf16", f"B={B} Hq={Hq} d={d}")
+
+
 def test_batch_larger_than_one_launch():
     """300 sequences (more than one launch's worth of batch entries), fp32 d=64."""
     W, P, Hq, Hkv, d = 8, 2, 4, 2, 64
